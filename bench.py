@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Throughput of the LAPLEX hot path on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sym2p24|small|phased_head|gram_image|sym1e9]
+
+A step is one training pass of the operator on one batch: sort the anchors,
+forward, backward (all gradients), and for N > 1 GPUs the all-reduce of the
+anchor gradient over the data-parallel ranks (each rank owns its own batch of
+vectors; the anchors are shared parameters).  The default workload is the
+symmetric operator at n = 2^24 anchors, U[0, 0.05 n], B = 16 vectors.  Inputs
+are seeded synthetic draws (structured_trainable_laplace_b200.inputs); every
+per-step input is larger than the 126 MB L2, so no flush is needed between steps.
+
+The line carries: value (elements/s = n * B * ranks / step time, train mode with
+the re-sort), infer (cached sort), e2e (the same through host buffers, copies
+included), the dominant kernel's roofline from live CUDA-event timings, clocks
+sampled during the timed region, and the fp64 oracle's CPU time on a bounded
+sample of the same workload.  --impl reference times that oracle alone.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from structured_trainable_laplace_b200 import inputs  # noqa: E402
+
+METRIC = "LAPLEX matvec elements/s (fwd+bwd)"
+UNIT = "elements/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ workloads
+
+def make_workload(name: str, rank: int):
+    """Inputs of the named workload; anchors (parameters) identical on every rank,
+    vectors drawn per rank."""
+    gen = {
+        "sym2p24": lambda s: inputs.sym_2p24_b16(s),
+        "small": lambda s: inputs.sym_small_ties(s),
+        "sym1e9": lambda s: inputs.sym_extreme(s),
+        "phased_head": lambda s: inputs.phased_head_2p22(s),
+        "gram_image": lambda s: inputs.gram_image(s),
+    }[name]
+    w = gen(rank)
+    if rank != 0:
+        w0 = gen(0)
+        for key in ("a", "b", "phi", "psi", "D"):
+            if key in w0:
+                w.arrays[key] = w0[key]
+    return w
+
+
+def elements(w) -> int:
+    """Units of the metric: scanned length x batch (the large side for rectangular ops)."""
+    return w.n * w.B
+
+
+def compulsory_bytes(w) -> int:
+    """Each input read once and each output written once, per step (train mode), in
+    the ABI's layout.  Intermediate sorted anchors and permutations count once as
+    written and once as read by each consumer call."""
+    n, B, k = w.n, w.B, w.k
+    if w.op == "sym":
+        sort = 4 * n + 8 * n
+        fwd = 8 * n + 4 * n * B + 4 * n * B
+        bwd = 8 * n + 8 * n * B + 4 * n * B + 4 * n
+        return sort + fwd + bwd
+    if w.op == "phased_transpose":
+        sort = 12 * n + 12 * k
+        fwd = 12 * n + 4 * n * B + 4 * k * B
+        bwd = 12 * n + 4 * n * B + 4 * k * B + 4 * n * B + 8 * n + 8 * k
+        return sort + fwd + bwd
+    if w.op == "gram":
+        sort = 12 * n + 12 * k
+        fwd = 8 * n + 4 * n * B + 4 * n * B + 4 * k
+        bwd = 8 * n + 4 * n * B + 4 * k
+        return sort + fwd + bwd
+    raise ValueError(w.op)
+
+
+# Algorithmic bytes per element row of each kernel (sorted anchor 4 + permutation 4
+# + the row values it must read or write), used for the roofline of the kernel
+# that dominates the step.  Units per launch: the rows that launch walks.
+def kernel_bytes_per_launch(kernel: str, w) -> float | None:
+    n, B, k = w.n, w.B, w.k
+    if w.op == "sym":
+        table = {
+            "sym_bwd": (8 + 4 * B + 4 * B + 4 * B + 4) * n,   # s, perm, x, g -> gx, ga
+            "sym_left": (8 + 4 * B + 4 * B) * n,             # s, perm, x -> y
+            "sym_right": (8 + 4 * B) * n,                    # s, perm, x (carries only)
+            "radix_pass": (12 * n + 3 * 16 * n) / 4.0,       # pass 0 reads a; passes 1-3 read+write key,value
+            "radix_hist": 4 * n,
+        }
+        return table.get(kernel)
+    if w.op == "phased_transpose":
+        table = {
+            "large_accum": (12 + 4 * B) * n,                 # s, perm, phi, x rows
+            "large_expand_grad": (12 + 4 * B + 4 * B + 8) * n,  # + gx rows, ga, gphi
+            "radix_pass": (12 * n + 3 * 16 * n) / 4.0,
+        }
+        return table.get(kernel)
+    if w.op == "gram":
+        table = {
+            "large_accum": (8 + 4 * B) * n,
+            "large_expand": (8 + 4 * B) * n,
+            "radix_pass": (12 * n + 3 * 16 * n) / 4.0,
+        }
+        return table.get(kernel)
+    return None
+
+
+# ------------------------------------------------------------------ the step
+
+class Step:
+    """Device buffers and one training step of the workload through the binding."""
+
+    def __init__(self, L, w, device, torch):
+        self.L, self.w, self.torch = L, w, torch
+        self.dev = device
+        self.t = {key: torch.from_numpy(np.ascontiguousarray(v)).to(device) for key, v in w.arrays.items()}
+        self.saved = None
+        if w.op == "sym":
+            self.saved = L.saved_buffer("sym", w.n, 1, w.B, device)
+        elif w.op == "phased_transpose":
+            self.saved = L.saved_buffer("phased_transpose", w.n, w.k, w.B, device)
+        self.sorted = None
+
+    def sort(self):
+        L, t = self.L, self.t
+        sa = L.sort_anchors(t["a"])
+        sb = L.sort_anchors(t["b"]) if "b" in t else None
+        self.sorted = (sa, sb)
+
+    def compute(self):
+        """Forward + backward from the current sorted anchors; returns the output tensors."""
+        L, t, w = self.L, self.t, self.w
+        (sa, pa), sb = self.sorted[0], self.sorted[1]
+        if w.op == "sym":
+            y = L.apply_sym(sa, pa, t["x"], saved=self.saved)
+            gr = L.backward("sym", sa, pa, t["x"], t["g"], saved=self.saved, need=("gx", "ga"))
+            return {"y": y, "gx": gr["gx"], "ga": gr["ga"]}
+        if w.op == "phased_transpose":
+            z = L.apply_phased(sa, pa, t["phi"], sb[0], sb[1], t["psi"], t["x"], transpose=True, saved=self.saved)
+            gr = L.backward("phased_transpose", sa, pa, t["x"], t["h"], b_sorted=sb[0], perm_b=sb[1], phi=t["phi"],
+                            psi=t["psi"], saved=self.saved)
+            return {"z": z, **gr}
+        if w.op == "gram":
+            y, gD = L.gram_apply(sa, pa, sb[0], sb[1], t["D"], t["v"], g=t["g"])
+            return {"y": y, "gD": gD}
+        raise ValueError(w.op)
+
+    def anchor_grads(self, out):
+        return [out[key] for key in ("ga", "gb", "gphi", "gpsi", "gD") if key in out]
+
+
+def sample_clocks(stop_path: str, out_path: str):
+    q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    try:
+        return subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "200"],
+                                stdout=open(out_path, "w"), stderr=subprocess.DEVNULL)
+    except (OSError, FileNotFoundError):
+        return None
+
+
+def summarize_clocks(path: str, gpu_index: int) -> dict:
+    sm, smax, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    try:
+        for line in open(path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or not f[0].isdigit() or int(f[0]) != gpu_index:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+    except OSError:
+        pass
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "structured_trainable_laplace_b200", "csrc", "*"))):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources (a line `traffic <kernel> <workload> <bytes> <source hash>`)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = source_hash()
+    for line in open(path):
+        f = line.split()
+        if len(f) == 5 and f[0] == "traffic" and f[1] == kernel and f[2] == workload and f[4] == cur:
+            return float(f[3])
+    return None
+
+
+def measured_peak():
+    try:
+        j = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(j["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_sample(w, budget_s: float):
+    """Run the fp64 oracle (sort + forward + backward) on a prefix-sized draw of the
+    same workload, growing the sample until it takes about budget_s.  Returns
+    (elements/s, description)."""
+    import oracle
+    n_s = 1 << 14
+    while True:
+        t0 = time.perf_counter()
+        if w.op == "sym":
+            ws = inputs.symmetric(n_s, w.B, seed=123, spacing=0.05)
+            oracle.sym_apply(ws["a"], ws["x"])
+            oracle.sym_backward(ws["a"], ws["x"], ws["g"])
+            units = n_s * w.B
+        elif w.op == "phased_transpose":
+            ws = inputs.phased_head(n_s, w.k, w.B, seed=123)
+            oracle.rect_apply(ws["a"], ws["b"], ws["x"], ws["phi"], ws["psi"], transpose=True)
+            oracle.rect_backward(ws["a"], ws["b"], ws["x"], ws["h"], ws["phi"], ws["psi"], transpose=True)
+            units = n_s * w.B
+        else:
+            k_s = max(1, int(round(w.k * n_s / w.n)))
+            ws = inputs.gram(n_s, k_s, w.B, seed=123)
+            oracle.gram_apply(ws["a"], ws["b"], ws["D"], ws["v"])
+            oracle.gram_backward_D(ws["a"], ws["b"], ws["v"], ws["g"])
+            units = n_s * w.B
+        dt = time.perf_counter() - t0
+        if dt >= budget_s or n_s >= w.n:
+            return units / dt, f"{w.op} n={n_s} (same recipe, seed 123), sort+fwd+bwd in fp64, {dt:.2f} s"
+        n_s = min(w.n, n_s * max(2, int(budget_s / max(dt, 1e-3))))
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="sym2p24",
+                    choices=["sym2p24", "small", "phased_head", "gram_image", "sym1e9"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return reference_arm(args, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    from structured_trainable_laplace_b200 import laplex as L
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    L.lib()  # fails loudly if the library is missing
+
+    w = make_workload(args.workload, rank)
+    st = Step(L, w, device, torch)
+    stream = torch.cuda.current_stream(device)
+
+    def train_step():
+        st.sort()
+        out = st.compute()
+        if world > 1:
+            for gtensor in st.anchor_grads(out):
+                dist.all_reduce(gtensor)
+        return out
+
+    def infer_step():
+        out = st.compute()
+        if world > 1:
+            for gtensor in st.anchor_grads(out):
+                dist.all_reduce(gtensor)
+        return out
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def timed(fn, steps):
+        barrier()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        ms = e0.elapsed_time(e1) / steps
+        if world > 1:
+            tt = torch.tensor([ms], device=device)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ms = float(tt.item())
+        return ms
+
+    for _ in range(args.warmup):
+        train_step()
+    L.check()
+
+    # headline: train mode (re-sort every step), clocks sampled meanwhile
+    clk_path = os.path.join("/tmp", f"laplex_clocks_{os.getpid()}.csv")
+    proc = sample_clocks(None, clk_path)
+    time.sleep(0.3)
+    ms_train = timed(train_step, args.steps)
+    time.sleep(0.2)
+    if proc is not None:
+        proc.terminate()
+        proc.wait()
+    clocks = summarize_clocks(clk_path, local)
+    L.check()
+
+    # inference mode: cached sort
+    st.sort()
+    ms_infer = timed(infer_step, args.steps)
+
+    # the same train steps with every kernel bracketed by CUDA events
+    L.profile_enable(True)
+    ms_prof = timed(train_step, args.steps)
+    prof = L.profile_report()
+    L.profile_enable(False)
+    L.check()
+
+    # end to end through host buffers: pinned host inputs -> device, step, outputs -> host
+    host_in = {key: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for key, v in w.arrays.items()}
+    outs = train_step()
+    host_out = {key: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for key, v in outs.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+
+    def e2e_step():
+        for key, v in host_in.items():
+            st.t[key].copy_(v, non_blocking=True)
+        out = train_step()
+        for key, v in out.items():
+            host_out[key].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    ms_e2e = timed(e2e_step, max(2, args.steps // 2))
+    peak_mem = torch.cuda.max_memory_allocated(device) / 1e9
+
+    units = elements(w) * world
+    value = units / (ms_train * 1e-3)
+    peak_gbs, peak_kind = measured_peak()
+    comp = compulsory_bytes(w)
+
+    # dominant kernel of the step and its roofline
+    dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
+    roof = None
+    launches_total = sum(v[0] for v in prof.values()) if prof else 0
+    if dom is not None:
+        name, (cnt, tot_ms) = dom
+        avg_ms = tot_ms / cnt
+        bpl = kernel_bytes_per_launch(name, w)
+        if bpl is not None:
+            achieved = bpl / (avg_ms * 1e-3) / 1e9
+            traffic = recorded_traffic(name, args.workload)
+            roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak_gbs,
+                    "unit": "GB/s", "frac": round(achieved / peak_gbs, 4), "traffic": traffic,
+                    "algorithmic_bytes_per_launch": bpl, "avg_launch_ms": round(avg_ms, 5),
+                    "peak_source": peak_kind}
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_train, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; anchors shared, vectors per rank)",
+        "config": {"workload": args.workload, "op": w.op, "n": w.n, "k": w.k, "B": w.B, "mode": "train (re-sort)",
+                   "l2": "per-step inputs > 126 MB L2, no flush", "parallelism": f"dp{world}" if world > 1 else "1 GPU"},
+        "infer": {"value": round(units / (ms_infer * 1e-3), 1), "ms_per_step": round(ms_infer, 4)},
+        "hbm": {"compulsory_bytes_per_step": comp, "achieved_gbs": round(comp / (ms_train * 1e-3) / 1e9, 1),
+                "frac_of_measured": round(comp / (ms_train * 1e-3) / 1e9 / peak_gbs, 4),
+                "frac_of_8tbs": round(comp / (ms_train * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4)},
+        "e2e": {"value": round(units / (ms_e2e * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
+        "roofline": roof,
+        "kernels": {kname: {"launches_per_step": v[0] / args.steps, "ms_per_step": round(v[1] / args.steps, 5)}
+                    for kname, v in sorted(prof.items(), key=lambda kv: -kv[1][1])},
+        "profiled_ms_per_step": round(ms_prof, 4),
+        "gpu_launches": int(launches_total),
+        "clocks": clocks,
+        "peak_mem_gb": round(peak_mem, 2),
+    }
+    if rank == 0 and world == 1:
+        v, desc = oracle_sample(w, args.cpu_budget)
+        result["cpu_baseline"] = {"value": round(v, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                                  "cpu": cpu_model()}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def reference_arm(args, world, rank):
+    """The fp64 oracle, as it stands, on the host cores; rank 0 only."""
+    if rank != 0:
+        return
+    w = make_workload(args.workload, 0)
+    per_step = []
+    desc = ""
+    for _ in range(args.warmup):
+        oracle_sample(w, min(2.0, args.cpu_budget / 4))
+    for _ in range(args.steps):
+        v, desc = oracle_sample(w, min(4.0, args.cpu_budget / 2))
+        per_step.append(v)
+    v = float(np.median(per_step))
+    units = elements(w)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(units / v * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "op": w.op, "n": w.n, "k": w.k, "B": w.B},
+        "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                         "cpu": cpu_model()},
+        "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * laplex.h -- C ABI of the B200 (sm_100a) LAPLEX operator library, liblaplex.so.
+ *
+ * LAPLEX ("LAPLEX: The FFT of Learnable Laplace Kernels", Struski, Blazhko,
+ * Kubaty, Tabor) is the dense matrix
+ *
+ *     E(a, b)_ij = exp(-|a_i - b_j|)                         (technical summary, section 2.1)
+ *     E(a, phi; b, psi)_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j)   (section 2.1, phased form)
+ *
+ * defined by learnable 1-D anchors a (n), b (k) and optional phases phi (n),
+ * psi (k).  This library applies it, its transpose, its gradients and the
+ * weighted Gram operator A diag(D) A^T (section 2.2, "Gram operators") to
+ * vectors without ever forming the matrix: the anchors are sorted once, after
+ * which every product is a pair of linear-recurrence scans (prefix and suffix)
+ * over the sorted order (section 2.2, "Exact scan algebra").  The results are
+ * exact in exact arithmetic; in fp32 every output o satisfies
+ * |o - o_exact| <= 1e-5 * twin(o) + 1e-30, where twin(o) is the same expression
+ * evaluated with every input replaced by its absolute value.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Pointers.   Every array pointer is a DEVICE pointer to caller-owned memory.
+ *             The library allocates nothing and frees nothing.  Inputs are
+ *             read-only; outputs must not overlap any input or each other
+ *             (LAPLEX_ERR_ARG if they do).  Every pointer must be 16-byte
+ *             aligned (LAPLEX_ERR_ALIGN).
+ * Layout.     Vectors are feature-major, row-major [rows][B] fp32, rows
+ *             contiguous (row i holds the B batch values of feature i, the
+ *             leading dimension is B).  B = 1 is a plain vector.
+ * Order.      x, y, g, gradients and phases are in ORIGINAL index order.  Anchors
+ *             are passed SORTED together with their permutation, exactly as
+ *             laplex_sort_anchors returns them: a_sorted[r] = a[perm[r]],
+ *             ascending, ties by ascending original index.  A sort can be reused
+ *             while the anchors do not change.
+ * Sizes.      1 <= n, k <= LAPLEX_MAX_N; 1 <= B <= LAPLEX_MAX_B.
+ * Workspace.  Scratch memory is passed as (ws, ws_bytes); query the size with
+ *             the matching *_workspace_size function (LAPLEX_ERR_WORKSPACE if
+ *             too small).  It holds nothing between calls.
+ * Saved.      Forward calls may fill an optional caller buffer `saved` (size from
+ *             laplex_saved_size) that the matching laplex_backward call reads,
+ *             so that the backward does not recompute the forward's scans.
+ *             NULL means "do not save" (forward) / "recompute" (backward).  Its
+ *             contents are opaque and only valid for the same sorted anchors.
+ * Streams.    Every call enqueues its work on `stream` (a cudaStream_t; NULL is
+ *             the legacy default stream) and returns without synchronising.
+ * Errors.     Argument errors are returned at once, before anything is launched.
+ *             Errors found by the kernels (non-finite anchors, a lookback wait
+ *             that exceeded its bound) are written to the optional device word
+ *             *d_status (first error wins; the caller zeroes it); read it with
+ *             laplex_read_status.  After any error the outputs are unspecified.
+ *             A failed launch returns LAPLEX_ERR_CUDA.
+ */
+#ifndef LAPLEX_H
+#define LAPLEX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (same underlying type). */
+typedef struct CUstream_st* laplex_stream_t;
+
+#define LAPLEX_MAX_N 4294967295LL /* 2^32 - 1: permutations are uint32 */
+#define LAPLEX_MAX_B 1024
+
+typedef enum laplex_status {
+    LAPLEX_OK = 0,
+    LAPLEX_ERR_ARG = 1,       /* bad size, NULL pointer, overlap, bad op */
+    LAPLEX_ERR_ALIGN = 2,     /* a pointer is not 16-byte aligned */
+    LAPLEX_ERR_WORKSPACE = 3, /* ws_bytes smaller than the *_workspace_size answer */
+    LAPLEX_ERR_NONFINITE = 4, /* an anchor (or phase) is NaN or infinite (device word) */
+    LAPLEX_ERR_TIMEOUT = 5,   /* a bounded lookback wait gave up (device word) */
+    LAPLEX_ERR_CUDA = 6       /* a CUDA launch or runtime call failed */
+} laplex_status;
+
+/* Operator selector for laplex_workspace_size, laplex_saved_size, laplex_backward. */
+typedef enum laplex_op {
+    LAPLEX_OP_SYM = 0,              /* y = K x, K = E(a, a)                      x [n][B] -> y [n][B] */
+    LAPLEX_OP_GENERAL = 1,          /* y = E(a, b) x                             x [k][B] -> y [n][B] */
+    LAPLEX_OP_TRANSPOSE = 2,        /* z = E(a, b)^T x                           x [n][B] -> z [k][B] */
+    LAPLEX_OP_PHASED = 3,           /* y = E(a, phi; b, psi) x                   x [k][B] -> y [n][B] */
+    LAPLEX_OP_PHASED_TRANSPOSE = 4, /* z = E(a, phi; b, psi)^T x                 x [n][B] -> z [k][B] */
+    LAPLEX_OP_GRAM = 5              /* y = A diag(D) A^T v, A = E(a, b)          v [n][B] -> y [n][B] */
+} laplex_op;
+
+/* Human-readable name of a status code (static string). */
+const char* laplex_status_string(laplex_status s);
+
+/* Synchronise `stream`, then copy *d_status to *h_status and return it as a
+ * laplex_status (LAPLEX_ERR_CUDA if the copy fails). */
+laplex_status laplex_read_status(const int32_t* d_status, laplex_stream_t stream, int32_t* h_status);
+
+/* ------------------------------------------------------------------ sort */
+
+/* Bytes of workspace laplex_sort_anchors needs for n anchors. */
+size_t laplex_sort_workspace_size(int64_t n);
+
+/* Sort the anchors (technical summary, section 2.2: "after sorting the anchors").
+ *   a         [n] fp32, original order (read only).
+ *   a_sorted  [n] fp32 out: the anchors ascending; -0.0 is returned as +0.0.
+ *   perm      [n] uint32 out: a_sorted[r] == a[perm[r]]; equal anchors keep
+ *             ascending original index, so perm is unique (stable sort).
+ * A least-significant-digit radix sort of an order-preserving uint32 key
+ * (4 passes of 8 bits).  NaN or infinite anchors set LAPLEX_ERR_NONFINITE. */
+laplex_status laplex_sort_anchors(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws,
+                                  size_t ws_bytes, int32_t* d_status, laplex_stream_t stream);
+
+/* ------------------------------------------------------------ operators */
+
+/* Bytes of workspace for the forward and the backward of `op` (the larger of
+ * the two).  k is ignored for LAPLEX_OP_SYM. */
+size_t laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t B);
+
+/* Bytes of the optional `saved` buffer that forwards of `op` fill. */
+size_t laplex_saved_size(laplex_op op, int64_t n, int64_t k, int64_t B);
+
+/* Symmetric operator (section 2.2, "symmetric case a = b"): y = K x with
+ * K_ij = exp(-|a_i - a_j|), computed as the prefix scan P_r = x_r + exp(a_(r-1) - a_(r)) P_(r-1)
+ * plus the mirrored suffix scan S_r, minus the diagonal counted twice:
+ * y = P + S - x, in sorted order, scattered back through perm.
+ *   a_sorted, perm [n]: from laplex_sort_anchors.   x [n][B] in, y [n][B] out. */
+laplex_status laplex_apply_sym(const float* a_sorted, const uint32_t* perm, int64_t n, const float* x, int64_t B,
+                               float* y, void* saved, void* ws, size_t ws_bytes, int32_t* d_status,
+                               laplex_stream_t stream);
+
+/* General rectangular operator (section 2.2, "general case a != b"): y = E x,
+ * E_ij = exp(-|a_i - b_j|), x [k][B] at the b anchors, y [n][B] at the a anchors.
+ * The inputs are scanned over sorted b and every a reads the state of its
+ * neighbours in the merged order. */
+laplex_status laplex_apply_general(const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* b_sorted,
+                                   const uint32_t* perm_b, int64_t k, const float* x, int64_t B, float* y,
+                                   void* saved, void* ws, size_t ws_bytes, int32_t* d_status,
+                                   laplex_stream_t stream);
+
+/* Transposed rectangular operator: z = E^T x, x [n][B] at a, z [k][B] at b.  The
+ * inputs are summed into the intervals of sorted b (strict-left sums u, strict-
+ * right sums v, ties t), then propagated across the intervals by the scan. */
+laplex_status laplex_apply_transpose(const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* b_sorted,
+                                     const uint32_t* perm_b, int64_t k, const float* x, int64_t B, float* z,
+                                     void* saved, void* ws, size_t ws_bytes, int32_t* d_status,
+                                     laplex_stream_t stream);
+
+/* Phased operator (section 2.1): E_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j),
+ * evaluated as the cos/sin split cos phi_i cos psi_j + sin phi_i sin psi_j (two
+ * scan channels per input channel).  phi [n], psi [k] in original order.
+ * transpose = 0: x [k][B] -> out [n][B];  transpose = 1: x [n][B] -> out [k][B]. */
+laplex_status laplex_apply_phased(const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* phi,
+                                  const float* b_sorted, const uint32_t* perm_b, int64_t k, const float* psi,
+                                  int transpose, const float* x, int64_t B, float* out, void* saved, void* ws,
+                                  size_t ws_bytes, int32_t* d_status, laplex_stream_t stream);
+
+/* Backward pass of any operator above (the anchors are trainable: abstract and
+ * section 2.3, "differentiability with respect to the anchors").  Given the
+ * forward's input x and the upstream gradient g (shape of the forward's output),
+ * writes the gradients of <g, out>:
+ *   gx   (shape of x)  = E^T g (the adjoint product),
+ *   ga [n], gb [k]     anchor gradients from sign-split sums: for an output row i,
+ *                      sum over the columns to its right minus the columns to
+ *                      its left, d|t|/dt = sign(t) with sign(0) = 0 (tied anchors
+ *                      contribute nothing),
+ *   gphi [n], gpsi [k] phase gradients (phased ops only).
+ * Any output pointer may be NULL to skip it; for LAPLEX_OP_SYM gb, gphi, gpsi,
+ * b_sorted, perm_b, psi and phi are ignored (ga holds the whole anchor gradient).
+ * `saved` is the buffer the matching forward filled, or NULL.
+ * LAPLEX_OP_GRAM is not accepted here: use laplex_gram_apply. */
+laplex_status laplex_backward(laplex_op op, const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* phi,
+                              const float* b_sorted, const uint32_t* perm_b, int64_t k, const float* psi,
+                              const float* x, const float* g, int64_t B, const void* saved, float* gx, float* ga,
+                              float* gb, float* gphi, float* gpsi, void* ws, size_t ws_bytes, int32_t* d_status,
+                              laplex_stream_t stream);
+
+/* Weighted Gram operator (section 2.2, "Gram operators": M = A diag(D) A^T):
+ * y = A diag(D) A^T v with A_ij = exp(-|a_i - b_j|), v, y [n][B], D [k], as two
+ * rectangular scan passes (w = A^T v at b, then y = A (D w) at a).
+ *   w_saved [k][B] (nullable): receives w = A^T v.
+ *   g [n][B], gD [k] (both NULL or both set): also the gradient of <g, y> with
+ *   respect to D, gD_j = sum_c (A^T g)_jc (A^T v)_jc. */
+laplex_status laplex_gram_apply(const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* b_sorted,
+                                const uint32_t* perm_b, int64_t k, const float* D, const float* v, int64_t B,
+                                float* y, float* w_saved, const float* g, float* gD, void* ws, size_t ws_bytes,
+                                int32_t* d_status, laplex_stream_t stream);
+
+/* ------------------------------------------------------------- tracing */
+
+/* Per-kernel timing aid (no counterpart on the pages; a measurement tool).
+ * laplex_profile_enable(1) clears the record and starts bracketing every kernel
+ * the library launches with a pair of CUDA events recorded on the launch
+ * stream; laplex_profile_enable(0) stops.  Adds one event pair per launch. */
+void laplex_profile_enable(int on);
+
+/* Synchronise on the recorded events and write, for up to max_kernels kernel
+ * names, the name (NUL-terminated, at most name_len bytes, into names +
+ * i * name_len), the number of launches and the summed device time in ms.
+ * Clears the record.  Returns the number of distinct kernel names, or -1 if an
+ * event query failed.  Any output pointer may be NULL. */
+int laplex_profile_report(int max_kernels, char* names, int name_len, int* launches, double* total_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAPLEX_H */

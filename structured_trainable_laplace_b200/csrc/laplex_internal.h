@@ -1,0 +1,71 @@
+// Internal launchers behind the C ABI (include/laplex.h).  All pointers are
+// device pointers; all launches go to `stream`; nothing synchronises.
+#pragma once
+
+#include <algorithm>
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace laplex {
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// profile.cu: optional CUDA-event bracket around each kernel launch.
+bool profiling();
+void* profile_begin(const char* name, cudaStream_t stream);
+void profile_end(void* token, cudaStream_t stream);
+struct ProfScope {
+    void* token;
+    cudaStream_t stream;
+    ProfScope(const char* name, cudaStream_t st) : token(profile_begin(name, st)), stream(st) {}
+    ~ProfScope() { profile_end(token, stream); }
+};
+#define LAPLEX_TIMED(name, stream, ...)        \
+    do {                                       \
+        ::laplex::ProfScope ps_(name, stream); \
+        __VA_ARGS__;                           \
+    } while (0)
+
+// sort.cu
+size_t sort_workspace_bytes(int64_t n);
+cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
+                        cudaStream_t stream);
+
+// sym.cu
+size_t sym_workspace_bytes(int64_t n, int64_t B);
+size_t sym_saved_bytes(int64_t n, int64_t B);
+cudaError_t launch_sym_forward(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B, float* y,
+                               void* saved, void* ws, int32_t* status, cudaStream_t stream);
+cudaError_t launch_sym_backward(const float* s, const uint32_t* perm, int64_t n, const float* x, const float* g,
+                                int64_t B, const void* saved, float* gx, float* ga, void* ws, int32_t* status,
+                                cudaStream_t stream);
+
+// rect.cu: rectangular operators in canonical form.  The "output side" O and the
+// "input side" I are each a sorted anchor set with its permutation and optional
+// phases (original order).
+struct Side {
+    const float* s;        // sorted anchors
+    const uint32_t* perm;  // s[r] = anchors[perm[r]]
+    const float* theta;    // phases in original order, or nullptr
+    int64_t m;             // number of anchors
+};
+
+size_t rect_workspace_bytes(int64_t n_out, int64_t n_in, int64_t B, bool phased);
+size_t rect_saved_bytes(int64_t n_out, int64_t n_in, int64_t B, bool phased);
+// out[O] = E(O, I) x[I], x [n_in][B], out [n_out][B].
+cudaError_t launch_rect_forward(Side O, Side I, const float* x, int64_t B, float* out, void* saved, void* ws,
+                                int32_t* status, cudaStream_t stream);
+// Gradients of <g, out> for launch_rect_forward (g at O):
+//   gx [n_in][B], gO/gI anchor gradients, gtO/gtI phase gradients (each nullable).
+cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g, int64_t B, const void* saved,
+                                 float* gx, float* gO, float* gI, float* gtO, float* gtI, void* ws, int32_t* status,
+                                 cudaStream_t stream);
+
+size_t gram_workspace_bytes(int64_t n, int64_t k, int64_t B);
+cudaError_t launch_gram(Side A, Side Bs, const float* D, const float* v, int64_t B, float* y, float* w_saved,
+                        const float* g, float* gD, void* ws, int32_t* status, cudaStream_t stream);
+
+}  // namespace laplex

@@ -1,0 +1,270 @@
+// Stable key-index radix sort of fp32 anchors ("LAPLEX: The FFT of Learnable
+// Laplace Kernels", technical summary section 2.2: the scan algebra starts by
+// sorting the anchors).
+//
+// Keys are the order-preserving uint32 images of the anchors (-0 folded onto
+// +0), values the original indices.  Least-significant digit first, 4 passes of
+// 8 bits.  Each pass is one kernel over tiles of 4096 keys claimed in order from
+// an atomic counter: the tile ranks its keys stably inside each warp (match-any
+// over the digit), publishes its per-digit counts, looks back over the tiles
+// before it for their per-digit prefixes (bounded waits), and scatters through
+// shared memory so that runs of equal digits leave as contiguous stores.
+// A histogram kernel computes the four global digit histograms in one read of
+// the anchors and flags non-finite anchors.
+#include "laplex_internal.h"
+
+namespace laplex {
+
+namespace {
+
+constexpr int kNT = 256;
+constexpr int kItems = 16;
+constexpr int kTile = kNT * kItems;
+constexpr int kNW = kNT / 32;
+constexpr int kRadix = 256;
+constexpr unsigned long long kValMask = (1ull << 62) - 1;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Exclusive scan of one value per thread over a 256-thread block.  Returns the
+// exclusive prefix; *total receives the sum.
+__device__ __forceinline__ uint32_t block_excl_scan_256(uint32_t v, uint32_t* s_warp, uint32_t* total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        uint32_t o = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += o;
+    }
+    if (lane == 31) s_warp[w] = inc;
+    __syncthreads();
+    uint32_t base = 0, tot = 0;
+#pragma unroll
+    for (int j = 0; j < kNW; ++j) {
+        uint32_t x = s_warp[j];
+        if (j < w) base += x;
+        tot += x;
+    }
+    __syncthreads();
+    *total = tot;
+    return base + inc - v;
+}
+
+__global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a, int64_t n, uint32_t* hist,
+                                                    unsigned long long* look0, int64_t look_words, int32_t* status) {
+    __shared__ uint32_t s_hist[4][kRadix];
+    for (int i = threadIdx.x; i < 4 * kRadix; i += kNT) (&s_hist[0][0])[i] = 0;
+    __syncthreads();
+    const int64_t stride = (int64_t)gridDim.x * kNT;
+    // zero the first pass's lookback region
+    for (int64_t i = (int64_t)blockIdx.x * kNT + threadIdx.x; i < look_words; i += stride) look0[i] = 0ull;
+    bool bad = false;
+    const int64_t nround = (n + 31) / 32 * 32;  // whole warps stay converged for match_any
+    for (int64_t i = (int64_t)blockIdx.x * kNT + threadIdx.x; i - threadIdx.x % 32 < nround; i += stride) {
+        const bool valid = i < n;
+        const uint32_t vm = __ballot_sync(0xffffffffu, valid);
+        if (valid) {
+            const float f = __ldg(a + i);
+            bad |= is_nonfinite(f);
+            const uint32_t key = float_to_key(f);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const uint32_t d = (key >> (8 * p)) & 0xffu;
+                const uint32_t peers = __match_any_sync(vm, d);
+                if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[p][d], __popc(peers));
+            }
+        }
+    }
+    if (bad) raise_status(status, kStatusNonFinite);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 4 * kRadix; i += kNT) {
+        const uint32_t v = (&s_hist[0][0])[i];
+        if (v) atomicAdd(hist + i, v);
+    }
+}
+
+// One LSD pass.  MODE 0: keys from the fp32 anchors, values = indices.
+// MODE 1: keys/values from the previous pass.  MODE 2: like 1, and the keys
+// leave as fp32 anchors (last pass).
+template <int MODE>
+__global__ void __launch_bounds__(kNT) k_radix_pass(const float* __restrict__ a, const uint32_t* __restrict__ keys_in,
+                                                    const uint32_t* __restrict__ vals_in, uint32_t* __restrict__ keys_out,
+                                                    uint32_t* __restrict__ vals_out, int64_t n, int shift,
+                                                    const uint32_t* __restrict__ hist, uint32_t* counter,
+                                                    unsigned long long* look, unsigned long long* look_next,
+                                                    int32_t* status) {
+    __shared__ uint32_t s_whist[kNW][kRadix];
+    __shared__ uint32_t s_keys[kTile];
+    __shared__ uint32_t s_vals[kTile];
+    __shared__ uint32_t s_base[kRadix];   // global destination of the tile's first key per digit
+    __shared__ uint32_t s_start[kRadix];  // tile-local start of each digit
+    __shared__ uint32_t s_scan[kNW];
+    __shared__ int64_t s_tile;
+
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    if (tid == 0) s_tile = atomicAdd(counter, 1u);
+    for (int i = tid; i < kNW * kRadix; i += kNT) (&s_whist[0][0])[i] = 0;
+    __syncthreads();
+    const int64_t tile = s_tile;
+    const int64_t base = tile * kTile;
+    look_next[tile * kRadix + tid] = 0ull;  // the pass after next reuses this region
+
+    // global exclusive digit offsets for this pass
+    uint32_t gtot;
+    const uint32_t gexcl = block_excl_scan_256(__ldg(hist + tid), s_scan, &gtot);
+
+    uint32_t key[kItems], val[kItems], rank[kItems];
+    const int64_t wbase = base + (int64_t)w * 32 * kItems;
+#pragma unroll
+    for (int i = 0; i < kItems; ++i) {
+        const int64_t idx = wbase + i * 32 + lane;
+        if (idx < n) {
+            if (MODE == 0) {
+                key[i] = float_to_key(__ldg(a + idx));
+                val[i] = (uint32_t)idx;
+            } else {
+                key[i] = __ldg(keys_in + idx);
+                val[i] = __ldg(vals_in + idx);
+            }
+        } else {
+            key[i] = 0xffffffffu;
+            val[i] = 0u;
+        }
+    }
+    // stable rank inside the warp, items in (i, lane) order = index order
+#pragma unroll
+    for (int i = 0; i < kItems; ++i) {
+        const int64_t idx = wbase + i * 32 + lane;
+        const bool valid = idx < n;
+        const uint32_t vm = __ballot_sync(0xffffffffu, valid);
+        uint32_t peers = 0, d = 0, before = 0;
+        if (valid) {
+            d = (key[i] >> shift) & 0xffu;
+            peers = __match_any_sync(vm, d);
+            before = s_whist[w][d];
+            rank[i] = before + __popc(peers & lanemask_lt());
+        }
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) s_whist[w][d] = before + __popc(peers);
+        __syncwarp();
+    }
+    __syncthreads();
+    // per-digit: warp offsets and tile count (thread tid handles digit tid)
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int j = 0; j < kNW; ++j) {
+        const uint32_t c = s_whist[j][tid];
+        s_whist[j][tid] = cnt;
+        cnt += c;
+    }
+    // decoupled lookback over earlier tiles for digit tid
+    {
+        unsigned long long* mine = look + tile * kRadix + tid;
+        if (tile == 0) {
+            st_release_u64(mine, (2ull << 62) | cnt);
+        } else {
+            st_release_u64(mine, (1ull << 62) | cnt);
+        }
+        unsigned long long excl = 0;
+        if (tile > 0) {
+            int64_t j = tile - 1;
+            while (true) {
+                unsigned long long v;
+                uint32_t spins = 0;
+                while (((v = ld_acquire_u64(look + j * kRadix + tid)) >> 62) == 0) {
+                    if (++spins > kSpinLimit) {
+                        raise_status(status, kStatusTimeout);
+                        v = 2ull << 62;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+                excl += v & kValMask;
+                if ((v >> 62) == 2) break;
+                --j;
+            }
+            st_release_u64(mine, (2ull << 62) | (excl + cnt));
+        }
+        s_base[tid] = gexcl + (uint32_t)excl;
+    }
+    uint32_t ttot;
+    s_start[tid] = block_excl_scan_256(cnt, s_scan, &ttot);
+    __syncthreads();
+    // place keys in shared memory in (digit, rank) order
+#pragma unroll
+    for (int i = 0; i < kItems; ++i) {
+        const int64_t idx = wbase + i * 32 + lane;
+        if (idx < n) {
+            const uint32_t d = (key[i] >> shift) & 0xffu;
+            const uint32_t p = s_start[d] + s_whist[w][d] + rank[i];
+            s_keys[p] = key[i];
+            s_vals[p] = val[i];
+        }
+    }
+    __syncthreads();
+    const int valid_count = (n - base) < kTile ? (int)(n - base) : kTile;
+    for (int p = tid; p < valid_count; p += kNT) {
+        const uint32_t k = s_keys[p];
+        const uint32_t d = (k >> shift) & 0xffu;
+        const uint32_t dst = s_base[d] + (uint32_t)(p - s_start[d]);
+        if ((int64_t)dst < n) {  // always true for consistent counts; a bad count never writes out of range
+            keys_out[dst] = (MODE == 2) ? __float_as_uint(key_to_float(k)) : k;
+            vals_out[dst] = s_vals[p];
+        }
+    }
+}
+
+}  // namespace
+
+size_t sort_workspace_bytes(int64_t n) {
+    const int64_t T = (n + kTile - 1) / kTile;
+    size_t b = 0;
+    b += align_up((size_t)n * 4, 256);            // keys_alt
+    b += align_up((size_t)n * 4, 256);            // vals_alt
+    b += align_up(4 * kRadix * 4 + 64, 256);      // hist + counters
+    b += 2 * align_up((size_t)T * kRadix * 8, 256);  // two lookback regions
+    return b;
+}
+
+cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
+                        cudaStream_t stream) {
+    const int64_t T = (n + kTile - 1) / kTile;
+    char* p = (char*)ws;
+    uint32_t* keys_alt = (uint32_t*)p;
+    p += align_up((size_t)n * 4, 256);
+    uint32_t* vals_alt = (uint32_t*)p;
+    p += align_up((size_t)n * 4, 256);
+    uint32_t* hist = (uint32_t*)p;
+    uint32_t* counters = hist + 4 * kRadix;
+    p += align_up(4 * kRadix * 4 + 64, 256);
+    unsigned long long* look[2];
+    look[0] = (unsigned long long*)p;
+    p += align_up((size_t)T * kRadix * 8, 256);
+    look[1] = (unsigned long long*)p;
+
+    cudaError_t e = cudaMemsetAsync(hist, 0, 4 * kRadix * 4 + 64, stream);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (n + kNT * 8 - 1) / (kNT * 8);
+    const int hblocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
+    LAPLEX_TIMED("radix_hist", stream, k_radix_hist<<<hblocks, kNT, 0, stream>>>(a, n, hist, look[0], T * kRadix, status));
+    uint32_t* ka = (uint32_t*)a_sorted;
+    // pass 0: a -> alt; pass 1: alt -> out; pass 2: out -> alt; pass 3: alt -> out
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<0><<<(unsigned)T, kNT, 0, stream>>>(a, nullptr, nullptr, keys_alt, vals_alt, n, 0, hist + 0 * kRadix,
+                                                     counters + 0, look[0], look[1], status));
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, 8, hist + 1 * kRadix,
+                                                     counters + 1, look[1], look[0], status));
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, ka, perm, keys_alt, vals_alt, n, 16, hist + 2 * kRadix,
+                                                     counters + 2, look[0], look[1], status));
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<2><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, 24, hist + 3 * kRadix,
+                                                     counters + 3, look[1], look[0], status));
+    return cudaGetLastError();
+}
+
+}  // namespace laplex
