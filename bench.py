@@ -162,9 +162,6 @@ class Step:
             return {"y": y, "gD": gD}
         raise ValueError(w.op)
 
-    def anchor_grads(self, out):
-        return [out[key] for key in ("ga", "gb", "gphi", "gpsi", "gD") if key in out]
-
 
 def sample_clocks(stop_path: str, out_path: str):
     q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -295,7 +292,7 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from structured_trainable_laplace_b200 import laplex as L
+    from structured_trainable_laplace_b200 import dp, laplex as L
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
@@ -310,18 +307,10 @@ def main():
 
     def train_step():
         st.sort()
-        out = st.compute()
-        if world > 1:
-            for gtensor in st.anchor_grads(out):
-                dist.all_reduce(gtensor)
-        return out
+        return dp.allreduce_param_grads(st.compute())
 
     def infer_step():
-        out = st.compute()
-        if world > 1:
-            for gtensor in st.anchor_grads(out):
-                dist.all_reduce(gtensor)
-        return out
+        return dp.allreduce_param_grads(st.compute())
 
     def barrier():
         if world > 1:

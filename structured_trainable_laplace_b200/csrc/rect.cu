@@ -432,9 +432,12 @@ __global__ void __launch_bounds__(256) k_large(LargePass A) {
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) {
                     const float val = w[p] * h[v];
-                    if (!tie) fu[p][v] = fmaf(eR, val, fu[p][v]);
-                    fv[p][v] = fmaf(eL, val, fv[p][v]);
-                    if (tie && cval) {
+                    // A row tied with a run of small-side anchors enters that run only
+                    // (TL, TR); the neighbours beyond it receive it through the scan.
+                    if (!tie) {
+                        fu[p][v] = fmaf(eR, val, fu[p][v]);
+                        fv[p][v] = fmaf(eL, val, fv[p][v]);
+                    } else if (cval) {
                         atomicAdd(A.TL + m * Cb + p * B + c0 + v, (double)val);
                         atomicAdd(A.TR + (mp - 1) * Cb + p * B + c0 + v, (double)val);
                     }
