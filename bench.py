@@ -44,11 +44,12 @@ FALLBACK_HBM_GBS = 6650.0
 
 # ------------------------------------------------------------------ workloads
 
-def make_workload(name: str, rank: int):
+def make_workload(name: str, rank: int, n: int | None = None):
     """Inputs of the named workload; anchors (parameters) identical on every rank,
-    vectors drawn per rank."""
+    vectors drawn per rank.  n overrides the symmetric workload's size (same recipe:
+    a ~ U[0, 0.05 n], B = 16), for profiling captures of a smaller case."""
     gen = {
-        "sym2p24": lambda s: inputs.sym_2p24_b16(s),
+        "sym2p24": lambda s: inputs.sym_2p24_b16(s, n=n or (1 << 24)),
         "small": lambda s: inputs.sym_small_ties(s),
         "sym1e9": lambda s: inputs.sym_extreme(s),
         "phased_head": lambda s: inputs.phased_head_2p22(s),
@@ -280,6 +281,7 @@ def main():
     ap.add_argument("--workload", default="sym2p24",
                     choices=["sym2p24", "small", "phased_head", "gram_image", "sym1e9"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
+    ap.add_argument("--n", type=int, default=None, help="anchors of the symmetric workload (profiling captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -301,7 +303,7 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
     L.lib()  # fails loudly if the library is missing
 
-    w = make_workload(args.workload, rank)
+    w = make_workload(args.workload, rank, args.n)
     st = Step(L, w, device, torch)
     stream = torch.cuda.current_stream(device)
 
@@ -434,7 +436,7 @@ def reference_arm(args, world, rank):
     """The fp64 oracle, as it stands, on the host cores; rank 0 only."""
     if rank != 0:
         return
-    w = make_workload(args.workload, 0)
+    w = make_workload(args.workload, 0, args.n)
     per_step = []
     desc = ""
     for _ in range(args.warmup):
