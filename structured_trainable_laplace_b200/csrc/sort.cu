@@ -56,33 +56,38 @@ __device__ __forceinline__ uint32_t block_excl_scan_256(uint32_t v, uint32_t* s_
 
 __global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a, int64_t n, uint32_t* hist,
                                                     unsigned long long* look0, int64_t look_words, int32_t* status) {
-    __shared__ uint32_t s_hist[4][kRadix];
-    for (int i = threadIdx.x; i < 4 * kRadix; i += kNT) (&s_hist[0][0])[i] = 0;
+    __shared__ uint32_t s_hist[kNW][4][kRadix];  // one histogram set per warp: fewer colliding atomics
+    for (int i = threadIdx.x; i < kNW * 4 * kRadix; i += kNT) (&s_hist[0][0][0])[i] = 0;
     __syncthreads();
     const int64_t stride = (int64_t)gridDim.x * kNT;
     // zero the first pass's lookback region
     for (int64_t i = (int64_t)blockIdx.x * kNT + threadIdx.x; i < look_words; i += stride) look0[i] = 0ull;
+    uint32_t(*wh)[kRadix] = s_hist[threadIdx.x >> 5];
     bool bad = false;
-    const int64_t nround = (n + 31) / 32 * 32;  // whole warps stay converged for match_any
-    for (int64_t i = (int64_t)blockIdx.x * kNT + threadIdx.x; i - threadIdx.x % 32 < nround; i += stride) {
-        const bool valid = i < n;
-        const uint32_t vm = __ballot_sync(0xffffffffu, valid);
-        if (valid) {
-            const float f = __ldg(a + i);
-            bad |= is_nonfinite(f);
-            const uint32_t key = float_to_key(f);
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const uint32_t d = (key >> (8 * p)) & 0xffu;
-                const uint32_t peers = __match_any_sync(vm, d);
-                if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&s_hist[p][d], __popc(peers));
-            }
-        }
+    auto add = [&](float f) {
+        bad |= is_nonfinite(f);
+        const uint32_t key = float_to_key(f);
+        atomicAdd(&wh[0][key & 0xffu], 1u);
+        atomicAdd(&wh[1][(key >> 8) & 0xffu], 1u);
+        atomicAdd(&wh[2][(key >> 16) & 0xffu], 1u);
+        atomicAdd(&wh[3][key >> 24], 1u);
+    };
+    const int64_t n4 = n / 4;  // the anchors are 16-byte aligned (ABI)
+    const float4* a4 = reinterpret_cast<const float4*>(a);
+    for (int64_t i = (int64_t)blockIdx.x * kNT + threadIdx.x; i < n4; i += stride) {
+        const float4 v = __ldg(a4 + i);
+        add(v.x);
+        add(v.y);
+        add(v.z);
+        add(v.w);
     }
+    for (int64_t i = n4 * 4 + (int64_t)blockIdx.x * kNT + threadIdx.x; i < n; i += stride) add(__ldg(a + i));
     if (bad) raise_status(status, kStatusNonFinite);
     __syncthreads();
     for (int i = threadIdx.x; i < 4 * kRadix; i += kNT) {
-        const uint32_t v = (&s_hist[0][0])[i];
+        uint32_t v = 0;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) v += (&s_hist[w][0][0])[i];
         if (v) atomicAdd(hist + i, v);
     }
 }
@@ -171,21 +176,33 @@ __global__ void __launch_bounds__(kNT) k_radix_pass(const float* __restrict__ a,
         }
         unsigned long long excl = 0;
         if (tile > 0) {
+            // read a window of kWin predecessors per round trip, newest first, and add
+            // their counts until one holds an inclusive prefix (tile 0 always does)
+            constexpr int kWin = 16;
             int64_t j = tile - 1;
-            while (true) {
-                unsigned long long v;
-                uint32_t spins = 0;
-                while (((v = ld_acquire_u64(look + j * kRadix + tid)) >> 62) == 0) {
-                    if (++spins > kSpinLimit) {
-                        raise_status(status, kStatusTimeout);
-                        v = 2ull << 62;
-                        break;
+            bool done = false;
+            while (!done) {
+                unsigned long long v[kWin];
+#pragma unroll
+                for (int q = 0; q < kWin; ++q) v[q] = (j - q >= 0) ? ld_relaxed_u64(look + (j - q) * kRadix + tid) : (2ull << 62);
+#pragma unroll
+                for (int q = 0; q < kWin; ++q) {
+                    if (done) break;
+                    unsigned long long vv = v[q];
+                    uint32_t spins = 0;
+                    while ((vv >> 62) == 0) {  // not yet published: poll this one (bounded)
+                        if (++spins > kSpinLimit) {
+                            raise_status(status, kStatusTimeout);
+                            vv = 2ull << 62;
+                            break;
+                        }
+                        __nanosleep(32);
+                        vv = ld_relaxed_u64(look + (j - q) * kRadix + tid);
                     }
-                    __nanosleep(32);
+                    excl += vv & kValMask;
+                    done = (vv >> 62) == 2;
                 }
-                excl += v & kValMask;
-                if ((v >> 62) == 2) break;
-                --j;
+                j -= kWin;
             }
             st_release_u64(mine, (2ull << 62) | (excl + cnt));
         }

@@ -7,13 +7,13 @@
 // Both directions of the scan are needed at every row, and the vectors do not
 // fit on chip, so each product reads its input twice.  The two reads are made
 // free of inter-tile waits by partitioning the sorted rows into P contiguous
-// ranges of tiles, one persistent CTA per (range, channel group):
-//   k_sym_agg    walks its range right to left and writes, per tile, the fp64
-//                suffix state of the range from that tile's first row on (RS),
-//                and the range's aggregates in both directions;
+// base ranges of tiles:
+//   k_sym_agg    walks its ranges right to left and writes, per tile, the fp64
+//                suffix state of the base range from that tile's first row on
+//                (RS), and each base range's aggregates in both directions;
 //   k_sym_carry  scans the P range aggregates (one CTA per channel group) into
-//                the fp64 carries entering each range from the left and right;
-//   k_sym_sweep  walks its range left to right, folding the left state tile by
+//                the fp64 carries entering each base range from the left/right;
+//   k_sym_sweep  walks its ranges left to right, folding the left state tile by
 //                tile and taking the right state from RS and the range carry,
 //                evaluates both directions inside each tile and writes
 //                y = P + S - x through the permutation (forward), or, over x and
@@ -21,9 +21,17 @@
 //                ga = sum_c g (R_x - L_x) + x (R_g - L_g) from the strict sums
 //                (ties excluded: sign(0) = 0); x's RS and carries come from the
 //                forward (the `saved` buffer) or are recomputed.
-// Every tile is staged with cp.async: anchors and permutation two tiles ahead,
-// the gathered rows one tile ahead, so the gathers of the next tile overlap the
-// arithmetic of the current one.  No kernel waits on another CTA.
+// Each persistent CTA walks m consecutive base ranges, m chosen per kernel so
+// that its grid is one full wave at that kernel's occupancy.
+//
+// Inside a CTA each warp owns whole channels of the tile: lane (cs, k) holds the
+// k-th segment of E rows of one channel, so the in-tile scan is a shuffle scan
+// over the lanes of that channel and the fp64 range fold runs in the channel's
+// first lane.  The only block barriers are the one that publishes a staged tile
+// and the one before the coalesced output stores.  Tiles are staged with
+// cp.async: the gathered rows AHEAD tiles ahead, anchors, permutation and
+// carries one tile further; per-row decays and the fp64 decays of the tile folds
+// are computed one tile ahead.  No kernel waits on another CTA.
 #include "laplex_internal.h"
 #include "pipeline.cuh"
 
@@ -31,12 +39,23 @@ namespace laplex {
 
 namespace {
 
-constexpr int kNT = 256;
-constexpr int kMaxRanges = 1024;  // per channel group
-constexpr int kRangesPerSM = 3;
+constexpr int kE = 16;
+constexpr int kMaxRanges = 8192;   // base ranges per channel group
+constexpr int kRangesPerSM = 12;   // base ranges per SM (divisible by the usual occupancies)
+constexpr int kAheadFwd = 2;       // gathered-row prefetch distance: aggregate and forward sweeps
+constexpr int kAheadBwd = 1;       // backward sweep (two staged vectors)
 
 template <int C>
-using SymGeo = TileGeo<C, kNT, (C == 1 ? 8 : 16)>;
+struct SymGeo {
+    static constexpr int NW = C < 8 ? C : 8;  // warps per CTA
+    static constexpr int NT = NW * 32;
+    static constexpr int CW = C / NW;  // channels per warp
+    static constexpr int SK = 32 / CW;  // segments per channel = lanes per channel group
+    using G = TileGeo<C, NT, kE, CW>;
+    static constexpr int R = G::R;  // rows per tile (SK * E)
+};
+
+inline int64_t rows_per_tile(int C) { return C <= 8 ? 32 * kE : (32 * kE * 8) / C; }
 
 struct SymScan {
     const float* s;
@@ -44,95 +63,163 @@ struct SymScan {
     int64_t n;
     int B;
     int64_t T;    // tiles per channel group
-    int P;        // ranges per channel group
-    int64_t tpr;  // tiles per range
+    int P;        // base ranges per channel group
+    int64_t tpr;  // tiles per base range
+    int m;        // base ranges walked by one CTA
 };
 
-// fp64 scan state of one vector, per channel group, range j, tile t and channel c
+// fp64 scan state of one vector, per channel group, base range J, tile t, channel c
 struct RangeState {
-    double2* RS;    // [G][T][C]  right state from tile t's first row to the range's end
+    double2* RS;    // [G][T][C]  right state from tile t's first row to its base range's end
     double2* Lagg;  // [G][P][C]  range aggregate, left direction (anchored at its last row)
     double2* Ragg;  // [G][P][C]  range aggregate, right direction (anchored at -its first row)
     double2* Lin;   // [G][P][C]  carry from the ranges before (anchored at the row before)
     double2* Rin;   // [G][P][C]  carry from the ranges after (anchored at -the row after)
 };
 
-template <int C, int NV>
+template <int C, int NV, int AHEAD>
 struct SymSmem {
-    using G = SymGeo<C>;
-    float s[3][G::SS];
-    uint32_t p[3][G::R];
-    float v[NV][2][G::XS];
-    float dl[G::R + 4];
-    ScanSmem<C, kNT / 32> sc[2 * NV];
-    double2 carry[2 * NV][C];
-    int has[2 * NV];
+    using G = typename SymGeo<C>::G;
+    static constexpr int MS = AHEAD + 2;  // anchor / permutation / carry slots
+    static constexpr int VS = AHEAD + 1;  // gathered-row slots
+    float s[MS][G::SS];
+    uint32_t p[MS][G::R];
+    double2 rs[MS][NV][C];   // RS[t+1] (sweep)
+    double2 rin[MS][NV][C];  // carry entering the tile's base range from the right (sweep)
+    float v[NV][VS][G::XS];
+    float dl[2][G::R + 4];  // per-row decays of the current and the next tile
+    double ed[2][2];        // fp64 decays of the two tile-level folds, current and next tile
 };
 
 __device__ __forceinline__ int64_t tile_lo(int64_t t, int R) { return t * (int64_t)R; }
 
-// ------------------------------------------------------------------ pass A
+__device__ __forceinline__ double2 to_d2(LP v) { return make_double2((double)v.L, (double)v.P); }
 
-template <int C>
-__global__ void __launch_bounds__(kNT, 3) k_sym_agg(SymScan a, const float* __restrict__ v, RangeState st) {
-    using G = SymGeo<C>;
-    constexpr int E = G::E, R = G::R;
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    SymSmem<C, 1>& sm = *reinterpret_cast<SymSmem<C, 1>*>(smem_raw);
-    const int grp = blockIdx.y, j = blockIdx.x;
-    const int64_t tb = (int64_t)j * a.tpr, te = min(a.T, tb + a.tpr);
-    const int nt = (int)(te - tb);
-    const int c = threadIdx.x % C, k = threadIdx.x / C, ch0 = grp * C;
-    // walk t = te-1, te-2, ..., tb
-    stage_meta<G>(a.s, a.perm, a.n, tile_lo(te - 1, R), sm.s[0], sm.p[0]);
-    cp_async_commit();
-    if (nt > 1) stage_meta<G>(a.s, a.perm, a.n, tile_lo(te - 2, R), sm.s[1], sm.p[1]);
-    cp_async_commit();
-    cp_async_wait_all();
-    __syncthreads();
-    stage_rows<G>(v, a.B, ch0, a.n, tile_lo(te - 1, R), sm.p[0], sm.v[0][0]);
-    cp_async_commit();
-    double2 runR = make_double2(0.0, 0.0), runL = make_double2(0.0, 0.0);
-    float uRunR = 0.f, uRunL = 0.f;
-    for (int i = 0; i < nt; ++i) {
-        const int64_t t = te - 1 - i;
-        cp_async_wait_all();
-        __syncthreads();
-        if (i + 1 < nt) stage_rows<G>(v, a.B, ch0, a.n, tile_lo(t - 1, R), sm.p[(i + 1) % 3], sm.v[0][(i + 1) & 1]);
-        cp_async_commit();
-        if (i + 2 < nt) stage_meta<G>(a.s, a.perm, a.n, tile_lo(t - 2, R), sm.s[(i + 2) % 3], sm.p[(i + 2) % 3]);
-        cp_async_commit();
-        const float* sb = sm.s[i % 3];
-        const float* xb = sm.v[0][i & 1] + k * G::SEG + c;
-        tile_decays<G>(sb, sm.dl);
-        __syncthreads();
-        LP str = {0.f, 0.f}, stl = {0.f, 0.f};
+__device__ __forceinline__ LP shfl_lp(LP v, int src, int width) {
+    LP o;
+    o.L = __shfl_sync(0xffffffffu, v.L, src, width);
+    o.P = __shfl_sync(0xffffffffu, v.P, src, width);
+    return o;
+}
+
+// Inclusive scans over the SK segments of one channel (the SK lanes of a group),
+// both directions, NV vectors.  sb: staged anchors; k: this lane's segment.
+template <int SK, int NV>
+__device__ __forceinline__ void group_scan(LP (&incL)[NV], LP (&incR)[NV], const float* sb, int k) {
 #pragma unroll
-        for (int e = E - 1; e >= 0; --e) str = lp_step_d(str, sm.dl[k * E + e + 1], 0.f, xb[e * C]);
+    for (int off = 1; off < SK; off <<= 1) {
+        const float uL = sb[4 + k * kE + kE - 1], uLo = sb[4 + max(k - off, 0) * kE + kE - 1];
+        const float uR = -sb[4 + k * kE], uRo = -sb[4 + min(k + off, SK - 1) * kE];
+        const float eL = expf(uLo - uL), eR = expf(uRo - uR);
 #pragma unroll
-        for (int e = 0; e < E; ++e) stl = lp_step_d(stl, sm.dl[k * E + e], 0.f, xb[e * C]);
-        LP ex;
-        bool hx;
-        block_scan_dir<C, kNT, true>(str, -sb[4 + k * E], -sb[4 + k * E + E], sm.sc[0], ex, hx);
-        block_scan_dir<C, kNT, false>(stl, sb[4 + k * E + E - 1], sb[4 + k * E - 1], sm.sc[1], ex, hx);
-        if (threadIdx.x < C) {
-            const LP tr = sm.sc[0].tot[c], tl = sm.sc[1].tot[c];
-            const double2 trd = make_double2(tr.L, tr.P), tld = make_double2(tl.L, tl.P);
-            const float u_first = -sb[4], u_last = sb[4 + R - 1];
-            runR = (i == 0) ? trd : lpd_combine(runR, uRunR, trd, u_first);
-            uRunR = u_first;
-            st.RS[((int64_t)grp * a.T + t) * C + c] = runR;
-            if (i == 0) {
-                runL = tld;
-                uRunL = u_last;
-            } else {
-                runL = lpd_combine(tld, u_last, runL, uRunL);
-            }
+        for (int v = 0; v < NV; ++v) {
+            LP oL, oR;
+            oL.L = __shfl_up_sync(0xffffffffu, incL[v].L, off, SK);
+            oL.P = __shfl_up_sync(0xffffffffu, incL[v].P, off, SK);
+            oR.L = __shfl_down_sync(0xffffffffu, incR[v].L, off, SK);
+            oR.P = __shfl_down_sync(0xffffffffu, incR[v].P, off, SK);
+            if (k >= off) incL[v] = combine_e(oL, incL[v], eL, uL > uLo);
+            if (k + off < SK) incR[v] = combine_e(oR, incR[v], eR, uR > uRo);
         }
     }
-    if (threadIdx.x < C) {
-        st.Lagg[((int64_t)grp * a.P + j) * C + c] = runL;
-        st.Ragg[((int64_t)grp * a.P + j) * C + c] = runR;
+}
+
+// Tiles walked by CTA blockIdx.x: those of base ranges [J0, J1).
+struct CtaTiles {
+    int J0, J1;
+    int64_t tb, te;
+};
+
+__device__ __forceinline__ CtaTiles cta_tiles(const SymScan& a) {
+    CtaTiles w;
+    w.J0 = blockIdx.x * a.m;
+    w.J1 = min(a.P, w.J0 + a.m);
+    w.tb = (int64_t)w.J0 * a.tpr;
+    w.te = min(a.T, (int64_t)w.J1 * a.tpr);
+    return w;
+}
+
+// ------------------------------------------------------------------ pass A
+
+// Walks tiles te-1 .. tb.  Per tile: the right total extends the running suffix of
+// its base range (RS[t]), the left total is prepended to the range's running left
+// aggregate; both restart at each base range's last tile and are written out at
+// its first.
+template <int C, int AHEAD>
+__global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
+    k_sym_agg(SymScan a, const float* __restrict__ v, RangeState st) {
+    using SG = SymGeo<C>;
+    using G = typename SG::G;
+    using SM = SymSmem<C, 1, AHEAD>;
+    constexpr int E = kE, R = G::R, SK = SG::SK, CW = SG::CW, MS = SM::MS, VS = SM::VS;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    SM& sm = *reinterpret_cast<SM*>(smem_raw);
+    const int grp = blockIdx.y;
+    const CtaTiles w = cta_tiles(a);
+    const int nt = (int)(w.te - w.tb);
+    const int lane = threadIdx.x & 31, cs = lane / SK, k = lane % SK;
+    const int c = (threadIdx.x >> 5) * CW + cs, ch0 = grp * C;
+    auto tile_of = [&](int i) { return w.te - 1 - i; };
+    // anchor of the last row of base range J
+    auto range_end = [&](int64_t J) { return __ldg(a.s + min(a.n, (J + 1) * a.tpr * (int64_t)R) - 1); };
+    auto tile_ed = [&](const float* sb, int64_t t, double* ed) {  // [0] right fold, [1] left fold
+        ed[0] = exp((double)sb[4] - (double)sb[4 + R]);
+        ed[1] = exp((double)sb[4 + R - 1] - (double)range_end(t / a.tpr));
+    };
+#pragma unroll
+    for (int q = 0; q <= AHEAD; ++q) {
+        if (q < nt) stage_meta<G>(a.s, a.perm, a.n, tile_lo(tile_of(q), R), sm.s[q % MS], sm.p[q % MS]);
+        cp_async_commit();
+    }
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < AHEAD; ++q) {
+        if (q < nt) stage_rows<G>(v, a.B, ch0, a.n, tile_lo(tile_of(q), R), sm.p[q % MS], sm.v[0][q % VS]);
+        cp_async_commit();
+    }
+    tile_decays<G>(sm.s[0], sm.dl[0]);
+    if (threadIdx.x == 0) tile_ed(sm.s[0], tile_of(0), sm.ed[0]);
+    double2 runR = make_double2(0.0, 0.0), runL = make_double2(0.0, 0.0);
+    for (int i = 0; i < nt; ++i) {
+        const int64_t t = tile_of(i);
+        const int64_t J = t / a.tpr;
+        cp_async_wait<AHEAD - 1>();  // this tile's rows and the next tiles' anchors are in
+        __syncthreads();
+        if (i + AHEAD + 1 < nt)
+            stage_meta<G>(a.s, a.perm, a.n, tile_lo(tile_of(i + AHEAD + 1), R), sm.s[(i + AHEAD + 1) % MS],
+                          sm.p[(i + AHEAD + 1) % MS]);
+        cp_async_commit();
+        if (i + AHEAD < nt)
+            stage_rows<G>(v, a.B, ch0, a.n, tile_lo(tile_of(i + AHEAD), R), sm.p[(i + AHEAD) % MS],
+                          sm.v[0][(i + AHEAD) % VS]);
+        cp_async_commit();
+        if (i + 1 < nt) {
+            tile_decays<G>(sm.s[(i + 1) % MS], sm.dl[(i + 1) & 1]);
+            if (threadIdx.x == 0) tile_ed(sm.s[(i + 1) % MS], tile_of(i + 1), sm.ed[(i + 1) & 1]);
+        }
+        const float* sb = sm.s[i % MS];
+        const float* dl = sm.dl[i & 1];
+        const float* xb = sm.v[0][i % VS] + k * G::SEG + c;
+        LP sr[1] = {{0.f, 0.f}}, sl[1] = {{0.f, 0.f}};
+#pragma unroll
+        for (int e = E - 1; e >= 0; --e) sr[0] = lp_step_d(sr[0], dl[k * E + e + 1], 0.f, xb[e * C]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) sl[0] = lp_step_d(sl[0], dl[k * E + e], 0.f, xb[e * C]);
+        group_scan<SK, 1>(sl, sr, sb, k);
+        const LP tl = shfl_lp(sl[0], SK - 1, SK);  // tile totals: left at the last segment, right at the first
+        if (k == 0) {
+            const double* ed = sm.ed[i & 1];
+            const bool last_of_range = (t + 1 == min(a.T, (J + 1) * a.tpr));  // the first one walked
+            const double2 trd = to_d2(sr[0]), tld = to_d2(tl);
+            runR = last_of_range ? trd : combine_ed(runR, trd, ed[0], sb[4] < sb[4 + R]);
+            st.RS[((int64_t)grp * a.T + t) * C + c] = runR;
+            runL = last_of_range ? tld : combine_ed(tld, runL, ed[1], range_end(J) > sb[4 + R - 1]);
+            if (t == J * a.tpr) {  // first tile of the base range: its aggregates are complete
+                st.Lagg[((int64_t)grp * a.P + J) * C + c] = runL;
+                st.Ragg[((int64_t)grp * a.P + J) * C + c] = runR;
+            }
+        }
     }
 }
 
@@ -142,8 +229,8 @@ __global__ void __launch_bounds__(kNT, 3) k_sym_agg(SymScan a, const float* __re
 // ranges; the blocks are then composed serially (at most QS steps) and re-walked
 // to produce the carry entering every range.
 template <int C>
-__global__ void __launch_bounds__(kNT) k_sym_carry(SymScan a, RangeState st) {
-    constexpr int QS = (kNT / C) < 16 ? (kNT / C) : 16;
+__global__ void __launch_bounds__(256) k_sym_carry(SymScan a, RangeState st) {
+    constexpr int QS = (256 / C) < 16 ? (256 / C) : 16;
     __shared__ double2 segL[QS][C], segR[QS][C];
     const int grp = blockIdx.x;
     const int c = threadIdx.x % C, q = threadIdx.x / C;
@@ -199,134 +286,170 @@ __global__ void __launch_bounds__(kNT) k_sym_carry(SymScan a, RangeState st) {
 
 // ------------------------------------------------------------------ pass C
 
-// NV = 1: forward (x -> y = out).  NV = 2: backward (x, g -> gx = out, ga).
+// Start copying, for tile t, RS[t+1] (if t+1 is in the same base range) and the
+// right carry of t's base range, for each vector.
 template <int C, int NV>
-__global__ void __launch_bounds__(kNT, (NV == 1 ? 3 : 2)) k_sym_sweep(SymScan a, const float* __restrict__ x, const float* __restrict__ g,
-                                                   RangeState sx, RangeState sg, float* __restrict__ out,
-                                                   float* __restrict__ ga, int ga_atomic) {
-    using G = SymGeo<C>;
-    constexpr int E = G::E, R = G::R;
+__device__ __forceinline__ void stage_carries(const SymScan& a, const RangeState* const* rs, int grp, int64_t t,
+                                              double2 (*rs_dst)[C], double2 (*rin_dst)[C]) {
+    const int64_t J = t / a.tpr;
+    const bool more = t + 1 < min(a.T, (J + 1) * a.tpr);
+    const bool hasRin = J + 1 < a.P;
+    for (int i = threadIdx.x; i < NV * C; i += SymGeo<C>::NT) {
+        const int w = i / C, c = i % C;
+        if (more) cp_async16(&rs_dst[w][c], rs[w]->RS + ((int64_t)grp * a.T + t + 1) * C + c);
+        if (hasRin) cp_async16(&rin_dst[w][c], rs[w]->Rin + ((int64_t)grp * a.P + J) * C + c);
+    }
+}
+
+// NV = 1: forward (x -> y = out).  NV = 2: backward (x, g -> gx = out, ga).
+template <int C, int NV, int AHEAD>
+__global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 1 ? 3 : 2) : 1)) k_sym_sweep(
+    SymScan a, const float* __restrict__ x, const float* __restrict__ g, RangeState sx, RangeState sg,
+    float* __restrict__ out, float* __restrict__ ga, int ga_atomic) {
+    using SG = SymGeo<C>;
+    using G = typename SG::G;
+    using SM = SymSmem<C, NV, AHEAD>;
+    constexpr int E = kE, R = G::R, SK = SG::SK, CW = SG::CW, NT = SG::NT, MS = SM::MS, VS = SM::VS;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    SymSmem<C, NV>& sm = *reinterpret_cast<SymSmem<C, NV>*>(smem_raw);
-    const int grp = blockIdx.y, j = blockIdx.x;
-    const int64_t tb = (int64_t)j * a.tpr, te = min(a.T, tb + a.tpr);
-    const int nt = (int)(te - tb);
-    const int c = threadIdx.x % C, k = threadIdx.x / C, ch0 = grp * C;
-    const int ch = ch0 + c;
-    const bool cval = ch < a.B;
+    SM& sm = *reinterpret_cast<SM*>(smem_raw);
+    const int grp = blockIdx.y;
+    const CtaTiles cw = cta_tiles(a);
+    const int nt = (int)(cw.te - cw.tb);
+    const int lane = threadIdx.x & 31, cs = lane / SK, k = lane % SK;
+    const int c = (threadIdx.x >> 5) * CW + cs, ch0 = grp * C;
     const float* src[2] = {x, g};
     const RangeState* rs[2] = {&sx, &sg};
-
-    stage_meta<G>(a.s, a.perm, a.n, tile_lo(tb, R), sm.s[0], sm.p[0]);
-    cp_async_commit();
-    if (nt > 1) stage_meta<G>(a.s, a.perm, a.n, tile_lo(tb + 1, R), sm.s[1], sm.p[1]);
-    cp_async_commit();
+    // oriented anchor of the row after base range J (where its right carry is anchored)
+    auto u_rin = [&](int64_t J) { return -__ldg(a.s + min(a.n - 1, (J + 1) * a.tpr * (int64_t)R)); };
+    auto tile_ed = [&](const float* sb, int64_t t, double* ed) {  // [0] left fold, [1] right carry
+        ed[0] = exp((double)sb[3] - (double)sb[4 + R - 1]);
+        ed[1] = exp((double)u_rin(t / a.tpr) + (double)sb[4 + R]);
+    };
+#pragma unroll
+    for (int q = 0; q <= AHEAD; ++q) {
+        if (q < nt) {
+            stage_meta<G>(a.s, a.perm, a.n, tile_lo(cw.tb + q, R), sm.s[q % MS], sm.p[q % MS]);
+            stage_carries<C, NV>(a, rs, grp, cw.tb + q, sm.rs[q % MS], sm.rin[q % MS]);
+        }
+        cp_async_commit();
+    }
     cp_async_wait_all();
     __syncthreads();
 #pragma unroll
-    for (int w = 0; w < NV; ++w) stage_rows<G>(src[w], a.B, ch0, a.n, tile_lo(tb, R), sm.p[0], sm.v[w][0]);
-    cp_async_commit();
-
-    // the left folds start from the carries entering the range
-    double2 runL[NV], rin[NV];
-    bool hasL = (j > 0);
-    const bool hasRin = (j + 1 < a.P);
-    const int64_t rng = ((int64_t)grp * a.P + j) * C + c;
-#pragma unroll
-    for (int w = 0; w < NV; ++w) {
-        runL[w] = (hasL && threadIdx.x < C) ? rs[w]->Lin[rng] : make_double2(0.0, 0.0);
-        rin[w] = (hasRin && threadIdx.x < C) ? rs[w]->Rin[rng] : make_double2(0.0, 0.0);
-    }
-    const float uRin = hasRin ? -__ldg(a.s + min(a.n - 1, te * (int64_t)R)) : 0.f;
-
-    for (int i = 0; i < nt; ++i) {
-        const int64_t t = tb + i, lo = tile_lo(t, R);
-        cp_async_wait_all();
-        __syncthreads();
-        if (i + 1 < nt) {
+    for (int q = 0; q < AHEAD; ++q) {
+        if (q < nt) {
 #pragma unroll
             for (int w = 0; w < NV; ++w)
-                stage_rows<G>(src[w], a.B, ch0, a.n, tile_lo(t + 1, R), sm.p[(i + 1) % 3], sm.v[w][(i + 1) & 1]);
+                stage_rows<G>(src[w], a.B, ch0, a.n, tile_lo(cw.tb + q, R), sm.p[q % MS], sm.v[w][q % VS]);
         }
         cp_async_commit();
-        if (i + 2 < nt) stage_meta<G>(a.s, a.perm, a.n, tile_lo(t + 2, R), sm.s[(i + 2) % 3], sm.p[(i + 2) % 3]);
-        cp_async_commit();
-        const float* sb = sm.s[i % 3];
-        const uint32_t* pb = sm.p[i % 3];
-        tile_decays<G>(sb, sm.dl);
+    }
+    tile_decays<G>(sm.s[0], sm.dl[0]);
+    if (threadIdx.x == 0) tile_ed(sm.s[0], cw.tb, sm.ed[0]);
+
+    // fp64 left folds of channel c, kept by the channel's first lane (k == 0)
+    double2 runL[NV];
+    bool hasL = (cw.J0 > 0);
+    const int64_t rng = ((int64_t)grp * a.P + cw.J0) * C + c;
+#pragma unroll
+    for (int w = 0; w < NV; ++w) runL[w] = hasL ? rs[w]->Lin[rng] : make_double2(0.0, 0.0);
+
+    for (int i = 0; i < nt; ++i) {
+        const int64_t t = cw.tb + i, lo = tile_lo(t, R);
+        const int64_t J = t / a.tpr;
+        cp_async_wait<AHEAD - 1>();
         __syncthreads();
-        const float ub_r = -sb[4 + k * E + E], ub_l = sb[4 + k * E - 1];
-        LP exR[NV], exL[NV];
-        bool hR[NV], hL[NV];
+        if (i + AHEAD + 1 < nt) {
+            stage_meta<G>(a.s, a.perm, a.n, tile_lo(t + AHEAD + 1, R), sm.s[(i + AHEAD + 1) % MS],
+                          sm.p[(i + AHEAD + 1) % MS]);
+            stage_carries<C, NV>(a, rs, grp, t + AHEAD + 1, sm.rs[(i + AHEAD + 1) % MS], sm.rin[(i + AHEAD + 1) % MS]);
+        }
+        cp_async_commit();
+        if (i + AHEAD < nt) {
+#pragma unroll
+            for (int w = 0; w < NV; ++w)
+                stage_rows<G>(src[w], a.B, ch0, a.n, tile_lo(t + AHEAD, R), sm.p[(i + AHEAD) % MS],
+                              sm.v[w][(i + AHEAD) % VS]);
+        }
+        cp_async_commit();
+        if (i + 1 < nt) {
+            tile_decays<G>(sm.s[(i + 1) % MS], sm.dl[(i + 1) & 1]);
+            if (threadIdx.x == 0) tile_ed(sm.s[(i + 1) % MS], t + 1, sm.ed[(i + 1) & 1]);
+        }
+        const float* sb = sm.s[i % MS];
+        const float* dl = sm.dl[i & 1];
+        float* vb[NV];
+#pragma unroll
+        for (int w = 0; w < NV; ++w) vb[w] = sm.v[w][i % VS] + k * G::SEG + c;
+        // pass 1: segment summaries, then the scans over the channel's segments
+        LP sr[NV], sl[NV];
 #pragma unroll
         for (int w = 0; w < NV; ++w) {
-            const float* vb = sm.v[w][i & 1] + k * G::SEG + c;
-            LP str = {0.f, 0.f}, stl = {0.f, 0.f};
+            sr[w] = LP{0.f, 0.f};
+            sl[w] = LP{0.f, 0.f};
 #pragma unroll
-            for (int e = E - 1; e >= 0; --e) str = lp_step_d(str, sm.dl[k * E + e + 1], 0.f, vb[e * C]);
+            for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dl[k * E + e + 1], 0.f, vb[w][e * C]);
 #pragma unroll
-            for (int e = 0; e < E; ++e) stl = lp_step_d(stl, sm.dl[k * E + e], 0.f, vb[e * C]);
-            block_scan_dir<C, kNT, true>(str, -sb[4 + k * E], ub_r, sm.sc[2 * w], exR[w], hR[w]);
-            block_scan_dir<C, kNT, false>(stl, sb[4 + k * E + E - 1], ub_l, sm.sc[2 * w + 1], exL[w], hL[w]);
+            for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dl[k * E + e], 0.f, vb[w][e * C]);
         }
-        // tile carries (threads < C), then fold the tile into the left state
-        if (threadIdx.x < C) {
+        group_scan<SK, NV>(sl, sr, sb, k);  // now inclusive over segments 0..k (left) / k..SK-1 (right)
+        // tile carries: the channel's first lane folds in fp64, then broadcasts
+        const bool more = (t + 1 < min(a.T, (J + 1) * a.tpr)), hasRin = (J + 1 < a.P);
+        const bool hl_tile = hasL, hr_tile = hasRin || more;
+        LP cL[NV], cR[NV];
 #pragma unroll
-            for (int w = 0; w < NV; ++w) {
-                sm.carry[2 * w + 1][c] = runL[w];
-                // right: the range carry (farther right) followed by the in-range suffix RS[t+1]
-                double2 cr = rin[w];
-                bool hr = hasRin;
-                if (t + 1 < te) {
-                    const double2 rsn = rs[w]->RS[((int64_t)grp * a.T + t + 1) * C + c];
-                    cr = hr ? lpd_combine(rin[w], uRin, rsn, -sb[4 + R]) : rsn;
-                    hr = true;
+        for (int w = 0; w < NV; ++w) {
+            const LP tl = shfl_lp(sl[w], SK - 1, SK);
+            cL[w] = LP{0.f, 0.f};
+            cR[w] = LP{0.f, 0.f};
+            if (k == 0) {
+                const double* ed = sm.ed[i & 1];
+                const double2 cl = runL[w];
+                double2 cr = hasRin ? sm.rin[i % MS][w][c] : make_double2(0.0, 0.0);
+                if (more) {
+                    const double2 rsn = sm.rs[i % MS][w][c];
+                    cr = hasRin ? combine_ed(cr, rsn, ed[1], -sb[4 + R] > u_rin(J)) : rsn;
                 }
-                sm.carry[2 * w][c] = cr;
-                if (c == 0) {
-                    sm.has[2 * w] = hr;
-                    sm.has[2 * w + 1] = hasL;
-                }
-                const LP tl = sm.sc[2 * w + 1].tot[c];
-                const double2 tld = make_double2(tl.L, tl.P);
-                runL[w] = hasL ? lpd_combine(runL[w], sb[3], tld, sb[4 + R - 1]) : tld;
+                cL[w] = LP{(float)cl.x, (float)cl.y};
+                cR[w] = LP{(float)cr.x, (float)cr.y};
+                const double2 tld = to_d2(tl);
+                runL[w] = hl_tile ? combine_ed(runL[w], tld, ed[0], sb[4 + R - 1] > sb[3]) : tld;
             }
+            cL[w] = shfl_lp(cL[w], 0, SK);
+            cR[w] = shfl_lp(cR[w], 0, SK);
         }
-        __syncthreads();
         hasL = true;
-        // second pass: both directions from the true incoming states
+        // incoming state of this segment: tile carry, then the segments before it
+        const float ub_r = -sb[4 + k * E + E], ub_l = sb[4 + k * E - 1];
         LP inR[NV], inL[NV];
 #pragma unroll
         for (int w = 0; w < NV; ++w) {
-            const double2 cr = sm.carry[2 * w][c], cl = sm.carry[2 * w + 1][c];
-            inR[w] = seg_incoming(sm.has[2 * w], LP{(float)cr.x, (float)cr.y}, -sb[4 + R], hR[w], exR[w], ub_r);
-            inL[w] = seg_incoming(sm.has[2 * w + 1], LP{(float)cl.x, (float)cl.y}, sb[3], hL[w], exL[w], ub_l);
+            const LP exL = shfl_lp(sl[w], (lane - 1) & 31, 32), exR = shfl_lp(sr[w], (lane + 1) & 31, 32);
+            inL[w] = seg_incoming(hl_tile, cL[w], sb[3], k >= 1, exL, ub_l);
+            inR[w] = seg_incoming(hr_tile, cR[w], -sb[4 + R], k + 1 < SK, exR, ub_r);
         }
+        // pass 2: results replace the staged values in place
         if (NV == 1) {
-            const float* vb = sm.v[0][i & 1] + k * G::SEG + c;
             float yv[E];
-            LP s2 = inR[0];
+            float Pr = inR[0].P;
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
-                const float xe = vb[e * C];
-                s2 = lp_step_d(s2, sm.dl[k * E + e + 1], 0.f, xe);
-                yv[e] = s2.P - xe;
+                const float xe = vb[0][e * C];
+                Pr = fmaf(fabsf(dl[k * E + e + 1]), Pr, xe);  // only the inclusive sums are needed here
+                yv[e] = Pr - xe;
             }
-            s2 = inL[0];
+            float Pl = inL[0].P;
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const int r = k * E + e;
-                s2 = lp_step_d(s2, sm.dl[r], 0.f, vb[e * C]);
-                if (cval && lo + r < a.n) out[(int64_t)min(pb[r], (uint32_t)(a.n - 1)) * a.B + ch] = yv[e] + s2.P;
+                Pl = fmaf(fabsf(dl[k * E + e]), Pl, vb[0][e * C]);
+                vb[0][e * C] = yv[e] + Pl;
             }
         } else {
-            const float* xv = sm.v[0][i & 1] + k * G::SEG + c;
-            const float* gv = sm.v[NV - 1][i & 1] + k * G::SEG + c;
             float gxp[E], gap[E];
             LP ax = inR[0], ag = inR[NV - 1];
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
-                const float xe = xv[e * C], ge = gv[e * C], dv = sm.dl[k * E + e + 1];
+                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dl[k * E + e + 1];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
                 gxp[e] = ag.P - ge;
@@ -336,22 +459,52 @@ __global__ void __launch_bounds__(kNT, (NV == 1 ? 3 : 2)) k_sym_sweep(SymScan a,
             ag = inL[NV - 1];
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const int r = k * E + e;
-                const float xe = xv[e * C], ge = gv[e * C], dv = sm.dl[r];
+                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dl[k * E + e];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
-                const bool valid = lo + r < a.n;
-                const int64_t row = min(pb[r], (uint32_t)(a.n - 1));
-                if (out != nullptr && cval && valid) out[row * a.B + ch] = gxp[e] + ag.P;
-                float part = gap[e] - fmaf(ge, ax.L, xe * ag.L);  // minus strict left sums
-#pragma unroll
-                for (int off = C / 2; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-                if (ga != nullptr && c == 0 && valid) {
-                    if (ga_atomic)
-                        atomicAdd(ga + row, part);
-                    else
-                        ga[row] = part;
+                vb[0][e * C] = gxp[e] + ag.P;                         // gx
+                vb[NV - 1][e * C] = gap[e] - fmaf(ge, ax.L, xe * ag.L);  // this channel's share of ga
+            }
+        }
+        __syncthreads();
+        // coalesced stores of whole rows through the permutation
+        const uint32_t* pb = sm.p[i % MS];
+        if (out != nullptr) {
+            constexpr int W = (G::VW > 1) ? G::VW : 1;
+            const float* ob = sm.v[0][i % VS];
+            if (W > 1 && (a.B % W) == 0) {
+                constexpr int Q = G::C >= W ? G::C / W : 1;
+                for (int q = threadIdx.x; q < R * Q; q += NT) {
+                    const int r = q / Q, cc = (q % Q) * W;
+                    if (lo + r < a.n && ch0 + cc < a.B) {
+                        float* dst = out + (int64_t)min(pb[r], (uint32_t)(a.n - 1)) * a.B + ch0 + cc;
+                        const float* sp = ob + G::xidx(r, cc);
+                        if (W == 4)
+                            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(sp);
+                        else
+                            *reinterpret_cast<float2*>(dst) = *reinterpret_cast<const float2*>(sp);
+                    }
                 }
+            } else {
+                for (int q = threadIdx.x; q < R * C; q += NT) {
+                    const int r = q / C, cc = q % C;
+                    if (lo + r < a.n && ch0 + cc < a.B)
+                        out[(int64_t)min(pb[r], (uint32_t)(a.n - 1)) * a.B + ch0 + cc] = ob[G::xidx(r, cc)];
+                }
+            }
+        }
+        if (NV == 2 && ga != nullptr) {
+            const float* gb = sm.v[NV - 1][i % VS];
+            for (int r = threadIdx.x; r < R; r += NT) {
+                if (lo + r >= a.n) continue;
+                float acc = 0.f;
+#pragma unroll
+                for (int cc = 0; cc < C; ++cc) acc += gb[G::xidx(r, cc)];  // channels past B hold zero
+                const int64_t row = min(pb[r], (uint32_t)(a.n - 1));
+                if (ga_atomic)
+                    atomicAdd(ga + row, acc);
+                else
+                    ga[row] = acc;
             }
         }
     }
@@ -370,7 +523,7 @@ SymPlan plan_sym(int64_t n, int64_t B, int sms) {
     SymPlan p;
     p.C = choose_channels(B);
     p.G = (int)((B + p.C - 1) / p.C);
-    p.R = (int64_t)kNT / p.C * (p.C == 1 ? 8 : 16);
+    p.R = rows_per_tile(p.C);
     p.T = (n + p.R - 1) / p.R;
     const int64_t want = std::max<int64_t>(1, ((int64_t)sms * kRangesPerSM + p.G - 1) / p.G);
     const int64_t P0 = std::min<int64_t>(std::min<int64_t>(p.T, want), kMaxRanges);
@@ -400,54 +553,21 @@ int device_sms() {
     return sms;
 }
 
+// Opt a kernel into its dynamic shared memory and return its resident CTAs per SM
+// (cached: one device type per process).
 template <class F>
-cudaError_t set_smem(F* f, size_t bytes) {
-    return cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+int prepare(F* f, int threads, size_t smem, int& cached) {
+    if (cached > 0) return cached;
+    int occ = 1;
+    if (cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, f, threads, smem) != cudaSuccess)
+        occ = 1;
+    cached = std::max(occ, 1);
+    return cached;
 }
 
-// Pass A + pass B for one vector.
-template <int C>
-cudaError_t sym_ranges_t(const SymScan& a, const SymPlan& p, const float* v, RangeState st, cudaStream_t s) {
-    const dim3 grid((unsigned)p.P, (unsigned)p.G);
-    const size_t smA = sizeof(SymSmem<C, 1>);
-    cudaError_t e = set_smem(k_sym_agg<C>, smA);
-    if (e != cudaSuccess) return e;
-    LAPLEX_TIMED("sym_agg", s, k_sym_agg<C><<<grid, kNT, smA, s>>>(a, v, st));
-    LAPLEX_TIMED("sym_carry", s, k_sym_carry<C><<<p.G, kNT, 0, s>>>(a, st));
-    return cudaGetLastError();
-}
-
-template <int C>
-cudaError_t sym_forward_t(const SymScan& a, const SymPlan& p, const float* x, float* y, RangeState sx, cudaStream_t s) {
-    cudaError_t e = sym_ranges_t<C>(a, p, x, sx, s);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)p.P, (unsigned)p.G);
-    const size_t smC = sizeof(SymSmem<C, 1>);
-    e = set_smem(k_sym_sweep<C, 1>, smC);
-    if (e != cudaSuccess) return e;
-    LAPLEX_TIMED("sym_fwd", s, k_sym_sweep<C, 1><<<grid, kNT, smC, s>>>(a, x, nullptr, sx, sx, y, nullptr, 0));
-    return cudaGetLastError();
-}
-
-template <int C>
-cudaError_t sym_backward_t(const SymScan& a, const SymPlan& p, const float* x, const float* g, float* gx, float* ga,
-                           RangeState sx, bool have_x, RangeState sg, cudaStream_t s) {
-    cudaError_t e;
-    if (!have_x) {
-        e = sym_ranges_t<C>(a, p, x, sx, s);
-        if (e != cudaSuccess) return e;
-    }
-    e = sym_ranges_t<C>(a, p, g, sg, s);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)p.P, (unsigned)p.G);
-    const size_t smC = sizeof(SymSmem<C, 2>);
-    e = set_smem(k_sym_sweep<C, 2>, smC);
-    if (e != cudaSuccess) return e;
-    LAPLEX_TIMED("sym_bwd", s, k_sym_sweep<C, 2><<<grid, kNT, smC, s>>>(a, x, g, sx, sg, gx, ga, p.G > 1 ? 1 : 0));
-    return cudaGetLastError();
-}
-
-SymScan scan_args(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B) {
+// Base ranges per CTA so that the grid is one wave at occupancy `occ`.
+SymScan scan_args(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms, int occ) {
     SymScan a;
     a.s = s;
     a.perm = perm;
@@ -456,7 +576,85 @@ SymScan scan_args(const SymPlan& p, const float* s, const uint32_t* perm, int64_
     a.T = p.T;
     a.P = p.P;
     a.tpr = p.tpr;
+    const int64_t slots = std::max<int64_t>(1, (int64_t)sms * occ / p.G);
+    a.m = (int)std::max<int64_t>(1, (p.P + slots - 1) / slots);
     return a;
+}
+
+// Pass A + pass B for one vector.
+template <int C>
+cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms,
+                         const float* v, RangeState st, cudaStream_t stream) {
+    using SM = SymSmem<C, 1, kAheadFwd>;
+    static int occ_cache = 0;
+    const int occ = prepare(k_sym_agg<C, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
+    LAPLEX_TIMED("sym_agg", stream,
+                 k_sym_agg<C, kAheadFwd><<<grid, SymGeo<C>::NT, sizeof(SM), stream>>>(a, v, st));
+    LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, 256, 0, stream>>>(a, st));
+    return cudaGetLastError();
+}
+
+template <int C>
+cudaError_t sym_forward_t(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B, float* y,
+                          void* saved, void* ws, cudaStream_t st) {
+    const int sms = device_sms();
+    const SymPlan p = plan_sym(n, B, sms);
+    RangeState sx = carve(p, (double2*)ws, true);
+    if (saved != nullptr) {  // RS and carries go to the caller's buffer; aggregates stay in ws
+        const RangeState sv = carve(p, (double2*)saved, false);
+        sx.RS = sv.RS;
+        sx.Lin = sv.Lin;
+        sx.Rin = sv.Rin;
+    }
+    cudaError_t e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, st);
+    if (e != cudaSuccess) return e;
+    using SM = SymSmem<C, 1, kAheadFwd>;
+    static int occ_cache = 0;
+    const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
+    LAPLEX_TIMED("sym_fwd", st,
+                 k_sym_sweep<C, 1, kAheadFwd>
+                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, x, nullptr, sx, sx, y, nullptr, 0));
+    return cudaGetLastError();
+}
+
+template <int C>
+cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, const float* x, const float* g, int64_t B,
+                           const void* saved, float* gx, float* ga, void* ws, cudaStream_t st) {
+    const int sms = device_sms();
+    const SymPlan p = plan_sym(n, B, sms);
+    const size_t half = align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
+    RangeState sx = carve(p, (double2*)ws, true);
+    const RangeState sg = carve(p, (double2*)((char*)ws + half), true);
+    if (saved != nullptr) {
+        const RangeState sv = carve(p, (double2*)saved, false);
+        sx.RS = sv.RS;
+        sx.Lin = sv.Lin;
+        sx.Rin = sv.Rin;
+    }
+    cudaError_t e;
+    if (ga != nullptr && p.G > 1) {
+        e = cudaMemsetAsync(ga, 0, sizeof(float) * n, st);
+        if (e != cudaSuccess) return e;
+    }
+    if (saved == nullptr) {
+        e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, st);
+        if (e != cudaSuccess) return e;
+    }
+    e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, st);
+    if (e != cudaSuccess) return e;
+    using SM = SymSmem<C, 2, kAheadBwd>;
+    static int occ_cache = 0;
+    const int occ = prepare(k_sym_sweep<C, 2, kAheadBwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
+    LAPLEX_TIMED("sym_bwd", st,
+                 k_sym_sweep<C, 2, kAheadBwd>
+                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, x, g, sx, sg, gx, ga, p.G > 1 ? 1 : 0));
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -481,17 +679,8 @@ size_t sym_saved_bytes(int64_t n, int64_t B) {
 cudaError_t launch_sym_forward(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B, float* y,
                                void* saved, void* ws, int32_t* status, cudaStream_t st) {
     (void)status;  // no kernel of this path waits on another CTA
-    const SymPlan p = plan_sym(n, B, device_sms());
-    const SymScan a = scan_args(p, s, perm, n, B);
-    RangeState sx = carve(p, (double2*)ws, true);
-    if (saved != nullptr) {  // RS and carries go to the caller's buffer; aggregates stay in ws
-        const RangeState sv = carve(p, (double2*)saved, false);
-        sx.RS = sv.RS;
-        sx.Lin = sv.Lin;
-        sx.Rin = sv.Rin;
-    }
-#define CALL(C) sym_forward_t<C>(a, p, x, y, sx, st)
-    LAPLEX_SYM_DISPATCH(p.C, CALL)
+#define CALL(C) sym_forward_t<C>(s, perm, n, x, B, y, saved, ws, st)
+    LAPLEX_SYM_DISPATCH(choose_channels(B), CALL)
 #undef CALL
 }
 
@@ -499,23 +688,8 @@ cudaError_t launch_sym_backward(const float* s, const uint32_t* perm, int64_t n,
                                 int64_t B, const void* saved, float* gx, float* ga, void* ws, int32_t* status,
                                 cudaStream_t st) {
     (void)status;
-    const SymPlan p = plan_sym(n, B, device_sms());
-    const SymScan a = scan_args(p, s, perm, n, B);
-    const size_t half = align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
-    RangeState sx = carve(p, (double2*)ws, true);
-    const RangeState sg = carve(p, (double2*)((char*)ws + half), true);
-    if (saved != nullptr) {
-        const RangeState sv = carve(p, (double2*)saved, false);
-        sx.RS = sv.RS;
-        sx.Lin = sv.Lin;
-        sx.Rin = sv.Rin;
-    }
-    if (ga != nullptr && p.G > 1) {
-        const cudaError_t e = cudaMemsetAsync(ga, 0, sizeof(float) * n, st);
-        if (e != cudaSuccess) return e;
-    }
-#define CALL(C) sym_backward_t<C>(a, p, x, g, gx, ga, sx, saved != nullptr, sg, st)
-    LAPLEX_SYM_DISPATCH(p.C, CALL)
+#define CALL(C) sym_backward_t<C>(s, perm, n, x, g, B, saved, gx, ga, ws, st)
+    LAPLEX_SYM_DISPATCH(choose_channels(B), CALL)
 #undef CALL
 }
 

@@ -72,9 +72,9 @@ def test_bad_arguments_are_rejected_before_launch(L):
     assert L.laplex_apply_sym(fake, fake, 8, fake, 1, ws, None, ws, 8, None, None) == 3
     # misaligned output
     assert L.laplex_apply_sym(P(1 << 20), P(1 << 22), 8, P(1 << 23), 1, P((1 << 24) + 4), None, P(1 << 25),
-                              1 << 20, None, None) == 2
+                              1 << 30, None, None) == 2
     # output overlapping the input
-    assert L.laplex_apply_sym(P(1 << 20), P(1 << 22), 8, P(1 << 23), 1, P(1 << 23), None, P(1 << 25), 1 << 20,
+    assert L.laplex_apply_sym(P(1 << 20), P(1 << 22), 8, P(1 << 23), 1, P(1 << 23), None, P(1 << 25), 1 << 30,
                               None, None) == 1
     # phased without phases
     assert L.laplex_apply_phased(fake, fake, 8, None, fake, fake, 4, None, 0, fake, 1, ws, None, ws, 1 << 30,
