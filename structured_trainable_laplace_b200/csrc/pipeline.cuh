@@ -118,17 +118,6 @@ __device__ __forceinline__ void stage_rows(const float* __restrict__ v, int B, i
     }
 }
 
-// Per-row decays of a staged tile: dl[r] = exp(a(r-1) - a(r)) for r in [0, R],
-// stored as -1 when a(r) == a(r-1) (tie: decay 1, no break).  The right-to-left
-// direction uses dl[r+1] for row r.
-template <class G>
-__device__ __forceinline__ void tile_decays(const float* s_buf, float* dl) {
-    for (int r = threadIdx.x; r <= G::R; r += G::NT) {
-        const float prev = s_buf[3 + r], cur = s_buf[4 + r];
-        dl[r] = (cur > prev) ? expf(prev - cur) : -1.f;
-    }
-}
-
 // Encoded decay between two oriented anchors uA <= uB: exp(uA - uB) when uB > uA
 // (a break), -1 when they are equal (a tie: decay 1, no break).
 __device__ __forceinline__ float enc_decay(float uA, float uB) { return (uB > uA) ? expf(uA - uB) : -1.f; }
@@ -158,141 +147,6 @@ __device__ __forceinline__ double2 combine_ed(double2 A, double2 B, double e, bo
     o.y = fma(e, A.y, B.y);
     o.x = brk ? fma(e, A.y, B.x) : (A.x + B.x);
     return o;
-}
-
-// Shared scratch of block_scan2 for NV vectors, both directions.
-template <int C, int NT, int NV>
-struct Scan2Smem {
-    static constexpr int NW = NT / 32;
-    LP wtL[NW][NV][C], wtR[NW][NV][C];  // warp totals
-    LP wxL[NW][NV][C], wxR[NW][NV][C];  // exclusive prefixes over warps
-    float wuL[NW], wuR[NW];             // oriented anchors of each warp's last row
-};
-
-// In-tile scan of NV vectors in both directions at once (one barrier pair).
-// Thread (c, k) = (tid % C, tid / C) owns segment k of channel c; left
-// processing order is k ascending, right is k descending.  segL/segR are the
-// segment summaries, anchored at uL_end = a(last row) and uR_end = -a(first row);
-// uL_before / uR_before are the oriented anchors of the row just before the
-// segment in each direction.  Returns the in-tile exclusive prefixes (anchored
-// at uL_before / uR_before) with has-flags.  on_total(c, totL, totR) runs once
-// per channel, after the tile totals are known and before the final barrier,
-// so it can publish tile carries to shared memory for every thread.
-template <int C, int NT, int NV, class F>
-__device__ __forceinline__ void block_scan2(const LP (&segL)[NV], const LP (&segR)[NV], float uL_end, float uL_before,
-                                            float uR_end, float uR_before, Scan2Smem<C, NT, NV>& sm, LP (&exL)[NV],
-                                            LP (&exR)[NV], bool& hL, bool& hR, F&& on_total) {
-    constexpr int SW = 32 / C;
-    constexpr int NW = NT / 32;
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, c = threadIdx.x % C;
-    const int ql = lane / C, qr = SW - 1 - ql;
-    LP incL[NV], incR[NV];
-#pragma unroll
-    for (int v = 0; v < NV; ++v) {
-        incL[v] = segL[v];
-        incR[v] = segR[v];
-    }
-#pragma unroll
-    for (int off = 1; off < SW; off <<= 1) {
-        const int sL = (lane - off * C) & 31, sR = (lane + off * C) & 31;
-        const float uoL = __shfl_sync(0xffffffffu, uL_end, sL), uoR = __shfl_sync(0xffffffffu, uR_end, sR);
-        const float eL = expf(uoL - uL_end), eR = expf(uoR - uR_end);
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            LP oL, oR;
-            oL.L = __shfl_sync(0xffffffffu, incL[v].L, sL);
-            oL.P = __shfl_sync(0xffffffffu, incL[v].P, sL);
-            oR.L = __shfl_sync(0xffffffffu, incR[v].L, sR);
-            oR.P = __shfl_sync(0xffffffffu, incR[v].P, sR);
-            if (ql >= off) incL[v] = combine_e(oL, incL[v], eL, uL_end > uoL);
-            if (qr >= off) incR[v] = combine_e(oR, incR[v], eR, uR_end > uoR);
-        }
-    }
-    {
-        const int sL = (lane - C) & 31, sR = (lane + C) & 31;
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            exL[v].L = __shfl_sync(0xffffffffu, incL[v].L, sL);
-            exL[v].P = __shfl_sync(0xffffffffu, incL[v].P, sL);
-            exR[v].L = __shfl_sync(0xffffffffu, incR[v].L, sR);
-            exR[v].P = __shfl_sync(0xffffffffu, incR[v].P, sR);
-        }
-        hL = ql >= 1;
-        hR = qr >= 1;
-    }
-    if (ql == SW - 1) {
-#pragma unroll
-        for (int v = 0; v < NV; ++v) sm.wtL[w][v][c] = incL[v];
-        if (c == 0) sm.wuL[w] = uL_end;
-    }
-    if (qr == SW - 1) {
-#pragma unroll
-        for (int v = 0; v < NV; ++v) sm.wtR[w][v][c] = incR[v];
-        if (c == 0) sm.wuR[w] = uR_end;
-    }
-    __syncthreads();
-    if (threadIdx.x < C * NW) {
-        const int cc = threadIdx.x % C, jp = threadIdx.x / C;
-        LP aL[NV], aR[NV];
-        // left: fold warps 0 .. jp-1
-        for (int j = 0; j < jp; ++j) {
-            const float e = (j > 0) ? expf(sm.wuL[j - 1] - sm.wuL[j]) : 0.f;
-            const bool brk = (j > 0) && sm.wuL[j] > sm.wuL[j - 1];
-#pragma unroll
-            for (int v = 0; v < NV; ++v) aL[v] = (j == 0) ? sm.wtL[0][v][cc] : combine_e(aL[v], sm.wtL[j][v][cc], e, brk);
-        }
-        // right: fold warps NW-1 .. NW-jp (processing order)
-        for (int j = 0; j < jp; ++j) {
-            const int wj = NW - 1 - j;
-            const float e = (j > 0) ? expf(sm.wuR[wj + 1] - sm.wuR[wj]) : 0.f;
-            const bool brk = (j > 0) && sm.wuR[wj] > sm.wuR[wj + 1];
-#pragma unroll
-            for (int v = 0; v < NV; ++v) aR[v] = (j == 0) ? sm.wtR[wj][v][cc] : combine_e(aR[v], sm.wtR[wj][v][cc], e, brk);
-        }
-        if (jp > 0) {
-#pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                sm.wxL[jp][v][cc] = aL[v];
-                sm.wxR[NW - 1 - jp][v][cc] = aR[v];
-            }
-        }
-        if (jp == NW - 1) {
-            LP tL[NV], tR[NV];
-            const float eL = (NW > 1) ? expf(sm.wuL[NW - 2] - sm.wuL[NW - 1]) : 0.f;
-            const bool bL = (NW > 1) && sm.wuL[NW - 1] > sm.wuL[NW - 2];
-            const float eR = (NW > 1) ? expf(sm.wuR[1] - sm.wuR[0]) : 0.f;
-            const bool bR = (NW > 1) && sm.wuR[0] > sm.wuR[1];
-#pragma unroll
-            for (int v = 0; v < NV; ++v) {
-                tL[v] = (NW > 1) ? combine_e(aL[v], sm.wtL[NW - 1][v][cc], eL, bL) : sm.wtL[0][v][cc];
-                tR[v] = (NW > 1) ? combine_e(aR[v], sm.wtR[0][v][cc], eR, bR) : sm.wtR[0][v][cc];
-            }
-            on_total(cc, tL, tR);
-        }
-    }
-    __syncthreads();
-    if (w > 0) {
-        const float uwe = sm.wuL[w - 1];
-        const float e = expf(uwe - uL_before);
-        const bool brk = uL_before > uwe;
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const LP we = sm.wxL[w][v][c];
-            exL[v] = hL ? combine_e(we, exL[v], e, brk) : we;
-        }
-        hL = true;
-    }
-    if (w < NW - 1) {
-        const float uwe = sm.wuR[w + 1];
-        const float e = expf(uwe - uR_before);
-        const bool brk = uR_before > uwe;
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-            const LP we = sm.wxR[w][v][c];
-            exR[v] = hR ? combine_e(we, exR[v], e, brk) : we;
-        }
-        hR = true;
-    }
 }
 
 }  // namespace laplex

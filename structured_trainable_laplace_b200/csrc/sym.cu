@@ -57,6 +57,88 @@ struct SymGeo {
 
 inline int64_t rows_per_tile(int C) { return C <= 8 ? 32 * kE : (32 * kE * 8) / C; }
 
+__host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+// Decays of one staged tile of SK segments, all encoded as by enc_decay and
+// computed once per tile (one tile ahead) instead of once per lane:
+//   d[k][e]   row k*E+e from the row before it, e in [0, E] (the last entry repeats
+//             the next segment's first, so each segment's row has E+1 entries
+//             and the SK lanes of a channel read distinct banks);
+//   gL/gR[j]  the step of width 2^j of the scans over segments (left: from the
+//             last row of segment k - 2^j to that of k; right: from -first row of
+//             k + 2^j to -first row of k);
+//   iL/iR[k]  from the tile carry to the state before segment k (left: row
+//             before the tile to the row before segment k; right: -row after the
+//             tile to -row after segment k).
+template <int SK>
+struct SegTab {
+    static constexpr int LOG = ilog2(SK) > 0 ? ilog2(SK) : 1;
+    float d[SK][kE + 1];
+    float gL[LOG][SK], gR[LOG][SK];
+    float iL[SK], iR[SK];
+};
+
+template <int SK, int NT>
+__device__ __forceinline__ void seg_tables(const float* sb, SegTab<SK>& tb) {
+    constexpr int E = kE, R = SK * E, LOG = ilog2(SK);
+    constexpr int N1 = SK * (E + 1), N2 = N1 + LOG * SK, N3 = N2 + SK;
+    for (int i = threadIdx.x; i < N3; i += NT) {
+        if (i < N1) {
+            const int k = i / (E + 1), e = i % (E + 1), r = k * E + e;
+            tb.d[k][e] = enc_decay(sb[3 + r], sb[4 + r]);
+        } else if (i < N2) {
+            const int j = (i - N1) / SK, k = (i - N1) % SK, off = 1 << j;
+            tb.gL[j][k] = (k >= off) ? enc_decay(sb[4 + (k - off) * E + E - 1], sb[4 + k * E + E - 1]) : -1.f;
+            tb.gR[j][k] = (k + off < SK) ? enc_decay(-sb[4 + (k + off) * E], -sb[4 + k * E]) : -1.f;
+        } else {
+            const int k = i - N2;
+            tb.iL[k] = enc_decay(sb[3], sb[3 + k * E]);
+            tb.iR[k] = enc_decay(-sb[4 + R], -sb[4 + (k + 1) * E]);
+        }
+    }
+}
+
+// State entering a segment: the tile carry (if any) followed by the exclusive
+// scan over the segments before it (if any); ev is the decay between the two.
+__device__ __forceinline__ LP seg_in(bool has_carry, LP carry, bool has_excl, LP excl, float ev) {
+    if (has_carry && has_excl) return combine_v(carry, excl, ev);
+    if (has_carry) return carry;
+    if (has_excl) return excl;
+    return LP{0.f, 0.f};
+}
+
+// Sum of v[E] over the CW lanes of a row group (lanes SK apart) by recursive
+// halving: afterwards lane cs holds in v[0, E/CW) the sums for rows
+// seg_rows_base<CW>(cs) + [0, E/CW) of its segment.
+template <int CW, int SK>
+__device__ __forceinline__ void reduce_scatter(float (&v)[kE], int cs) {
+    int len = kE;
+#pragma unroll
+    for (int o = 1; o < CW; o <<= 1) {
+        len >>= 1;
+        const bool upper = (cs & o) != 0;
+#pragma unroll
+        for (int i = 0; i < kE / 2; ++i) {
+            if (i < len) {
+                const float keep = upper ? v[i + len] : v[i];
+                const float send = upper ? v[i] : v[i + len];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o * SK);
+            }
+        }
+    }
+}
+
+template <int CW>
+__device__ __forceinline__ int seg_rows_base(int cs) {
+    int base = 0, len = kE;
+#pragma unroll
+    for (int o = 1; o < CW; o <<= 1) {
+        len >>= 1;
+        if (cs & o) base += len;
+    }
+    return base;
+}
+
 struct SymScan {
     const float* s;
     const uint32_t* perm;
@@ -87,8 +169,11 @@ struct SymSmem {
     double2 rs[MS][NV][C];   // RS[t+1] (sweep)
     double2 rin[MS][NV][C];  // carry entering the tile's base range from the right (sweep)
     float v[NV][VS][G::XS];
-    float dl[2][G::R + 4];  // per-row decays of the current and the next tile
-    double ed[2][2];        // fp64 decays of the two tile-level folds, current and next tile
+    SegTab<SymGeo<C>::SK> tab[2];  // decay tables of the current and the next tile
+    double ed[2][2];               // fp64 decays of the two tile-level folds, current and next tile
+    // backward: per-warp sums of the ga shares of the warp's channels, rows padded
+    // as in SegTab::d
+    float gp[NV == 2 ? SymGeo<C>::NW : 1][NV == 2 ? SymGeo<C>::SK * (kE + 1) : 1];
 };
 
 __device__ __forceinline__ int64_t tile_lo(int64_t t, int R) { return t * (int64_t)R; }
@@ -103,14 +188,12 @@ __device__ __forceinline__ LP shfl_lp(LP v, int src, int width) {
 }
 
 // Inclusive scans over the SK segments of one channel (the SK lanes of a group),
-// both directions, NV vectors.  sb: staged anchors; k: this lane's segment.
+// both directions, NV vectors.  tb: the tile's decay tables; k: this lane's segment.
 template <int SK, int NV>
-__device__ __forceinline__ void group_scan(LP (&incL)[NV], LP (&incR)[NV], const float* sb, int k) {
+__device__ __forceinline__ void group_scan(LP (&incL)[NV], LP (&incR)[NV], const SegTab<SK>& tb, int k) {
 #pragma unroll
-    for (int off = 1; off < SK; off <<= 1) {
-        const float uL = sb[4 + k * kE + kE - 1], uLo = sb[4 + max(k - off, 0) * kE + kE - 1];
-        const float uR = -sb[4 + k * kE], uRo = -sb[4 + min(k + off, SK - 1) * kE];
-        const float eL = expf(uLo - uL), eR = expf(uRo - uR);
+    for (int j = 0, off = 1; off < SK; ++j, off <<= 1) {
+        const float evL = tb.gL[j][k], evR = tb.gR[j][k];
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
             LP oL, oR;
@@ -118,8 +201,8 @@ __device__ __forceinline__ void group_scan(LP (&incL)[NV], LP (&incR)[NV], const
             oL.P = __shfl_up_sync(0xffffffffu, incL[v].P, off, SK);
             oR.L = __shfl_down_sync(0xffffffffu, incR[v].L, off, SK);
             oR.P = __shfl_down_sync(0xffffffffu, incR[v].P, off, SK);
-            if (k >= off) incL[v] = combine_e(oL, incL[v], eL, uL > uLo);
-            if (k + off < SK) incR[v] = combine_e(oR, incR[v], eR, uR > uRo);
+            if (k >= off) incL[v] = combine_v(oL, incL[v], evL);
+            if (k + off < SK) incR[v] = combine_v(oR, incR[v], evR);
         }
     }
 }
@@ -178,7 +261,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
         if (q < nt) stage_rows<G>(v, a.B, ch0, a.n, tile_lo(tile_of(q), R), sm.p[q % MS], sm.v[0][q % VS]);
         cp_async_commit();
     }
-    tile_decays<G>(sm.s[0], sm.dl[0]);
+    seg_tables<SK, SG::NT>(sm.s[0], sm.tab[0]);
     if (threadIdx.x == 0) tile_ed(sm.s[0], tile_of(0), sm.ed[0]);
     double2 runR = make_double2(0.0, 0.0), runL = make_double2(0.0, 0.0);
     for (int i = 0; i < nt; ++i) {
@@ -195,18 +278,19 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
                           sm.v[0][(i + AHEAD) % VS]);
         cp_async_commit();
         if (i + 1 < nt) {
-            tile_decays<G>(sm.s[(i + 1) % MS], sm.dl[(i + 1) & 1]);
+            seg_tables<SK, SG::NT>(sm.s[(i + 1) % MS], sm.tab[(i + 1) & 1]);
             if (threadIdx.x == 0) tile_ed(sm.s[(i + 1) % MS], tile_of(i + 1), sm.ed[(i + 1) & 1]);
         }
         const float* sb = sm.s[i % MS];
-        const float* dl = sm.dl[i & 1];
+        const SegTab<SK>& tb = sm.tab[i & 1];
+        const float* dk = tb.d[k];
         const float* xb = sm.v[0][i % VS] + k * G::SEG + c;
         LP sr[1] = {{0.f, 0.f}}, sl[1] = {{0.f, 0.f}};
 #pragma unroll
-        for (int e = E - 1; e >= 0; --e) sr[0] = lp_step_d(sr[0], dl[k * E + e + 1], 0.f, xb[e * C]);
+        for (int e = E - 1; e >= 0; --e) sr[0] = lp_step_d(sr[0], dk[e + 1], 0.f, xb[e * C]);
 #pragma unroll
-        for (int e = 0; e < E; ++e) sl[0] = lp_step_d(sl[0], dl[k * E + e], 0.f, xb[e * C]);
-        group_scan<SK, 1>(sl, sr, sb, k);
+        for (int e = 0; e < E; ++e) sl[0] = lp_step_d(sl[0], dk[e], 0.f, xb[e * C]);
+        group_scan<SK, 1>(sl, sr, tb, k);
         const LP tl = shfl_lp(sl[0], SK - 1, SK);  // tile totals: left at the last segment, right at the first
         if (k == 0) {
             const double* ed = sm.ed[i & 1];
@@ -225,61 +309,111 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
 
 // ------------------------------------------------------------------ pass B
 
-// One CTA per channel group.  Thread (c, q), q < QS, folds a contiguous block of
-// ranges; the blocks are then composed serially (at most QS steps) and re-walked
-// to produce the carry entering every range.
+// One CTA of kCarryThreads per channel group.  Thread (c, q) owns block q of PS
+// consecutive ranges: it folds their aggregates in both directions (loads issued
+// kCarryBatch at a time, ahead of the dependent folds), the NB block aggregates
+// are scanned in shared memory by doubling (log2 NB steps), and each thread then
+// re-walks its block, writing the carry entering every range.
+constexpr int kCarryThreads = 512;
+constexpr int kCarryBatch = 8;
+
 template <int C>
-__global__ void __launch_bounds__(256) k_sym_carry(SymScan a, RangeState st) {
-    constexpr int QS = (256 / C) < 16 ? (256 / C) : 16;
-    __shared__ double2 segL[QS][C], segR[QS][C];
+__global__ void __launch_bounds__(kCarryThreads) k_sym_carry(SymScan a, RangeState st) {
+    constexpr int QS = kCarryThreads / C, U = kCarryBatch;
+    __shared__ double2 sL[QS][C], sR[QS][C];
+    __shared__ float eL[QS], eR[QS];  // oriented end anchor of each block, per direction
     const int grp = blockIdx.x;
     const int c = threadIdx.x % C, q = threadIdx.x / C;
     const int P = a.P;
-    const int PS = (P + QS - 1) / QS;
+    const int PS = (P + QS - 1) / QS, NB = (P + PS - 1) / PS;
     const int j0 = min(P, q * PS), j1 = min(P, j0 + PS);
     const int64_t RR = a.tpr * (int64_t)SymGeo<C>::R;  // rows per range
     auto uL = [&](int jj) { return __ldg(a.s + min(a.n, (jj + 1) * RR) - 1); };  // left anchor of range jj
     auto uR = [&](int jj) { return -__ldg(a.s + jj * RR); };                    // right anchor of range jj
-    const int64_t base = (int64_t)grp * P * C + c;
-    const bool mine = q < QS && j0 < j1;
+    const double2* Lagg = st.Lagg + (int64_t)grp * P * C + c;
+    const double2* Ragg = st.Ragg + (int64_t)grp * P * C + c;
+    const bool mine = q < NB;  // blocks q >= NB are empty
+
+    // block aggregates (left: ranges j0 .. j1-1 in order; right: j1-1 .. j0)
+    double2 fl = make_double2(0.0, 0.0), fr = make_double2(0.0, 0.0);
+    float ufl = 0.f, ufr = 0.f;
     if (mine) {
-        double2 fl = st.Lagg[base + (int64_t)j0 * C];
-        for (int jj = j0 + 1; jj < j1; ++jj) fl = lpd_combine(fl, uL(jj - 1), st.Lagg[base + (int64_t)jj * C], uL(jj));
-        double2 fr = st.Ragg[base + (int64_t)(j1 - 1) * C];
-        for (int jj = j1 - 2; jj >= j0; --jj)
-            fr = lpd_combine(fr, uR(jj + 1), st.Ragg[base + (int64_t)jj * C], uR(jj));
-        segL[q][c] = fl;
-        segR[q][c] = fr;
+        for (int jb = j0; jb < j1; jb += U) {
+            double2 vl[U], vr[U];
+            float ul[U], ur[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int jl = jb + u, jr = j1 - 1 - (jb - j0) - u;
+                if (jl < j1) {
+                    vl[u] = Lagg[(int64_t)jl * C];
+                    ul[u] = uL(jl);
+                    vr[u] = Ragg[(int64_t)jr * C];
+                    ur[u] = uR(jr);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (jb + u < j1) {
+                    const bool first = (jb + u == j0);
+                    fl = first ? vl[u] : lpd_combine(fl, ufl, vl[u], ul[u]);
+                    fr = first ? vr[u] : lpd_combine(fr, ufr, vr[u], ur[u]);
+                    ufl = ul[u];
+                    ufr = ur[u];
+                }
+            }
+        }
+        sL[q][c] = fl;
+        sR[q][c] = fr;
+        if (c == 0) {
+            eL[q] = ufl;
+            eR[q] = ufr;
+        }
     }
     __syncthreads();
-    if (mine) {
-        bool hl = false;  // carry entering block q from the left: blocks 0 .. q-1
-        double2 cl = make_double2(0.0, 0.0);
-        for (int qq = 0; qq < q; ++qq) {
-            const int a0 = qq * PS, a1 = min(P, a0 + PS);
-            if (a0 >= a1) continue;
-            cl = hl ? lpd_combine(cl, uL(a0 - 1), segL[qq][c], uL(a1 - 1)) : segL[qq][c];
-            hl = true;
+    // inclusive scans over the blocks: left over 0..q, right over q..NB-1
+    for (int off = 1; off < NB; off <<= 1) {
+        const bool dl = mine && q >= off, dr = mine && q + off < NB;
+        double2 nl, nr;
+        if (dl) nl = lpd_combine(sL[q - off][c], eL[q - off], sL[q][c], eL[q]);
+        if (dr) nr = lpd_combine(sR[q + off][c], eR[q + off], sR[q][c], eR[q]);
+        __syncthreads();
+        if (dl) sL[q][c] = nl;
+        if (dr) sR[q][c] = nr;
+        __syncthreads();
+    }
+    if (!mine) return;
+    // carries entering the block, then entering each of its ranges
+    bool hl = q >= 1, hr = q + 1 < NB;
+    double2 cl = hl ? sL[q - 1][c] : make_double2(0.0, 0.0);
+    double2 cr = hr ? sR[q + 1][c] : make_double2(0.0, 0.0);
+    float ucl = hl ? eL[q - 1] : 0.f, ucr = hr ? eR[q + 1] : 0.f;
+    double2* Lin = st.Lin + (int64_t)grp * P * C + c;
+    double2* Rin = st.Rin + (int64_t)grp * P * C + c;
+    for (int jb = j0; jb < j1; jb += U) {
+        double2 vl[U], vr[U];
+        float ul[U], ur[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int jl = jb + u, jr = j1 - 1 - (jb - j0) - u;
+            if (jl < j1) {
+                vl[u] = Lagg[(int64_t)jl * C];
+                ul[u] = uL(jl);
+                vr[u] = Ragg[(int64_t)jr * C];
+                ur[u] = uR(jr);
+            }
         }
-        bool hr = false;  // from the right: blocks QS-1 .. q+1
-        double2 cr = make_double2(0.0, 0.0);
-        for (int qq = QS - 1; qq > q; --qq) {
-            const int a0 = qq * PS, a1 = min(P, a0 + PS);
-            if (a0 >= a1) continue;
-            cr = hr ? lpd_combine(cr, uR(a1), segR[qq][c], uR(a0)) : segR[qq][c];
-            hr = true;
-        }
-        for (int jj = j0; jj < j1; ++jj) {
-            st.Lin[base + (int64_t)jj * C] = cl;  // zero (unused) for the first range
-            const double2 ag = st.Lagg[base + (int64_t)jj * C];
-            cl = hl ? lpd_combine(cl, uL(jj - 1), ag, uL(jj)) : ag;
-            hl = true;
-        }
-        for (int jj = j1 - 1; jj >= j0; --jj) {
-            st.Rin[base + (int64_t)jj * C] = cr;  // zero (unused) for the last range
-            const double2 ag = st.Ragg[base + (int64_t)jj * C];
-            cr = hr ? lpd_combine(cr, uR(jj + 1), ag, uR(jj)) : ag;
-            hr = true;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int jl = jb + u, jr = j1 - 1 - (jb - j0) - u;
+            if (jl < j1) {
+                Lin[(int64_t)jl * C] = cl;  // zero (unused) for the first range
+                Rin[(int64_t)jr * C] = cr;  // zero (unused) for the last range
+                cl = hl ? lpd_combine(cl, ucl, vl[u], ul[u]) : vl[u];
+                cr = hr ? lpd_combine(cr, ucr, vr[u], ur[u]) : vr[u];
+                ucl = ul[u];
+                ucr = ur[u];
+                hl = hr = true;
+            }
         }
     }
 }
@@ -289,15 +423,18 @@ __global__ void __launch_bounds__(256) k_sym_carry(SymScan a, RangeState st) {
 // Start copying, for tile t, RS[t+1] (if t+1 is in the same base range) and the
 // right carry of t's base range, for each vector.
 template <int C, int NV>
-__device__ __forceinline__ void stage_carries(const SymScan& a, const RangeState* const* rs, int grp, int64_t t,
+__device__ __forceinline__ void stage_carries(const SymScan& a, const RangeState& sx, const RangeState& sg, int grp,
+                                              int64_t t,
                                               double2 (*rs_dst)[C], double2 (*rin_dst)[C]) {
     const int64_t J = t / a.tpr;
     const bool more = t + 1 < min(a.T, (J + 1) * a.tpr);
     const bool hasRin = J + 1 < a.P;
     for (int i = threadIdx.x; i < NV * C; i += SymGeo<C>::NT) {
         const int w = i / C, c = i % C;
-        if (more) cp_async16(&rs_dst[w][c], rs[w]->RS + ((int64_t)grp * a.T + t + 1) * C + c);
-        if (hasRin) cp_async16(&rin_dst[w][c], rs[w]->Rin + ((int64_t)grp * a.P + J) * C + c);
+        const double2* RS = (w == 0) ? sx.RS : sg.RS;
+        const double2* Rin = (w == 0) ? sx.Rin : sg.Rin;
+        if (more) cp_async16(&rs_dst[w][c], RS + ((int64_t)grp * a.T + t + 1) * C + c);
+        if (hasRin) cp_async16(&rin_dst[w][c], Rin + ((int64_t)grp * a.P + J) * C + c);
     }
 }
 
@@ -317,8 +454,6 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
     const int nt = (int)(cw.te - cw.tb);
     const int lane = threadIdx.x & 31, cs = lane / SK, k = lane % SK;
     const int c = (threadIdx.x >> 5) * CW + cs, ch0 = grp * C;
-    const float* src[2] = {x, g};
-    const RangeState* rs[2] = {&sx, &sg};
     // oriented anchor of the row after base range J (where its right carry is anchored)
     auto u_rin = [&](int64_t J) { return -__ldg(a.s + min(a.n - 1, (J + 1) * a.tpr * (int64_t)R)); };
     auto tile_ed = [&](const float* sb, int64_t t, double* ed) {  // [0] left fold, [1] right carry
@@ -329,7 +464,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
     for (int q = 0; q <= AHEAD; ++q) {
         if (q < nt) {
             stage_meta<G>(a.s, a.perm, a.n, tile_lo(cw.tb + q, R), sm.s[q % MS], sm.p[q % MS]);
-            stage_carries<C, NV>(a, rs, grp, cw.tb + q, sm.rs[q % MS], sm.rin[q % MS]);
+            stage_carries<C, NV>(a, sx, sg, grp, cw.tb + q, sm.rs[q % MS], sm.rin[q % MS]);
         }
         cp_async_commit();
     }
@@ -340,11 +475,11 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         if (q < nt) {
 #pragma unroll
             for (int w = 0; w < NV; ++w)
-                stage_rows<G>(src[w], a.B, ch0, a.n, tile_lo(cw.tb + q, R), sm.p[q % MS], sm.v[w][q % VS]);
+                stage_rows<G>(w == 0 ? x : g, a.B, ch0, a.n, tile_lo(cw.tb + q, R), sm.p[q % MS], sm.v[w][q % VS]);
         }
         cp_async_commit();
     }
-    tile_decays<G>(sm.s[0], sm.dl[0]);
+    seg_tables<SK, NT>(sm.s[0], sm.tab[0]);
     if (threadIdx.x == 0) tile_ed(sm.s[0], cw.tb, sm.ed[0]);
 
     // fp64 left folds of channel c, kept by the channel's first lane (k == 0)
@@ -352,7 +487,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
     bool hasL = (cw.J0 > 0);
     const int64_t rng = ((int64_t)grp * a.P + cw.J0) * C + c;
 #pragma unroll
-    for (int w = 0; w < NV; ++w) runL[w] = hasL ? rs[w]->Lin[rng] : make_double2(0.0, 0.0);
+    for (int w = 0; w < NV; ++w) runL[w] = hasL ? (w == 0 ? sx.Lin : sg.Lin)[rng] : make_double2(0.0, 0.0);
 
     for (int i = 0; i < nt; ++i) {
         const int64_t t = cw.tb + i, lo = tile_lo(t, R);
@@ -362,22 +497,24 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         if (i + AHEAD + 1 < nt) {
             stage_meta<G>(a.s, a.perm, a.n, tile_lo(t + AHEAD + 1, R), sm.s[(i + AHEAD + 1) % MS],
                           sm.p[(i + AHEAD + 1) % MS]);
-            stage_carries<C, NV>(a, rs, grp, t + AHEAD + 1, sm.rs[(i + AHEAD + 1) % MS], sm.rin[(i + AHEAD + 1) % MS]);
+            stage_carries<C, NV>(a, sx, sg, grp, t + AHEAD + 1, sm.rs[(i + AHEAD + 1) % MS],
+                                 sm.rin[(i + AHEAD + 1) % MS]);
         }
         cp_async_commit();
         if (i + AHEAD < nt) {
 #pragma unroll
             for (int w = 0; w < NV; ++w)
-                stage_rows<G>(src[w], a.B, ch0, a.n, tile_lo(t + AHEAD, R), sm.p[(i + AHEAD) % MS],
+                stage_rows<G>(w == 0 ? x : g, a.B, ch0, a.n, tile_lo(t + AHEAD, R), sm.p[(i + AHEAD) % MS],
                               sm.v[w][(i + AHEAD) % VS]);
         }
         cp_async_commit();
         if (i + 1 < nt) {
-            tile_decays<G>(sm.s[(i + 1) % MS], sm.dl[(i + 1) & 1]);
+            seg_tables<SK, NT>(sm.s[(i + 1) % MS], sm.tab[(i + 1) & 1]);
             if (threadIdx.x == 0) tile_ed(sm.s[(i + 1) % MS], t + 1, sm.ed[(i + 1) & 1]);
         }
         const float* sb = sm.s[i % MS];
-        const float* dl = sm.dl[i & 1];
+        const SegTab<SK>& tb = sm.tab[i & 1];
+        const float* dk = tb.d[k];
         float* vb[NV];
 #pragma unroll
         for (int w = 0; w < NV; ++w) vb[w] = sm.v[w][i % VS] + k * G::SEG + c;
@@ -388,11 +525,11 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
             sr[w] = LP{0.f, 0.f};
             sl[w] = LP{0.f, 0.f};
 #pragma unroll
-            for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dl[k * E + e + 1], 0.f, vb[w][e * C]);
+            for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dk[e + 1], 0.f, vb[w][e * C]);
 #pragma unroll
-            for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dl[k * E + e], 0.f, vb[w][e * C]);
+            for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dk[e], 0.f, vb[w][e * C]);
         }
-        group_scan<SK, NV>(sl, sr, sb, k);  // now inclusive over segments 0..k (left) / k..SK-1 (right)
+        group_scan<SK, NV>(sl, sr, tb, k);  // now inclusive over segments 0..k (left) / k..SK-1 (right)
         // tile carries: the channel's first lane folds in fp64, then broadcasts
         const bool more = (t + 1 < min(a.T, (J + 1) * a.tpr)), hasRin = (J + 1 < a.P);
         const bool hl_tile = hasL, hr_tile = hasRin || more;
@@ -420,13 +557,13 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         }
         hasL = true;
         // incoming state of this segment: tile carry, then the segments before it
-        const float ub_r = -sb[4 + k * E + E], ub_l = sb[4 + k * E - 1];
+        const float evl = tb.iL[k], evr = tb.iR[k];
         LP inR[NV], inL[NV];
 #pragma unroll
         for (int w = 0; w < NV; ++w) {
             const LP exL = shfl_lp(sl[w], (lane - 1) & 31, 32), exR = shfl_lp(sr[w], (lane + 1) & 31, 32);
-            inL[w] = seg_incoming(hl_tile, cL[w], sb[3], k >= 1, exL, ub_l);
-            inR[w] = seg_incoming(hr_tile, cR[w], -sb[4 + R], k + 1 < SK, exR, ub_r);
+            inL[w] = seg_in(hl_tile, cL[w], k >= 1, exL, evl);
+            inR[w] = seg_in(hr_tile, cR[w], k + 1 < SK, exR, evr);
         }
         // pass 2: results replace the staged values in place
         if (NV == 1) {
@@ -435,13 +572,13 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
                 const float xe = vb[0][e * C];
-                Pr = fmaf(fabsf(dl[k * E + e + 1]), Pr, xe);  // only the inclusive sums are needed here
+                Pr = fmaf(fabsf(dk[e + 1]), Pr, xe);  // only the inclusive sums are needed here
                 yv[e] = Pr - xe;
             }
             float Pl = inL[0].P;
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                Pl = fmaf(fabsf(dl[k * E + e]), Pl, vb[0][e * C]);
+                Pl = fmaf(fabsf(dk[e]), Pl, vb[0][e * C]);
                 vb[0][e * C] = yv[e] + Pl;
             }
         } else {
@@ -449,7 +586,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
             LP ax = inR[0], ag = inR[NV - 1];
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
-                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dl[k * E + e + 1];
+                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dk[e + 1];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
                 gxp[e] = ag.P - ge;
@@ -459,12 +596,18 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
             ag = inL[NV - 1];
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dl[k * E + e];
+                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dk[e];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
-                vb[0][e * C] = gxp[e] + ag.P;                         // gx
-                vb[NV - 1][e * C] = gap[e] - fmaf(ge, ax.L, xe * ag.L);  // this channel's share of ga
+                vb[0][e * C] = gxp[e] + ag.P;              // gx
+                gap[e] = gap[e] - fmaf(ge, ax.L, xe * ag.L);  // this channel's share of ga
             }
+            // sum over the warp's channels, then one padded row per warp in shared memory
+            reduce_scatter<CW, SK>(gap, cs);
+            const int rb = seg_rows_base<CW>(cs);
+            float* gpw = sm.gp[threadIdx.x >> 5] + k * (E + 1) + rb;
+#pragma unroll
+            for (int e = 0; e < E / CW; ++e) gpw[e] = gap[e];
         }
         __syncthreads();
         // coalesced stores of whole rows through the permutation
@@ -494,12 +637,11 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
             }
         }
         if (NV == 2 && ga != nullptr) {
-            const float* gb = sm.v[NV - 1][i % VS];
             for (int r = threadIdx.x; r < R; r += NT) {
                 if (lo + r >= a.n) continue;
                 float acc = 0.f;
 #pragma unroll
-                for (int cc = 0; cc < C; ++cc) acc += gb[G::xidx(r, cc)];  // channels past B hold zero
+                for (int q = 0; q < SG::NW; ++q) acc += sm.gp[q][r + r / E];  // channels past B hold zero
                 const int64_t row = min(pb[r], (uint32_t)(a.n - 1));
                 if (ga_atomic)
                     atomicAdd(ga + row, acc);
@@ -592,7 +734,7 @@ cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm,
     const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
     LAPLEX_TIMED("sym_agg", stream,
                  k_sym_agg<C, kAheadFwd><<<grid, SymGeo<C>::NT, sizeof(SM), stream>>>(a, v, st));
-    LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, 256, 0, stream>>>(a, st));
+    LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, kCarryThreads, 0, stream>>>(a, st));
     return cudaGetLastError();
 }
 
