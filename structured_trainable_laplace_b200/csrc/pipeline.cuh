@@ -81,41 +81,97 @@ __device__ __forceinline__ void stage_meta(const float* __restrict__ s, const ui
     }
 }
 
+// Per-thread walk over the (row, chunk) copies of one tile: W floats per copy, Q
+// copies per row, thread tid handles chunk tid % Q of rows tid / Q + it * RPI.
+template <class G, int W>
+struct RowWalk {
+    static constexpr int Q = G::C >= W ? G::C / W : 1;
+    static_assert(G::NT % Q == 0, "threads must cover whole rows");
+    static constexpr int RPI = G::NT / Q;  // rows per iteration
+    static constexpr int ITER = (G::R + RPI - 1) / RPI;
+    int r0, c;
+    __device__ __forceinline__ RowWalk() : r0(threadIdx.x / Q), c((threadIdx.x % Q) * W) {}
+    __device__ __forceinline__ int row(int it) const { return r0 + it * RPI; }
+    __device__ __forceinline__ int off(int it) const {  // offset of the copy in the staged layout
+        if constexpr (RPI % G::E == 0)
+            return G::xidx(r0, c) + it * (RPI / G::E) * G::SEG;
+        else
+            return G::xidx(row(it), c);
+    }
+};
+
 // Start gathering channels [ch0, ch0 + C) of the rows perm[lo + r] of v [n][B].
 // Copies of G::VW floats (16 or 8 bytes) when the rows of v keep that alignment,
-// else 4 bytes.
+// else 4 bytes.  Rows past n and channels past B are staged as zero.
+template <class G, int W>
+__device__ __forceinline__ void stage_rows_w(const float* __restrict__ v, int B, int ch0, int64_t n, int64_t lo,
+                                             const uint32_t* p_buf, float* x_buf) {
+    const RowWalk<G, W> wk;
+    const int rem = (int)((n - lo) < (int64_t)G::R ? (n - lo) : (int64_t)G::R);
+    const uint32_t last = (uint32_t)(n - 1);
+    const bool cok = ch0 + wk.c < B;
+    const float* src0 = v + ch0 + wk.c;
+#pragma unroll
+    for (int it = 0; it < RowWalk<G, W>::ITER; ++it) {
+        const int r = wk.row(it);
+        if (G::R % RowWalk<G, W>::RPI != 0 && r >= G::R) break;
+        float* dst = x_buf + wk.off(it);
+        if (r < rem && cok) {
+            const float* src = src0 + (size_t)min(p_buf[r], last) * B;
+            if constexpr (W == 4)
+                cp_async16(dst, src);
+            else if constexpr (W == 2)
+                cp_async8(dst, src);
+            else
+                cp_async4(dst, src);
+        } else {
+#pragma unroll
+            for (int q = 0; q < W; ++q) dst[q] = 0.f;
+        }
+    }
+}
+
 template <class G>
 __device__ __forceinline__ void stage_rows(const float* __restrict__ v, int B, int ch0, int64_t n, int64_t lo,
                                            const uint32_t* p_buf, float* x_buf) {
-    if (G::VW > 1 && (B % G::VW) == 0) {
-        constexpr int W = G::VW > 1 ? G::VW : 2;
-        constexpr int Q = G::C >= W ? G::C / W : 1;
-        for (int i = threadIdx.x; i < G::R * Q; i += G::NT) {
-            const int r = i / Q, c = (i % Q) * W;
-            float* dst = x_buf + G::xidx(r, c);
-            if (lo + r < n && ch0 + c < B) {
-                const uint32_t row = min(p_buf[r], (uint32_t)(n - 1));
-                if (W == 4)
-                    cp_async16(dst, v + (int64_t)row * B + ch0 + c);
-                else
-                    cp_async8(dst, v + (int64_t)row * B + ch0 + c);
-            } else {
+    if (G::VW > 1 && (B % G::VW) == 0)
+        stage_rows_w<G, G::VW>(v, B, ch0, n, lo, p_buf, x_buf);
+    else
+        stage_rows_w<G, 1>(v, B, ch0, n, lo, p_buf, x_buf);
+}
+
+// Store a staged tile back to the rows perm[lo + r] of out [n][B] (the inverse
+// of stage_rows; rows past n and channels past B are skipped).
+template <class G, int W>
+__device__ __forceinline__ void store_rows_w(float* __restrict__ out, int B, int ch0, int64_t n, int64_t lo,
+                                             const uint32_t* p_buf, const float* x_buf) {
+    const RowWalk<G, W> wk;
+    const int rem = (int)((n - lo) < (int64_t)G::R ? (n - lo) : (int64_t)G::R);
+    const uint32_t last = (uint32_t)(n - 1);
+    if (ch0 + wk.c >= B) return;
+    float* dst0 = out + ch0 + wk.c;
 #pragma unroll
-                for (int q = 0; q < W; ++q) dst[q] = 0.f;
-            }
-        }
-    } else {
-        for (int i = threadIdx.x; i < G::R * G::C; i += G::NT) {
-            const int r = i / G::C, c = i % G::C;
-            float* dst = x_buf + G::xidx(r, c);
-            if (lo + r < n && ch0 + c < B) {
-                const uint32_t row = min(p_buf[r], (uint32_t)(n - 1));
-                cp_async4(dst, v + (int64_t)row * B + ch0 + c);
-            } else {
-                *dst = 0.f;
-            }
-        }
+    for (int it = 0; it < RowWalk<G, W>::ITER; ++it) {
+        const int r = wk.row(it);
+        if (r >= rem || (G::R % RowWalk<G, W>::RPI != 0 && r >= G::R)) break;
+        float* dst = dst0 + (size_t)min(p_buf[r], last) * B;
+        const float* sp = x_buf + wk.off(it);
+        if constexpr (W == 4)
+            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(sp);
+        else if constexpr (W == 2)
+            *reinterpret_cast<float2*>(dst) = *reinterpret_cast<const float2*>(sp);
+        else
+            *dst = *sp;
     }
+}
+
+template <class G>
+__device__ __forceinline__ void store_rows(float* __restrict__ out, int B, int ch0, int64_t n, int64_t lo,
+                                           const uint32_t* p_buf, const float* x_buf) {
+    if (G::VW > 1 && (B % G::VW) == 0)
+        store_rows_w<G, G::VW>(out, B, ch0, n, lo, p_buf, x_buf);
+    else
+        store_rows_w<G, 1>(out, B, ch0, n, lo, p_buf, x_buf);
 }
 
 // Encoded decay between two oriented anchors uA <= uB: exp(uA - uB) when uB > uA

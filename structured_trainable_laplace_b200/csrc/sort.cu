@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a,
 // MODE 1: keys/values from the previous pass.  MODE 2: like 1, and the keys
 // leave as fp32 anchors (last pass).
 template <int MODE>
-__global__ void __launch_bounds__(kNT) k_radix_pass(const float* __restrict__ a, const uint32_t* __restrict__ keys_in,
+__global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__ a, const uint32_t* __restrict__ keys_in,
                                                     const uint32_t* __restrict__ vals_in, uint32_t* __restrict__ keys_out,
                                                     uint32_t* __restrict__ vals_out, int64_t n, int shift,
                                                     const uint32_t* __restrict__ hist, uint32_t* counter,
@@ -166,14 +166,25 @@ __global__ void __launch_bounds__(kNT) k_radix_pass(const float* __restrict__ a,
         s_whist[j][tid] = cnt;
         cnt += c;
     }
+    // publish this tile's count for digit tid (tile 0's is already its inclusive prefix)
+    unsigned long long* mine = look + tile * kRadix + tid;
+    st_release_u64(mine, ((tile == 0 ? 2ull : 1ull) << 62) | cnt);
+    uint32_t ttot;
+    s_start[tid] = block_excl_scan_256(cnt, s_scan, &ttot);
+    __syncthreads();
+    // place keys in shared memory in (digit, rank) order
+#pragma unroll
+    for (int i = 0; i < kItems; ++i) {
+        const int64_t idx = wbase + i * 32 + lane;
+        if (idx < n) {
+            const uint32_t d = (key[i] >> shift) & 0xffu;
+            const uint32_t p = s_start[d] + s_whist[w][d] + rank[i];
+            s_keys[p] = key[i];
+            s_vals[p] = val[i];
+        }
+    }
     // decoupled lookback over earlier tiles for digit tid
     {
-        unsigned long long* mine = look + tile * kRadix + tid;
-        if (tile == 0) {
-            st_release_u64(mine, (2ull << 62) | cnt);
-        } else {
-            st_release_u64(mine, (1ull << 62) | cnt);
-        }
         unsigned long long excl = 0;
         if (tile > 0) {
             // read a window of kWin predecessors per round trip, newest first, and add
@@ -207,20 +218,6 @@ __global__ void __launch_bounds__(kNT) k_radix_pass(const float* __restrict__ a,
             st_release_u64(mine, (2ull << 62) | (excl + cnt));
         }
         s_base[tid] = gexcl + (uint32_t)excl;
-    }
-    uint32_t ttot;
-    s_start[tid] = block_excl_scan_256(cnt, s_scan, &ttot);
-    __syncthreads();
-    // place keys in shared memory in (digit, rank) order
-#pragma unroll
-    for (int i = 0; i < kItems; ++i) {
-        const int64_t idx = wbase + i * 32 + lane;
-        if (idx < n) {
-            const uint32_t d = (key[i] >> shift) & 0xffu;
-            const uint32_t p = s_start[d] + s_whist[w][d] + rank[i];
-            s_keys[p] = key[i];
-            s_vals[p] = val[i];
-        }
     }
     __syncthreads();
     const int valid_count = (n - base) < kTile ? (int)(n - base) : kTile;

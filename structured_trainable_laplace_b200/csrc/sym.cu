@@ -41,7 +41,7 @@ namespace {
 
 constexpr int kE = 16;
 constexpr int kMaxRanges = 8192;   // base ranges per channel group
-constexpr int kRangesPerSM = 12;   // base ranges per SM (divisible by the usual occupancies)
+constexpr int kRangesPerSM = 6;    // base ranges per SM (divisible by the usual occupancies)
 constexpr int kAheadFwd = 2;       // gathered-row prefetch distance: aggregate and forward sweeps
 constexpr int kAheadBwd = 1;       // backward sweep (two staged vectors)
 
@@ -207,6 +207,25 @@ __device__ __forceinline__ void group_scan(LP (&incL)[NV], LP (&incR)[NV], const
     }
 }
 
+// The same scans for the inclusive sums P alone (the forward product).
+template <int SK>
+__device__ __forceinline__ void group_scan_p(float& pl, float& pr, const SegTab<SK>& tb, int k) {
+#pragma unroll
+    for (int j = 0, off = 1; off < SK; ++j, off <<= 1) {
+        const float oL = __shfl_up_sync(0xffffffffu, pl, off, SK);
+        const float oR = __shfl_down_sync(0xffffffffu, pr, off, SK);
+        if (k >= off) pl = fmaf(fabsf(tb.gL[j][k]), oL, pl);
+        if (k + off < SK) pr = fmaf(fabsf(tb.gR[j][k]), oR, pr);
+    }
+}
+
+__device__ __forceinline__ float seg_in_p(bool has_carry, float carry, bool has_excl, float excl, float ev) {
+    if (has_carry && has_excl) return fmaf(fabsf(ev), carry, excl);
+    if (has_carry) return carry;
+    if (has_excl) return excl;
+    return 0.f;
+}
+
 // Tiles walked by CTA blockIdx.x: those of base ranges [J0, J1).
 struct CtaTiles {
     int J0, J1;
@@ -245,9 +264,13 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
     auto tile_of = [&](int i) { return w.te - 1 - i; };
     // anchor of the last row of base range J
     auto range_end = [&](int64_t J) { return __ldg(a.s + min(a.n, (J + 1) * a.tpr * (int64_t)R) - 1); };
-    auto tile_ed = [&](const float* sb, int64_t t, double* ed) {  // [0] right fold, [1] left fold
-        ed[0] = exp((double)sb[4] - (double)sb[4 + R]);
-        ed[1] = exp((double)sb[4 + R - 1] - (double)range_end(t / a.tpr));
+    // fp64 decays of the tile folds, negative for a tie (decay 1, no break): [0] right
+    // fold (-row after the tile -> -its first row), [1] left fold (the tile's last row
+    // -> its base range's last row)
+    auto tile_ed = [&](const float* sb, int64_t t, double* ed) {
+        const float ue = range_end(t / a.tpr);
+        ed[0] = (sb[4 + R] > sb[4]) ? exp((double)sb[4] - (double)sb[4 + R]) : -1.0;
+        ed[1] = (ue > sb[4 + R - 1]) ? exp((double)sb[4 + R - 1] - (double)ue) : -1.0;
     };
 #pragma unroll
     for (int q = 0; q <= AHEAD; ++q) {
@@ -296,9 +319,9 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
             const double* ed = sm.ed[i & 1];
             const bool last_of_range = (t + 1 == min(a.T, (J + 1) * a.tpr));  // the first one walked
             const double2 trd = to_d2(sr[0]), tld = to_d2(tl);
-            runR = last_of_range ? trd : combine_ed(runR, trd, ed[0], sb[4] < sb[4 + R]);
+            runR = last_of_range ? trd : combine_ed(runR, trd, fabs(ed[0]), ed[0] >= 0.0);
             st.RS[((int64_t)grp * a.T + t) * C + c] = runR;
-            runL = last_of_range ? tld : combine_ed(tld, runL, ed[1], range_end(J) > sb[4 + R - 1]);
+            runL = last_of_range ? tld : combine_ed(tld, runL, fabs(ed[1]), ed[1] >= 0.0);
             if (t == J * a.tpr) {  // first tile of the base range: its aggregates are complete
                 st.Lagg[((int64_t)grp * a.P + J) * C + c] = runL;
                 st.Ragg[((int64_t)grp * a.P + J) * C + c] = runR;
@@ -456,9 +479,13 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
     const int c = (threadIdx.x >> 5) * CW + cs, ch0 = grp * C;
     // oriented anchor of the row after base range J (where its right carry is anchored)
     auto u_rin = [&](int64_t J) { return -__ldg(a.s + min(a.n - 1, (J + 1) * a.tpr * (int64_t)R)); };
-    auto tile_ed = [&](const float* sb, int64_t t, double* ed) {  // [0] left fold, [1] right carry
-        ed[0] = exp((double)sb[3] - (double)sb[4 + R - 1]);
-        ed[1] = exp((double)u_rin(t / a.tpr) + (double)sb[4 + R]);
+    // fp64 decays of the tile folds, negative for a tie (decay 1, no break):
+    // [0] left fold (row before the tile -> its last row), [1] right carry (the row
+    // after the base range -> the row after the tile)
+    auto tile_ed = [&](const float* sb, int64_t t, double* ed) {
+        const float ur = u_rin(t / a.tpr);
+        ed[0] = (sb[4 + R - 1] > sb[3]) ? exp((double)sb[3] - (double)sb[4 + R - 1]) : -1.0;
+        ed[1] = (-sb[4 + R] > ur) ? exp((double)ur + (double)sb[4 + R]) : -1.0;
     };
 #pragma unroll
     for (int q = 0; q <= AHEAD; ++q) {
@@ -518,70 +545,96 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         float* vb[NV];
 #pragma unroll
         for (int w = 0; w < NV; ++w) vb[w] = sm.v[w][i % VS] + k * G::SEG + c;
-        // pass 1: segment summaries, then the scans over the channel's segments
-        LP sr[NV], sl[NV];
-#pragma unroll
-        for (int w = 0; w < NV; ++w) {
-            sr[w] = LP{0.f, 0.f};
-            sl[w] = LP{0.f, 0.f};
-#pragma unroll
-            for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dk[e + 1], 0.f, vb[w][e * C]);
-#pragma unroll
-            for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dk[e], 0.f, vb[w][e * C]);
-        }
-        group_scan<SK, NV>(sl, sr, tb, k);  // now inclusive over segments 0..k (left) / k..SK-1 (right)
-        // tile carries: the channel's first lane folds in fp64, then broadcasts
         const bool more = (t + 1 < min(a.T, (J + 1) * a.tpr)), hasRin = (J + 1 < a.P);
         const bool hl_tile = hasL, hr_tile = hasRin || more;
-        LP cL[NV], cR[NV];
-#pragma unroll
-        for (int w = 0; w < NV; ++w) {
-            const LP tl = shfl_lp(sl[w], SK - 1, SK);
-            cL[w] = LP{0.f, 0.f};
-            cR[w] = LP{0.f, 0.f};
-            if (k == 0) {
-                const double* ed = sm.ed[i & 1];
-                const double2 cl = runL[w];
-                double2 cr = hasRin ? sm.rin[i % MS][w][c] : make_double2(0.0, 0.0);
-                if (more) {
-                    const double2 rsn = sm.rs[i % MS][w][c];
-                    cr = hasRin ? combine_ed(cr, rsn, ed[1], -sb[4 + R] > u_rin(J)) : rsn;
-                }
-                cL[w] = LP{(float)cl.x, (float)cl.y};
-                cR[w] = LP{(float)cr.x, (float)cr.y};
-                const double2 tld = to_d2(tl);
-                runL[w] = hl_tile ? combine_ed(runL[w], tld, ed[0], sb[4 + R - 1] > sb[3]) : tld;
-            }
-            cL[w] = shfl_lp(cL[w], 0, SK);
-            cR[w] = shfl_lp(cR[w], 0, SK);
-        }
+        const double* ed = sm.ed[i & 1];
         hasL = true;
-        // incoming state of this segment: tile carry, then the segments before it
-        const float evl = tb.iL[k], evr = tb.iR[k];
-        LP inR[NV], inL[NV];
+        if constexpr (NV == 1) {
+            // forward: y = P + S - x needs only the inclusive sums (ties enter with decay 1)
+            float* xb = vb[0];
+            float pr = 0.f, pl = 0.f;
 #pragma unroll
-        for (int w = 0; w < NV; ++w) {
-            const LP exL = shfl_lp(sl[w], (lane - 1) & 31, 32), exR = shfl_lp(sr[w], (lane + 1) & 31, 32);
-            inL[w] = seg_in(hl_tile, cL[w], k >= 1, exL, evl);
-            inR[w] = seg_in(hr_tile, cR[w], k + 1 < SK, exR, evr);
-        }
-        // pass 2: results replace the staged values in place
-        if (NV == 1) {
+            for (int e = E - 1; e >= 0; --e) pr = fmaf(fabsf(dk[e + 1]), pr, xb[e * C]);
+#pragma unroll
+            for (int e = 0; e < E; ++e) pl = fmaf(fabsf(dk[e]), pl, xb[e * C]);
+            group_scan_p<SK>(pl, pr, tb, k);
+            // tile carries: the channel's first lane folds in fp64, then broadcasts
+            const float tl = __shfl_sync(0xffffffffu, pl, SK - 1, SK);
+            float cl = 0.f, cr = 0.f;
+            if (k == 0) {
+                double crd = hasRin ? sm.rin[i % MS][0][c].y : 0.0;
+                if (more) {
+                    const double rsn = sm.rs[i % MS][0][c].y;
+                    crd = hasRin ? fma(fabs(ed[1]), crd, rsn) : rsn;
+                }
+                cl = (float)runL[0].y;
+                cr = (float)crd;
+                runL[0].y = hl_tile ? fma(fabs(ed[0]), runL[0].y, (double)tl) : (double)tl;
+            }
+            cl = __shfl_sync(0xffffffffu, cl, 0, SK);
+            cr = __shfl_sync(0xffffffffu, cr, 0, SK);
+            // incoming state of this segment: tile carry, then the segments before it
+            const float exl = __shfl_sync(0xffffffffu, pl, (lane - 1) & 31);
+            const float exr = __shfl_sync(0xffffffffu, pr, (lane + 1) & 31);
+            float Pr = seg_in_p(hr_tile, cr, k + 1 < SK, exr, tb.iR[k]);
+            float Pl = seg_in_p(hl_tile, cl, k >= 1, exl, tb.iL[k]);
+            // pass 2: y replaces the staged x in place
             float yv[E];
-            float Pr = inR[0].P;
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
-                const float xe = vb[0][e * C];
-                Pr = fmaf(fabsf(dk[e + 1]), Pr, xe);  // only the inclusive sums are needed here
+                const float xe = xb[e * C];
+                Pr = fmaf(fabsf(dk[e + 1]), Pr, xe);
                 yv[e] = Pr - xe;
             }
-            float Pl = inL[0].P;
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                Pl = fmaf(fabsf(dk[e]), Pl, vb[0][e * C]);
-                vb[0][e * C] = yv[e] + Pl;
+                Pl = fmaf(fabsf(dk[e]), Pl, xb[e * C]);
+                xb[e * C] = yv[e] + Pl;
             }
         } else {
+            // backward: the strict sums L (and R) are needed for ga, so both scans
+            // carry (L, P)
+            LP sr[NV], sl[NV];
+#pragma unroll
+            for (int w = 0; w < NV; ++w) {
+                sr[w] = LP{0.f, 0.f};
+                sl[w] = LP{0.f, 0.f};
+#pragma unroll
+                for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dk[e + 1], 0.f, vb[w][e * C]);
+#pragma unroll
+                for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dk[e], 0.f, vb[w][e * C]);
+            }
+            group_scan<SK, NV>(sl, sr, tb, k);  // now inclusive over segments 0..k (left) / k..SK-1 (right)
+            LP cL[NV], cR[NV];
+#pragma unroll
+            for (int w = 0; w < NV; ++w) {
+                const LP tl = shfl_lp(sl[w], SK - 1, SK);
+                cL[w] = LP{0.f, 0.f};
+                cR[w] = LP{0.f, 0.f};
+                if (k == 0) {
+                    const double2 cl = runL[w];
+                    double2 cr = hasRin ? sm.rin[i % MS][w][c] : make_double2(0.0, 0.0);
+                    if (more) {
+                        const double2 rsn = sm.rs[i % MS][w][c];
+                        cr = hasRin ? combine_ed(cr, rsn, fabs(ed[1]), ed[1] >= 0.0) : rsn;
+                    }
+                    cL[w] = LP{(float)cl.x, (float)cl.y};
+                    cR[w] = LP{(float)cr.x, (float)cr.y};
+                    const double2 tld = to_d2(tl);
+                    runL[w] = hl_tile ? combine_ed(runL[w], tld, fabs(ed[0]), ed[0] >= 0.0) : tld;
+                }
+                cL[w] = shfl_lp(cL[w], 0, SK);
+                cR[w] = shfl_lp(cR[w], 0, SK);
+            }
+            const float evl = tb.iL[k], evr = tb.iR[k];
+            LP inR[NV], inL[NV];
+#pragma unroll
+            for (int w = 0; w < NV; ++w) {
+                const LP exL = shfl_lp(sl[w], (lane - 1) & 31, 32), exR = shfl_lp(sr[w], (lane + 1) & 31, 32);
+                inL[w] = seg_in(hl_tile, cL[w], k >= 1, exL, evl);
+                inR[w] = seg_in(hr_tile, cR[w], k + 1 < SK, exR, evr);
+            }
+            // pass 2: gx replaces the staged x in place; ga goes to the per-warp sums
             float gxp[E], gap[E];
             LP ax = inR[0], ag = inR[NV - 1];
 #pragma unroll
@@ -612,30 +665,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         __syncthreads();
         // coalesced stores of whole rows through the permutation
         const uint32_t* pb = sm.p[i % MS];
-        if (out != nullptr) {
-            constexpr int W = (G::VW > 1) ? G::VW : 1;
-            const float* ob = sm.v[0][i % VS];
-            if (W > 1 && (a.B % W) == 0) {
-                constexpr int Q = G::C >= W ? G::C / W : 1;
-                for (int q = threadIdx.x; q < R * Q; q += NT) {
-                    const int r = q / Q, cc = (q % Q) * W;
-                    if (lo + r < a.n && ch0 + cc < a.B) {
-                        float* dst = out + (int64_t)min(pb[r], (uint32_t)(a.n - 1)) * a.B + ch0 + cc;
-                        const float* sp = ob + G::xidx(r, cc);
-                        if (W == 4)
-                            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(sp);
-                        else
-                            *reinterpret_cast<float2*>(dst) = *reinterpret_cast<const float2*>(sp);
-                    }
-                }
-            } else {
-                for (int q = threadIdx.x; q < R * C; q += NT) {
-                    const int r = q / C, cc = q % C;
-                    if (lo + r < a.n && ch0 + cc < a.B)
-                        out[(int64_t)min(pb[r], (uint32_t)(a.n - 1)) * a.B + ch0 + cc] = ob[G::xidx(r, cc)];
-                }
-            }
-        }
+        if (out != nullptr) store_rows<G>(out, a.B, ch0, a.n, lo, pb, sm.v[0][i % VS]);
         if (NV == 2 && ga != nullptr) {
             for (int r = threadIdx.x; r < R; r += NT) {
                 if (lo + r >= a.n) continue;
