@@ -166,9 +166,11 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
         s_whist[j][tid] = cnt;
         cnt += c;
     }
-    // publish this tile's count for digit tid (tile 0's is already its inclusive prefix)
+    // publish this tile's count for digit tid (tile 0's is already its inclusive prefix);
+    // a lookback word carries its own status bits and nothing else is read on the
+    // strength of it, so relaxed stores and loads suffice
     unsigned long long* mine = look + tile * kRadix + tid;
-    st_release_u64(mine, ((tile == 0 ? 2ull : 1ull) << 62) | cnt);
+    st_relaxed_u64(mine, ((tile == 0 ? 2ull : 1ull) << 62) | cnt);
     uint32_t ttot;
     s_start[tid] = block_excl_scan_256(cnt, s_scan, &ttot);
     __syncthreads();
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
                 }
                 j -= kWin;
             }
-            st_release_u64(mine, (2ull << 62) | (excl + cnt));
+            st_relaxed_u64(mine, (2ull << 62) | (excl + cnt));
         }
         s_base[tid] = gexcl + (uint32_t)excl;
     }

@@ -42,8 +42,9 @@ namespace {
 constexpr int kE = 16;
 constexpr int kMaxRanges = 8192;   // base ranges per channel group
 constexpr int kRangesPerSM = 6;    // base ranges per SM (divisible by the usual occupancies)
-constexpr int kAheadFwd = 2;       // gathered-row prefetch distance: aggregate and forward sweeps
-constexpr int kAheadBwd = 1;       // backward sweep (two staged vectors)
+constexpr int kAheadAgg = 2;       // prefetch distance of the gathered rows (aggregate pass)
+constexpr int kAheadFwd = 1;       // of the streamed sorted tiles: forward sweep
+constexpr int kAheadBwd = 1;       // backward sweep (two streamed vectors)
 
 template <int C>
 struct SymGeo {
@@ -159,22 +160,63 @@ struct RangeState {
     double2* Rin;   // [G][P][C]  carry from the ranges after (anchored at -the row after)
 };
 
-template <int C, int NV, int AHEAD>
-struct SymSmem {
+// Shared memory of the aggregate pass, which gathers rows through the permutation.
+template <int C, int AHEAD>
+struct AggSmem {
     using G = typename SymGeo<C>::G;
-    static constexpr int MS = AHEAD + 2;  // anchor / permutation / carry slots
+    static constexpr int MS = AHEAD + 2;  // anchor / permutation slots
     static constexpr int VS = AHEAD + 1;  // gathered-row slots
     float s[MS][G::SS];
     uint32_t p[MS][G::R];
-    double2 rs[MS][NV][C];   // RS[t+1] (sweep)
-    double2 rin[MS][NV][C];  // carry entering the tile's base range from the right (sweep)
-    float v[NV][VS][G::XS];
+    float v[1][VS][G::XS];
     SegTab<SymGeo<C>::SK> tab[2];  // decay tables of the current and the next tile
     double ed[2][2];               // fp64 decays of the two tile-level folds, current and next tile
+};
+
+// Shared memory of the sweeps, which stream the sorted copies written by the
+// aggregate pass (see SortedTile) instead of gathering rows.
+template <int C, int NV, int AHEAD>
+struct SweepSmem {
+    using SG = SymGeo<C>;
+    using G = typename SG::G;
+    static constexpr int MS = AHEAD + 2;      // anchor / permutation / carry slots
+    static constexpr int VS = AHEAD + 1;      // sorted-tile slots
+    static constexpr int KS = C * kE + 4;     // floats per staged segment (4 of padding)
+    static constexpr int TS = SG::SK * KS;    // floats per staged sorted tile
+    float s[MS][G::SS];
+    uint32_t p[MS][G::R];
+    double2 rs[MS][NV][C];   // RS[t+1]
+    double2 rin[MS][NV][C];  // carry entering the tile's base range from the right
+    alignas(16) float v[NV][VS][TS];
+    float o[G::XS];          // output rows (y or gx) in the gathered layout, for the scatter
+    SegTab<SG::SK> tab[2];   // decay tables of the current and the next tile
+    double ed[2][2];         // fp64 decays of the two tile-level folds, current and next tile
     // backward: per-warp sums of the ga shares of the warp's channels, rows padded
     // as in SegTab::d
-    float gp[NV == 2 ? SymGeo<C>::NW : 1][NV == 2 ? SymGeo<C>::SK * (kE + 1) : 1];
+    float gp[NV == 2 ? SG::NW : 1][NV == 2 ? SG::SK * (kE + 1) : 1];
 };
+
+// Sorted copy of one vector: tile t of channel group grp is R*C contiguous floats
+// holding the value of sorted row k*E + e, channel c, at [k][c][e], so that each
+// lane's E values are contiguous.  Rows past n and channels past B hold zero.
+template <class F>
+__device__ __forceinline__ F* sorted_tile(F* vs, int grp, int64_t T, int64_t t, int R, int C) {
+    return vs + ((int64_t)grp * T + t) * (int64_t)R * C;
+}
+
+// Start copying one sorted tile into the staged segment-major layout (16-byte
+// copies; KS-float segment stride keeps the lanes' 16-byte reads conflict-free).
+template <int C>
+__device__ __forceinline__ void stage_sorted(const float* __restrict__ src, float* dst) {
+    using SG = SymGeo<C>;
+    constexpr int SEGF = C * kE, KS = SEGF + 4, NCOPY = SG::SK * SEGF / 4;
+    static_assert(NCOPY % SG::NT == 0, "whole copies per thread");
+#pragma unroll
+    for (int q = 0; q < NCOPY / SG::NT; ++q) {
+        const int f = 4 * (threadIdx.x + q * SG::NT), k = f / SEGF;
+        cp_async16(dst + k * KS + (f - k * SEGF), src + f);
+    }
+}
 
 __device__ __forceinline__ int64_t tile_lo(int64_t t, int R) { return t * (int64_t)R; }
 
@@ -249,10 +291,10 @@ __device__ __forceinline__ CtaTiles cta_tiles(const SymScan& a) {
 // its first.
 template <int C, int AHEAD>
 __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
-    k_sym_agg(SymScan a, const float* __restrict__ v, RangeState st) {
+    k_sym_agg(SymScan a, const float* __restrict__ v, RangeState st, float* __restrict__ vs) {
     using SG = SymGeo<C>;
     using G = typename SG::G;
-    using SM = SymSmem<C, 1, AHEAD>;
+    using SM = AggSmem<C, AHEAD>;
     constexpr int E = kE, R = G::R, SK = SG::SK, CW = SG::CW, MS = SM::MS, VS = SM::VS;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SM& sm = *reinterpret_cast<SM*>(smem_raw);
@@ -308,11 +350,19 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
         const SegTab<SK>& tb = sm.tab[i & 1];
         const float* dk = tb.d[k];
         const float* xb = sm.v[0][i % VS] + k * G::SEG + c;
+        float xv[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) xv[e] = xb[e * C];
+        {  // this lane's E values of the sorted copy
+            float4* dst = reinterpret_cast<float4*>(sorted_tile(vs, grp, a.T, t, R, C) + (k * C + c) * E);
+#pragma unroll
+            for (int q = 0; q < E / 4; ++q) dst[q] = make_float4(xv[4 * q], xv[4 * q + 1], xv[4 * q + 2], xv[4 * q + 3]);
+        }
         LP sr[1] = {{0.f, 0.f}}, sl[1] = {{0.f, 0.f}};
 #pragma unroll
-        for (int e = E - 1; e >= 0; --e) sr[0] = lp_step_d(sr[0], dk[e + 1], 0.f, xb[e * C]);
+        for (int e = E - 1; e >= 0; --e) sr[0] = lp_step_d(sr[0], dk[e + 1], 0.f, xv[e]);
 #pragma unroll
-        for (int e = 0; e < E; ++e) sl[0] = lp_step_d(sl[0], dk[e], 0.f, xb[e * C]);
+        for (int e = 0; e < E; ++e) sl[0] = lp_step_d(sl[0], dk[e], 0.f, xv[e]);
         group_scan<SK, 1>(sl, sr, tb, k);
         const LP tl = shfl_lp(sl[0], SK - 1, SK);  // tile totals: left at the last segment, right at the first
         if (k == 0) {
@@ -462,14 +512,15 @@ __device__ __forceinline__ void stage_carries(const SymScan& a, const RangeState
 }
 
 // NV = 1: forward (x -> y = out).  NV = 2: backward (x, g -> gx = out, ga).
+// xs / gs are the sorted copies of x and g that the aggregate passes wrote.
 template <int C, int NV, int AHEAD>
 __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 1 ? 3 : 2) : 1)) k_sym_sweep(
-    SymScan a, const float* __restrict__ x, const float* __restrict__ g, RangeState sx, RangeState sg,
+    SymScan a, const float* __restrict__ xs, const float* __restrict__ gs, RangeState sx, RangeState sg,
     float* __restrict__ out, float* __restrict__ ga, int ga_atomic) {
     using SG = SymGeo<C>;
     using G = typename SG::G;
-    using SM = SymSmem<C, NV, AHEAD>;
-    constexpr int E = kE, R = G::R, SK = SG::SK, CW = SG::CW, NT = SG::NT, MS = SM::MS, VS = SM::VS;
+    using SM = SweepSmem<C, NV, AHEAD>;
+    constexpr int E = kE, R = G::R, SK = SG::SK, CW = SG::CW, NT = SG::NT, MS = SM::MS, VS = SM::VS, KS = SM::KS;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SM& sm = *reinterpret_cast<SM*>(smem_raw);
     const int grp = blockIdx.y;
@@ -487,6 +538,10 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         ed[0] = (sb[4 + R - 1] > sb[3]) ? exp((double)sb[3] - (double)sb[4 + R - 1]) : -1.0;
         ed[1] = (-sb[4 + R] > ur) ? exp((double)ur + (double)sb[4 + R]) : -1.0;
     };
+    auto stage_vecs = [&](int64_t tt, int slot) {
+#pragma unroll
+        for (int w = 0; w < NV; ++w) stage_sorted<C>(sorted_tile(w == 0 ? xs : gs, grp, a.T, tt, R, C), sm.v[w][slot]);
+    };
 #pragma unroll
     for (int q = 0; q <= AHEAD; ++q) {
         if (q < nt) {
@@ -499,11 +554,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < AHEAD; ++q) {
-        if (q < nt) {
-#pragma unroll
-            for (int w = 0; w < NV; ++w)
-                stage_rows<G>(w == 0 ? x : g, a.B, ch0, a.n, tile_lo(cw.tb + q, R), sm.p[q % MS], sm.v[w][q % VS]);
-        }
+        if (q < nt) stage_vecs(cw.tb + q, q % VS);
         cp_async_commit();
     }
     seg_tables<SK, NT>(sm.s[0], sm.tab[0]);
@@ -528,35 +579,40 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                                  sm.rin[(i + AHEAD + 1) % MS]);
         }
         cp_async_commit();
-        if (i + AHEAD < nt) {
-#pragma unroll
-            for (int w = 0; w < NV; ++w)
-                stage_rows<G>(w == 0 ? x : g, a.B, ch0, a.n, tile_lo(t + AHEAD, R), sm.p[(i + AHEAD) % MS],
-                              sm.v[w][(i + AHEAD) % VS]);
-        }
+        if (i + AHEAD < nt) stage_vecs(t + AHEAD, (i + AHEAD) % VS);
         cp_async_commit();
         if (i + 1 < nt) {
             seg_tables<SK, NT>(sm.s[(i + 1) % MS], sm.tab[(i + 1) & 1]);
             if (threadIdx.x == 0) tile_ed(sm.s[(i + 1) % MS], t + 1, sm.ed[(i + 1) & 1]);
         }
-        const float* sb = sm.s[i % MS];
         const SegTab<SK>& tb = sm.tab[i & 1];
         const float* dk = tb.d[k];
-        float* vb[NV];
-#pragma unroll
-        for (int w = 0; w < NV; ++w) vb[w] = sm.v[w][i % VS] + k * G::SEG + c;
+        float* ob = sm.o + k * G::SEG + c;  // this lane's output column (gathered layout)
         const bool more = (t + 1 < min(a.T, (J + 1) * a.tpr)), hasRin = (J + 1 < a.P);
         const bool hl_tile = hasL, hr_tile = hasRin || more;
         const double* ed = sm.ed[i & 1];
         hasL = true;
+        // this lane's E values of each vector (segment k, channel c)
+        float xr[NV][E];
+#pragma unroll
+        for (int w = 0; w < NV; ++w) {
+            const float4* src = reinterpret_cast<const float4*>(sm.v[w][i % VS] + k * KS + c * E);
+#pragma unroll
+            for (int q = 0; q < E / 4; ++q) {
+                const float4 f = src[q];
+                xr[w][4 * q] = f.x;
+                xr[w][4 * q + 1] = f.y;
+                xr[w][4 * q + 2] = f.z;
+                xr[w][4 * q + 3] = f.w;
+            }
+        }
         if constexpr (NV == 1) {
             // forward: y = P + S - x needs only the inclusive sums (ties enter with decay 1)
-            float* xb = vb[0];
             float pr = 0.f, pl = 0.f;
 #pragma unroll
-            for (int e = E - 1; e >= 0; --e) pr = fmaf(fabsf(dk[e + 1]), pr, xb[e * C]);
+            for (int e = E - 1; e >= 0; --e) pr = fmaf(fabsf(dk[e + 1]), pr, xr[0][e]);
 #pragma unroll
-            for (int e = 0; e < E; ++e) pl = fmaf(fabsf(dk[e]), pl, xb[e * C]);
+            for (int e = 0; e < E; ++e) pl = fmaf(fabsf(dk[e]), pl, xr[0][e]);
             group_scan_p<SK>(pl, pr, tb, k);
             // tile carries: the channel's first lane folds in fp64, then broadcasts
             const float tl = __shfl_sync(0xffffffffu, pl, SK - 1, SK);
@@ -578,18 +634,17 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
             const float exr = __shfl_sync(0xffffffffu, pr, (lane + 1) & 31);
             float Pr = seg_in_p(hr_tile, cr, k + 1 < SK, exr, tb.iR[k]);
             float Pl = seg_in_p(hl_tile, cl, k >= 1, exl, tb.iL[k]);
-            // pass 2: y replaces the staged x in place
+            // pass 2
             float yv[E];
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
-                const float xe = xb[e * C];
-                Pr = fmaf(fabsf(dk[e + 1]), Pr, xe);
-                yv[e] = Pr - xe;
+                Pr = fmaf(fabsf(dk[e + 1]), Pr, xr[0][e]);
+                yv[e] = Pr - xr[0][e];
             }
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                Pl = fmaf(fabsf(dk[e]), Pl, xb[e * C]);
-                xb[e * C] = yv[e] + Pl;
+                Pl = fmaf(fabsf(dk[e]), Pl, xr[0][e]);
+                ob[e * C] = yv[e] + Pl;
             }
         } else {
             // backward: the strict sums L (and R) are needed for ga, so both scans
@@ -600,9 +655,9 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 sr[w] = LP{0.f, 0.f};
                 sl[w] = LP{0.f, 0.f};
 #pragma unroll
-                for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dk[e + 1], 0.f, vb[w][e * C]);
+                for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dk[e + 1], 0.f, xr[w][e]);
 #pragma unroll
-                for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dk[e], 0.f, vb[w][e * C]);
+                for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dk[e], 0.f, xr[w][e]);
             }
             group_scan<SK, NV>(sl, sr, tb, k);  // now inclusive over segments 0..k (left) / k..SK-1 (right)
             LP cL[NV], cR[NV];
@@ -634,12 +689,12 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 inL[w] = seg_in(hl_tile, cL[w], k >= 1, exL, evl);
                 inR[w] = seg_in(hr_tile, cR[w], k + 1 < SK, exR, evr);
             }
-            // pass 2: gx replaces the staged x in place; ga goes to the per-warp sums
+            // pass 2: gx to the output rows, ga to the per-warp sums
             float gxp[E], gap[E];
             LP ax = inR[0], ag = inR[NV - 1];
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
-                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dk[e + 1];
+                const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e + 1];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
                 gxp[e] = ag.P - ge;
@@ -649,10 +704,10 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
             ag = inL[NV - 1];
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                const float xe = vb[0][e * C], ge = vb[NV - 1][e * C], dv = dk[e];
+                const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
-                vb[0][e * C] = gxp[e] + ag.P;              // gx
+                ob[e * C] = gxp[e] + ag.P;                    // gx
                 gap[e] = gap[e] - fmaf(ge, ax.L, xe * ag.L);  // this channel's share of ga
             }
             // sum over the warp's channels, then one padded row per warp in shared memory
@@ -665,7 +720,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         __syncthreads();
         // coalesced stores of whole rows through the permutation
         const uint32_t* pb = sm.p[i % MS];
-        if (out != nullptr) store_rows<G>(out, a.B, ch0, a.n, lo, pb, sm.v[0][i % VS]);
+        if (out != nullptr) store_rows<G>(out, a.B, ch0, a.n, lo, pb, sm.o);
         if (NV == 2 && ga != nullptr) {
             for (int r = threadIdx.x; r < R; r += NT) {
                 if (lo + r >= a.n) continue;
@@ -688,6 +743,9 @@ struct SymPlan {
     int C, G, P;
     int64_t R, T, tpr;
     size_t rs_elems, rng_elems;  // double2 counts of one RS array / one range array
+    size_t state_bytes;          // RS, Lin, Rin, Lagg, Ragg of one vector
+    size_t saved_state_bytes;    // RS, Lin, Rin of one vector
+    size_t sorted_bytes;         // sorted copy of one vector (G * T * R * C floats)
     size_t total;
 };
 
@@ -703,8 +761,11 @@ SymPlan plan_sym(int64_t n, int64_t B, int sms) {
     p.P = (int)((p.T + p.tpr - 1) / p.tpr);
     p.rs_elems = (size_t)p.G * p.T * p.C;
     p.rng_elems = (size_t)p.G * kMaxRanges * p.C;
-    // per vector: RS, Lin, Rin, Lagg, Ragg; two vectors (x, g)
-    p.total = 2 * align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
+    p.state_bytes = align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
+    p.saved_state_bytes = align_up(sizeof(double2) * (p.rs_elems + 2 * p.rng_elems), 256);
+    p.sorted_bytes = align_up(sizeof(float) * (size_t)p.G * p.T * p.R * p.C, 256);
+    // per vector (x, g): the scan state and the sorted copy
+    p.total = 2 * (p.state_bytes + p.sorted_bytes);
     return p;
 }
 
@@ -756,14 +817,14 @@ SymScan scan_args(const SymPlan& p, const float* s, const uint32_t* perm, int64_
 // Pass A + pass B for one vector.
 template <int C>
 cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms,
-                         const float* v, RangeState st, cudaStream_t stream) {
-    using SM = SymSmem<C, 1, kAheadFwd>;
+                         const float* v, RangeState st, float* vs, cudaStream_t stream) {
+    using SM = AggSmem<C, kAheadAgg>;
     static int occ_cache = 0;
-    const int occ = prepare(k_sym_agg<C, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+    const int occ = prepare(k_sym_agg<C, kAheadAgg>, SymGeo<C>::NT, sizeof(SM), occ_cache);
     const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
     const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
     LAPLEX_TIMED("sym_agg", stream,
-                 k_sym_agg<C, kAheadFwd><<<grid, SymGeo<C>::NT, sizeof(SM), stream>>>(a, v, st));
+                 k_sym_agg<C, kAheadAgg><<<grid, SymGeo<C>::NT, sizeof(SM), stream>>>(a, v, st, vs));
     LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, kCarryThreads, 0, stream>>>(a, st));
     return cudaGetLastError();
 }
@@ -774,22 +835,24 @@ cudaError_t sym_forward_t(const float* s, const uint32_t* perm, int64_t n, const
     const int sms = device_sms();
     const SymPlan p = plan_sym(n, B, sms);
     RangeState sx = carve(p, (double2*)ws, true);
-    if (saved != nullptr) {  // RS and carries go to the caller's buffer; aggregates stay in ws
+    float* xs = (float*)((char*)ws + 2 * p.state_bytes);
+    if (saved != nullptr) {  // RS, carries and the sorted copy go to the caller's buffer
         const RangeState sv = carve(p, (double2*)saved, false);
         sx.RS = sv.RS;
         sx.Lin = sv.Lin;
         sx.Rin = sv.Rin;
+        xs = (float*)((char*)saved + p.saved_state_bytes);
     }
-    cudaError_t e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, st);
+    cudaError_t e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
     if (e != cudaSuccess) return e;
-    using SM = SymSmem<C, 1, kAheadFwd>;
+    using SM = SweepSmem<C, 1, kAheadFwd>;
     static int occ_cache = 0;
     const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
     const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
     const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
     LAPLEX_TIMED("sym_fwd", st,
                  k_sym_sweep<C, 1, kAheadFwd>
-                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, x, nullptr, sx, sx, y, nullptr, 0));
+                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, nullptr, sx, sx, y, nullptr, 0));
     return cudaGetLastError();
 }
 
@@ -798,14 +861,16 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
                            const void* saved, float* gx, float* ga, void* ws, cudaStream_t st) {
     const int sms = device_sms();
     const SymPlan p = plan_sym(n, B, sms);
-    const size_t half = align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
     RangeState sx = carve(p, (double2*)ws, true);
-    const RangeState sg = carve(p, (double2*)((char*)ws + half), true);
+    const RangeState sg = carve(p, (double2*)((char*)ws + p.state_bytes), true);
+    float* xs = (float*)((char*)ws + 2 * p.state_bytes);
+    float* gs = (float*)((char*)xs + p.sorted_bytes);
     if (saved != nullptr) {
         const RangeState sv = carve(p, (double2*)saved, false);
         sx.RS = sv.RS;
         sx.Lin = sv.Lin;
         sx.Rin = sv.Rin;
+        xs = (float*)((char*)saved + p.saved_state_bytes);
     }
     cudaError_t e;
     if (ga != nullptr && p.G > 1) {
@@ -813,19 +878,19 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
         if (e != cudaSuccess) return e;
     }
     if (saved == nullptr) {
-        e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, st);
+        e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
         if (e != cudaSuccess) return e;
     }
-    e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, st);
+    e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, gs, st);
     if (e != cudaSuccess) return e;
-    using SM = SymSmem<C, 2, kAheadBwd>;
+    using SM = SweepSmem<C, 2, kAheadBwd>;
     static int occ_cache = 0;
     const int occ = prepare(k_sym_sweep<C, 2, kAheadBwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
     const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
     const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
     LAPLEX_TIMED("sym_bwd", st,
                  k_sym_sweep<C, 2, kAheadBwd>
-                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, x, g, sx, sg, gx, ga, p.G > 1 ? 1 : 0));
+                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, gs, sx, sg, gx, ga, p.G > 1 ? 1 : 0));
     return cudaGetLastError();
 }
 
@@ -835,7 +900,7 @@ size_t sym_workspace_bytes(int64_t n, int64_t B) { return plan_sym(n, B, 1).tota
 
 size_t sym_saved_bytes(int64_t n, int64_t B) {
     const SymPlan p = plan_sym(n, B, 1);
-    return sizeof(double2) * (p.rs_elems + 2 * p.rng_elems);
+    return p.saved_state_bytes + p.sorted_bytes;
 }
 
 #define LAPLEX_SYM_DISPATCH(C_, CALL) \
