@@ -22,6 +22,51 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
 }
 
+// L2 eviction priorities (createpolicy).  Data streamed through once is marked
+// evict-first, so that lines written piecewise elsewhere (scattered 4-byte
+// gradient rows) stay in L2 until they are complete instead of being written back
+// half-filled.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem, uint64_t pol) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 4, %2;" ::"r"(s), "l"(gmem), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem, uint64_t pol) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 8, %2;" ::"r"(s), "l"(gmem), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, uint64_t pol) {
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_hint(float* p, float v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_hint(float2* p, float2 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v2.f32 [%0], {%1, %2}, %3;" ::"l"(p), "f"(v.x), "f"(v.y), "l"(pol) : "memory");
+}
+
+__device__ __forceinline__ void st_hint(float4* p, float4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
@@ -56,12 +101,12 @@ struct TileGeo {
 // of one tile; rows outside [0, n) get sentinels (plain stores).
 template <class G>
 __device__ __forceinline__ void stage_meta(const float* __restrict__ s, const uint32_t* __restrict__ perm, int64_t n,
-                                           int64_t lo, float* s_buf, uint32_t* p_buf) {
+                                           int64_t lo, float* s_buf, uint32_t* p_buf, uint64_t pol) {
     for (int r = threadIdx.x; r < G::R; r += G::NT) {
         const int64_t g = lo + r;
         if (g < n) {
-            cp_async4(s_buf + 4 + r, s + g);
-            cp_async4(p_buf + r, perm + g);
+            cp_async4(s_buf + 4 + r, s + g, pol);
+            cp_async4(p_buf + r, perm + g, pol);
         } else {
             s_buf[4 + r] = kHighAnchor;
             p_buf[r] = 0u;
@@ -69,13 +114,13 @@ __device__ __forceinline__ void stage_meta(const float* __restrict__ s, const ui
     }
     if (threadIdx.x == 0) {
         if (lo > 0)
-            cp_async4(s_buf + 3, s + lo - 1);
+            cp_async4(s_buf + 3, s + lo - 1, pol);
         else
             s_buf[3] = kLowAnchor;
     }
     if (threadIdx.x == G::NT - 1) {
         if (lo + G::R < n)
-            cp_async4(s_buf + 4 + G::R, s + lo + G::R);
+            cp_async4(s_buf + 4 + G::R, s + lo + G::R, pol);
         else
             s_buf[4 + G::R] = kHighAnchor;
     }
@@ -105,7 +150,7 @@ struct RowWalk {
 // else 4 bytes.  Rows past n and channels past B are staged as zero.
 template <class G, int W>
 __device__ __forceinline__ void stage_rows_w(const float* __restrict__ v, int B, int ch0, int64_t n, int64_t lo,
-                                             const uint32_t* p_buf, float* x_buf) {
+                                             const uint32_t* p_buf, float* x_buf, uint64_t pol) {
     const RowWalk<G, W> wk;
     const int rem = (int)((n - lo) < (int64_t)G::R ? (n - lo) : (int64_t)G::R);
     const uint32_t last = (uint32_t)(n - 1);
@@ -119,11 +164,11 @@ __device__ __forceinline__ void stage_rows_w(const float* __restrict__ v, int B,
         if (r < rem && cok) {
             const float* src = src0 + (size_t)min(p_buf[r], last) * B;
             if constexpr (W == 4)
-                cp_async16(dst, src);
+                cp_async16(dst, src, pol);
             else if constexpr (W == 2)
-                cp_async8(dst, src);
+                cp_async8(dst, src, pol);
             else
-                cp_async4(dst, src);
+                cp_async4(dst, src, pol);
         } else {
 #pragma unroll
             for (int q = 0; q < W; ++q) dst[q] = 0.f;
@@ -133,18 +178,18 @@ __device__ __forceinline__ void stage_rows_w(const float* __restrict__ v, int B,
 
 template <class G>
 __device__ __forceinline__ void stage_rows(const float* __restrict__ v, int B, int ch0, int64_t n, int64_t lo,
-                                           const uint32_t* p_buf, float* x_buf) {
+                                           const uint32_t* p_buf, float* x_buf, uint64_t pol) {
     if (G::VW > 1 && (B % G::VW) == 0)
-        stage_rows_w<G, G::VW>(v, B, ch0, n, lo, p_buf, x_buf);
+        stage_rows_w<G, G::VW>(v, B, ch0, n, lo, p_buf, x_buf, pol);
     else
-        stage_rows_w<G, 1>(v, B, ch0, n, lo, p_buf, x_buf);
+        stage_rows_w<G, 1>(v, B, ch0, n, lo, p_buf, x_buf, pol);
 }
 
 // Store a staged tile back to the rows perm[lo + r] of out [n][B] (the inverse
 // of stage_rows; rows past n and channels past B are skipped).
 template <class G, int W>
 __device__ __forceinline__ void store_rows_w(float* __restrict__ out, int B, int ch0, int64_t n, int64_t lo,
-                                             const uint32_t* p_buf, const float* x_buf) {
+                                             const uint32_t* p_buf, const float* x_buf, uint64_t pol) {
     const RowWalk<G, W> wk;
     const int rem = (int)((n - lo) < (int64_t)G::R ? (n - lo) : (int64_t)G::R);
     const uint32_t last = (uint32_t)(n - 1);
@@ -157,21 +202,21 @@ __device__ __forceinline__ void store_rows_w(float* __restrict__ out, int B, int
         float* dst = dst0 + (size_t)min(p_buf[r], last) * B;
         const float* sp = x_buf + wk.off(it);
         if constexpr (W == 4)
-            *reinterpret_cast<float4*>(dst) = *reinterpret_cast<const float4*>(sp);
+            st_hint(reinterpret_cast<float4*>(dst), *reinterpret_cast<const float4*>(sp), pol);
         else if constexpr (W == 2)
-            *reinterpret_cast<float2*>(dst) = *reinterpret_cast<const float2*>(sp);
+            st_hint(reinterpret_cast<float2*>(dst), *reinterpret_cast<const float2*>(sp), pol);
         else
-            *dst = *sp;
+            st_hint(dst, *sp, pol);
     }
 }
 
 template <class G>
 __device__ __forceinline__ void store_rows(float* __restrict__ out, int B, int ch0, int64_t n, int64_t lo,
-                                           const uint32_t* p_buf, const float* x_buf) {
+                                           const uint32_t* p_buf, const float* x_buf, uint64_t pol) {
     if (G::VW > 1 && (B % G::VW) == 0)
-        store_rows_w<G, G::VW>(out, B, ch0, n, lo, p_buf, x_buf);
+        store_rows_w<G, G::VW>(out, B, ch0, n, lo, p_buf, x_buf, pol);
     else
-        store_rows_w<G, 1>(out, B, ch0, n, lo, p_buf, x_buf);
+        store_rows_w<G, 1>(out, B, ch0, n, lo, p_buf, x_buf, pol);
 }
 
 // Encoded decay between two oriented anchors uA <= uB: exp(uA - uB) when uB > uA

@@ -42,7 +42,7 @@ namespace {
 constexpr int kE = 16;
 constexpr int kMaxRanges = 8192;   // base ranges per channel group
 constexpr int kRangesPerSM = 6;    // base ranges per SM (divisible by the usual occupancies)
-constexpr int kAheadAgg = 2;       // prefetch distance of the gathered rows (aggregate pass)
+constexpr int kAheadAgg = 3;       // prefetch distance of the gathered rows (aggregate pass)
 constexpr int kAheadFwd = 1;       // of the streamed sorted tiles: forward sweep
 constexpr int kAheadBwd = 1;       // backward sweep (two streamed vectors)
 
@@ -52,7 +52,10 @@ struct SymGeo {
     static constexpr int NT = NW * 32;
     static constexpr int CW = C / NW;  // channels per warp
     static constexpr int SK = 32 / CW;  // segments per channel = lanes per channel group
-    using G = TileGeo<C, NT, kE, CW>;
+    // staged rows padded by CW floats per segment (conflict-free column reads), or
+    // by 4 when CW = 2, which keeps the rows 16-byte aligned for 16-byte copies at
+    // the price of 2-way conflicts
+    using G = TileGeo<C, NT, kE, (CW == 2 ? 4 : CW)>;
     static constexpr int R = G::R;  // rows per tile (SK * E)
 };
 
@@ -164,7 +167,8 @@ struct RangeState {
 template <int C, int AHEAD>
 struct AggSmem {
     using G = typename SymGeo<C>::G;
-    static constexpr int MS = AHEAD + 2;  // anchor / permutation slots
+    static constexpr int MA = AHEAD + 2;  // anchors and permutation are staged MA tiles ahead
+    static constexpr int MS = MA + 1;     // anchor / permutation slots
     static constexpr int VS = AHEAD + 1;  // gathered-row slots
     float s[MS][G::SS];
     uint32_t p[MS][G::R];
@@ -207,14 +211,14 @@ __device__ __forceinline__ F* sorted_tile(F* vs, int grp, int64_t T, int64_t t, 
 // Start copying one sorted tile into the staged segment-major layout (16-byte
 // copies; KS-float segment stride keeps the lanes' 16-byte reads conflict-free).
 template <int C>
-__device__ __forceinline__ void stage_sorted(const float* __restrict__ src, float* dst) {
+__device__ __forceinline__ void stage_sorted(const float* __restrict__ src, float* dst, uint64_t pol) {
     using SG = SymGeo<C>;
     constexpr int SEGF = C * kE, KS = SEGF + 4, NCOPY = SG::SK * SEGF / 4;
     static_assert(NCOPY % SG::NT == 0, "whole copies per thread");
 #pragma unroll
     for (int q = 0; q < NCOPY / SG::NT; ++q) {
         const int f = 4 * (threadIdx.x + q * SG::NT), k = f / SEGF;
-        cp_async16(dst + k * KS + (f - k * SEGF), src + f);
+        cp_async16(dst + k * KS + (f - k * SEGF), src + f, pol);
     }
 }
 
@@ -290,7 +294,7 @@ __device__ __forceinline__ CtaTiles cta_tiles(const SymScan& a) {
 // aggregate; both restart at each base range's last tile and are written out at
 // its first.
 template <int C, int AHEAD>
-__global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
+__global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
     k_sym_agg(SymScan a, const float* __restrict__ v, RangeState st, float* __restrict__ vs) {
     using SG = SymGeo<C>;
     using G = typename SG::G;
@@ -304,6 +308,9 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
     const int lane = threadIdx.x & 31, cs = lane / SK, k = lane % SK;
     const int c = (threadIdx.x >> 5) * CW + cs, ch0 = grp * C;
     auto tile_of = [&](int i) { return w.te - 1 - i; };
+    // anchors, permutation and the sorted copy stream through once; the gathered
+    // rows keep normal priority (the other row of a 128-byte line may follow soon)
+    const uint64_t pol_f = l2_evict_first(), pol_n = l2_evict_normal();
     // anchor of the last row of base range J
     auto range_end = [&](int64_t J) { return __ldg(a.s + min(a.n, (J + 1) * a.tpr * (int64_t)R) - 1); };
     // fp64 decays of the tile folds, negative for a tie (decay 1, no break): [0] right
@@ -314,16 +321,24 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
         ed[0] = (sb[4 + R] > sb[4]) ? exp((double)sb[4] - (double)sb[4 + R]) : -1.0;
         ed[1] = (ue > sb[4 + R - 1]) ? exp((double)sb[4 + R - 1] - (double)ue) : -1.0;
     };
+    // cp.async groups, in commit order: anchors+permutation of tiles 0 .. MA-1
+    // (waited for at once), rows of tiles 0 .. AHEAD-1, then per iteration j the
+    // anchors+permutation of tile j+MA and the rows of tile j+AHEAD.  At the top
+    // of iteration i at most WAIT groups may stay pending: the rows of tile i have
+    // at least AHEAD-1 groups after them and the permutation of tile i+AHEAD
+    // (read when its rows are staged) has three.
+    constexpr int MA = SM::MA, WAIT = (AHEAD - 1 < 3) ? AHEAD - 1 : 3;
+    static_assert(AHEAD >= 1, "at least one tile of prefetch");
 #pragma unroll
-    for (int q = 0; q <= AHEAD; ++q) {
-        if (q < nt) stage_meta<G>(a.s, a.perm, a.n, tile_lo(tile_of(q), R), sm.s[q % MS], sm.p[q % MS]);
+    for (int q = 0; q < MA; ++q) {
+        if (q < nt) stage_meta<G>(a.s, a.perm, a.n, tile_lo(tile_of(q), R), sm.s[q % MS], sm.p[q % MS], pol_f);
         cp_async_commit();
     }
     cp_async_wait_all();
     __syncthreads();
 #pragma unroll
     for (int q = 0; q < AHEAD; ++q) {
-        if (q < nt) stage_rows<G>(v, a.B, ch0, a.n, tile_lo(tile_of(q), R), sm.p[q % MS], sm.v[0][q % VS]);
+        if (q < nt) stage_rows<G>(v, a.B, ch0, a.n, tile_lo(tile_of(q), R), sm.p[q % MS], sm.v[0][q % VS], pol_n);
         cp_async_commit();
     }
     seg_tables<SK, SG::NT>(sm.s[0], sm.tab[0]);
@@ -332,15 +347,15 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
     for (int i = 0; i < nt; ++i) {
         const int64_t t = tile_of(i);
         const int64_t J = t / a.tpr;
-        cp_async_wait<AHEAD - 1>();  // this tile's rows and the next tiles' anchors are in
+        cp_async_wait<WAIT>();  // this tile's rows and the anchors of the tiles ahead are in
         __syncthreads();
-        if (i + AHEAD + 1 < nt)
-            stage_meta<G>(a.s, a.perm, a.n, tile_lo(tile_of(i + AHEAD + 1), R), sm.s[(i + AHEAD + 1) % MS],
-                          sm.p[(i + AHEAD + 1) % MS]);
+        if (i + MA < nt)
+            stage_meta<G>(a.s, a.perm, a.n, tile_lo(tile_of(i + MA), R), sm.s[(i + MA) % MS], sm.p[(i + MA) % MS],
+                          pol_f);
         cp_async_commit();
         if (i + AHEAD < nt)
             stage_rows<G>(v, a.B, ch0, a.n, tile_lo(tile_of(i + AHEAD), R), sm.p[(i + AHEAD) % MS],
-                          sm.v[0][(i + AHEAD) % VS]);
+                          sm.v[0][(i + AHEAD) % VS], pol_n);
         cp_async_commit();
         if (i + 1 < nt) {
             seg_tables<SK, SG::NT>(sm.s[(i + 1) % MS], sm.tab[(i + 1) & 1]);
@@ -356,7 +371,8 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
         {  // this lane's E values of the sorted copy
             float4* dst = reinterpret_cast<float4*>(sorted_tile(vs, grp, a.T, t, R, C) + (k * C + c) * E);
 #pragma unroll
-            for (int q = 0; q < E / 4; ++q) dst[q] = make_float4(xv[4 * q], xv[4 * q + 1], xv[4 * q + 2], xv[4 * q + 3]);
+            for (int q = 0; q < E / 4; ++q)
+                st_hint(dst + q, make_float4(xv[4 * q], xv[4 * q + 1], xv[4 * q + 2], xv[4 * q + 3]), pol_f);
         }
         LP sr[1] = {{0.f, 0.f}}, sl[1] = {{0.f, 0.f}};
 #pragma unroll
@@ -538,14 +554,22 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         ed[0] = (sb[4 + R - 1] > sb[3]) ? exp((double)sb[3] - (double)sb[4 + R - 1]) : -1.0;
         ed[1] = (-sb[4 + R] > ur) ? exp((double)ur + (double)sb[4 + R]) : -1.0;
     };
+    // everything but the scattered 4-byte ga rows streams through L2 once
+    const uint64_t pol_f = l2_evict_first();
+    // cp.async groups per iteration j: anchors+permutation+carries of tile j+AHEAD+1,
+    // then the sorted tiles of tile j+AHEAD; waiting until AHEAD-1 groups remain
+    // leaves the current tile's data and the next tile's anchors complete when
+    // AHEAD <= 2
+    static_assert(AHEAD >= 1 && AHEAD <= 2, "prefetch distance of the sweeps");
     auto stage_vecs = [&](int64_t tt, int slot) {
 #pragma unroll
-        for (int w = 0; w < NV; ++w) stage_sorted<C>(sorted_tile(w == 0 ? xs : gs, grp, a.T, tt, R, C), sm.v[w][slot]);
+        for (int w = 0; w < NV; ++w)
+            stage_sorted<C>(sorted_tile(w == 0 ? xs : gs, grp, a.T, tt, R, C), sm.v[w][slot], pol_f);
     };
 #pragma unroll
     for (int q = 0; q <= AHEAD; ++q) {
         if (q < nt) {
-            stage_meta<G>(a.s, a.perm, a.n, tile_lo(cw.tb + q, R), sm.s[q % MS], sm.p[q % MS]);
+            stage_meta<G>(a.s, a.perm, a.n, tile_lo(cw.tb + q, R), sm.s[q % MS], sm.p[q % MS], pol_f);
             stage_carries<C, NV>(a, sx, sg, grp, cw.tb + q, sm.rs[q % MS], sm.rin[q % MS]);
         }
         cp_async_commit();
@@ -574,7 +598,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         __syncthreads();
         if (i + AHEAD + 1 < nt) {
             stage_meta<G>(a.s, a.perm, a.n, tile_lo(t + AHEAD + 1, R), sm.s[(i + AHEAD + 1) % MS],
-                          sm.p[(i + AHEAD + 1) % MS]);
+                          sm.p[(i + AHEAD + 1) % MS], pol_f);
             stage_carries<C, NV>(a, sx, sg, grp, t + AHEAD + 1, sm.rs[(i + AHEAD + 1) % MS],
                                  sm.rin[(i + AHEAD + 1) % MS]);
         }
@@ -690,14 +714,14 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 inR[w] = seg_in(hr_tile, cR[w], k + 1 < SK, exR, evr);
             }
             // pass 2: gx to the output rows, ga to the per-warp sums
-            float gxp[E], gap[E];
+            float gap[E];
             LP ax = inR[0], ag = inR[NV - 1];
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
                 const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e + 1];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
-                gxp[e] = ag.P - ge;
+                ob[e * C] = ag.P - ge;               // gx, right part
                 gap[e] = fmaf(ge, ax.L, xe * ag.L);  // strict right sums
             }
             ax = inL[0];
@@ -707,7 +731,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e];
                 ax = lp_step_d(ax, dv, 0.f, xe);
                 ag = lp_step_d(ag, dv, 0.f, ge);
-                ob[e * C] = gxp[e] + ag.P;                    // gx
+                ob[e * C] += ag.P;                            // gx
                 gap[e] = gap[e] - fmaf(ge, ax.L, xe * ag.L);  // this channel's share of ga
             }
             // sum over the warp's channels, then one padded row per warp in shared memory
@@ -720,7 +744,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         __syncthreads();
         // coalesced stores of whole rows through the permutation
         const uint32_t* pb = sm.p[i % MS];
-        if (out != nullptr) store_rows<G>(out, a.B, ch0, a.n, lo, pb, sm.o);
+        if (out != nullptr) store_rows<G>(out, a.B, ch0, a.n, lo, pb, sm.o, pol_f);
         if (NV == 2 && ga != nullptr) {
             for (int r = threadIdx.x; r < R; r += NT) {
                 if (lo + r >= a.n) continue;
