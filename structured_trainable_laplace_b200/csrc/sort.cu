@@ -140,16 +140,22 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
             val[i] = 0u;
         }
     }
-    // stable rank inside the warp, items in (i, lane) order = index order
+    // stable rank inside the warp, items in (i, lane) order = index order.  The
+    // masks of lanes holding the same digit do not depend on the running counts,
+    // so all are formed first (independent match operations); only the count
+    // updates form a chain.  rank[] holds the mask until the rank replaces it.
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
-        const int64_t idx = wbase + i * 32 + lane;
-        const bool valid = idx < n;
-        const uint32_t vm = __ballot_sync(0xffffffffu, valid);
-        uint32_t peers = 0, d = 0, before = 0;
+        const bool valid = wbase + i * 32 + lane < n;
+        const uint32_t d = (key[i] >> shift) & 0xffu;
+        rank[i] = __match_any_sync(0xffffffffu, valid ? d : 0x100u);  // rows past n group apart
+    }
+#pragma unroll
+    for (int i = 0; i < kItems; ++i) {
+        const bool valid = wbase + i * 32 + lane < n;
+        const uint32_t d = (key[i] >> shift) & 0xffu, peers = rank[i];
+        uint32_t before = 0;
         if (valid) {
-            d = (key[i] >> shift) & 0xffu;
-            peers = __match_any_sync(vm, d);
             before = s_whist[w][d];
             rank[i] = before + __popc(peers & lanemask_lt());
         }

@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         ed[1] = (-sb[4 + R] > ur) ? exp((double)ur + (double)sb[4 + R]) : -1.0;
     };
     // everything but the scattered 4-byte ga rows streams through L2 once
-    const uint64_t pol_f = l2_evict_first();
+    const uint64_t pol_f = l2_evict_first(), pol_l = l2_evict_last();
     // cp.async groups per iteration j: anchors+permutation+carries of tile j+AHEAD+1,
     // then the sorted tiles of tile j+AHEAD; waiting until AHEAD-1 groups remain
     // leaves the current tile's data and the next tile's anchors complete when
@@ -755,7 +755,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 if (ga_atomic)
                     atomicAdd(ga + row, acc);
                 else
-                    ga[row] = acc;
+                    st_hint(ga + row, acc, pol_l);  // kept in L2 until its lines are complete
             }
         }
     }
