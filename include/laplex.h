@@ -126,6 +126,28 @@ laplex_status laplex_apply_sym(const float* a_sorted, const uint32_t* perm, int6
                                float* y, void* saved, void* ws, size_t ws_bytes, int32_t* d_status,
                                laplex_stream_t stream);
 
+/* laplex_apply_sym without a workspace.  This entry point has no counterpart in
+ * the paper: it is an interface convenience for callers that cannot hand the
+ * library scratch memory -- code that owns no device allocator (a plain C host
+ * program that only holds device pointers to its inputs and outputs), or a loop
+ * that must not allocate or grow buffers between its calls.  Its scratch is a
+ * static device array inside the library (LAPLEX_NOALLOC_SCRATCH_BYTES, one copy
+ * per device), so the call allocates and frees nothing.  Contract:
+ *   - the same arguments and result as laplex_apply_sym with saved = NULL;
+ *   - size limit: n * Bp <= LAPLEX_NOALLOC_MAX_ELEMS, where Bp is B rounded up to
+ *     the next of 1, 2, 4, 8, 16, 32, or to a multiple of 32 above 32 (B = 16
+ *     allows n up to 65536); larger problems return LAPLEX_ERR_WORKSPACE before
+ *     anything is launched -- use laplex_apply_sym for them;
+ *   - the first call on each device performs a one-time setup (it looks up the
+ *     device address of the static array), so make it before any stream capture;
+ *   - calls must not overlap on one device: two calls in flight at once (on two
+ *     streams, or from two host threads) share the scratch and race;
+ *   - nothing has to be zeroed beforehand. */
+#define LAPLEX_NOALLOC_MAX_ELEMS (1LL << 20)
+#define LAPLEX_NOALLOC_SCRATCH_BYTES (8LL << 20)
+laplex_status laplex_apply_sym_noalloc(const float* a_sorted, const uint32_t* perm, int64_t n, const float* x,
+                                       int64_t B, float* y, int32_t* d_status, laplex_stream_t stream);
+
 /* General rectangular operator (section 2.2, "general case a != b"): y = E x,
  * E_ij = exp(-|a_i - b_j|), x [k][B] at the b anchors, y [n][B] at the a anchors.
  * The inputs are scanned over sorted b and every a reads the state of its

@@ -157,6 +157,16 @@ laplex_status laplex_apply_sym(const float* a_sorted, const uint32_t* perm, int6
     return cuda_status(launch_sym_forward(a_sorted, perm, n, x, B, y, saved, ws, d_status, (cudaStream_t)stream));
 }
 
+laplex_status laplex_apply_sym_noalloc(const float* a_sorted, const uint32_t* perm, int64_t n, const float* x,
+                                       int64_t B, float* y, int32_t* d_status, laplex_stream_t stream) {
+    if (!size_ok(n) || !batch_ok(B) || !a_sorted || !perm || !x || !y) return LAPLEX_ERR_ARG;
+    if (n > LAPLEX_NOALLOC_MAX_ELEMS / sym_padded_batch(B)) return LAPLEX_ERR_WORKSPACE;
+    laplex_status s = check_ranges({{a_sorted, fbytes(n)}, {perm, fbytes(n)}, {x, fbytes(n * B)}},
+                                   {{y, fbytes(n * B)}, {d_status, 4}});
+    if (s != LAPLEX_OK) return s;
+    return cuda_status(launch_sym_forward_noalloc(a_sorted, perm, n, x, B, y, d_status, (cudaStream_t)stream));
+}
+
 laplex_status laplex_apply_general(const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* b_sorted,
                                    const uint32_t* perm_b, int64_t k, const float* x, int64_t B, float* y,
                                    void* saved, void* ws, size_t ws_bytes, int32_t* d_status,

@@ -42,6 +42,12 @@ cudaError_t launch_sym_forward(const float* s, const uint32_t* perm, int64_t n, 
 cudaError_t launch_sym_backward(const float* s, const uint32_t* perm, int64_t n, const float* x, const float* g,
                                 int64_t B, const void* saved, float* gx, float* ga, void* ws, int32_t* status,
                                 cudaStream_t stream);
+// The symmetric forward on the library's static scratch (laplex_apply_sym_noalloc):
+// B rounded up to whole channel groups, and the launcher.  The launcher returns
+// cudaErrorInvalidValue if the problem does not fit the scratch.
+int64_t sym_padded_batch(int64_t B);
+cudaError_t launch_sym_forward_noalloc(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B,
+                                       float* y, int32_t* status, cudaStream_t stream);
 
 // rect.cu: rectangular operators in canonical form.  The "output side" O and the
 // "input side" I are each a sorted anchor set with its permutation and optional

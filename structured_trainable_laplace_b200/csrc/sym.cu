@@ -32,6 +32,9 @@
 // cp.async: the gathered rows AHEAD tiles ahead, anchors, permutation and
 // carries one tile further; per-row decays and the fp64 decays of the tile folds
 // are computed one tile ahead.  No kernel waits on another CTA.
+#include <mutex>
+
+#include "laplex.h"
 #include "laplex_internal.h"
 #include "pipeline.cuh"
 
@@ -950,6 +953,84 @@ cudaError_t launch_sym_backward(const float* s, const uint32_t* perm, int64_t n,
                                 cudaStream_t st) {
     (void)status;
 #define CALL(C) sym_backward_t<C>(s, perm, n, x, g, B, saved, gx, ga, ws, st)
+    LAPLEX_SYM_DISPATCH(choose_channels(B), CALL)
+#undef CALL
+}
+
+// ------------------------------------------------------- static-scratch forward
+
+// Scratch of laplex_apply_sym_noalloc: part of the library's static device
+// memory (one copy per device, created with the module), so that entry point
+// takes no workspace and allocates nothing.  LAPLEX_NOALLOC_SCRATCH_BYTES covers
+// every problem with n * sym_padded_batch(B) <= LAPLEX_NOALLOC_MAX_ELEMS.
+// Nothing in it has to start at zero: every word the kernels read is written
+// earlier in the same call.  Calls whose work overlaps on one device (two
+// streams, or two host threads) share the array and corrupt each other.
+static __device__ __align__(256) unsigned char g_sym_scratch[LAPLEX_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_sym_scratch on the current device, looked up the first
+// time a device is used (the only setup step; later calls reuse it).
+cudaError_t sym_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_sym_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+// The forward of sym_forward_t with its scratch carved from g_sym_scratch: range
+// arrays sized for this device's ranges only, no saved state.
+template <int C>
+cudaError_t sym_forward_static_t(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B, float* y,
+                                 cudaStream_t st) {
+    void* scratch = nullptr;
+    cudaError_t e = sym_scratch(&scratch);
+    if (e != cudaSuccess) return e;
+    const int sms = device_sms();
+    SymPlan p = plan_sym(n, B, sms);
+    p.rng_elems = (size_t)p.G * p.P * p.C;
+    const size_t state = align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
+    if (state + p.sorted_bytes > (size_t)LAPLEX_NOALLOC_SCRATCH_BYTES) return cudaErrorInvalidValue;
+    const RangeState sx = carve(p, (double2*)scratch, true);
+    float* xs = (float*)((char*)scratch + state);
+    e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
+    if (e != cudaSuccess) return e;
+    using SM = SweepSmem<C, 1, kAheadFwd>;
+    static int occ_cache = 0;
+    const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
+    LAPLEX_TIMED("sym_fwd", st,
+                 k_sym_sweep<C, 1, kAheadFwd>
+                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, nullptr, sx, sx, y, nullptr, 0));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int64_t sym_padded_batch(int64_t B) {
+    const int64_t C = choose_channels(B);
+    return (B + C - 1) / C * C;
+}
+
+cudaError_t launch_sym_forward_noalloc(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B,
+                                       float* y, int32_t* status, cudaStream_t st) {
+    (void)status;
+#define CALL(C) sym_forward_static_t<C>(s, perm, n, x, B, y, st)
     LAPLEX_SYM_DISPATCH(choose_channels(B), CALL)
 #undef CALL
 }

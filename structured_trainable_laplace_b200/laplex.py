@@ -53,6 +53,7 @@ def lib():
             "laplex_workspace_size": ([I, I64, I64, I64], SZ),
             "laplex_saved_size": ([I, I64, I64, I64], SZ),
             "laplex_apply_sym": ([P, P, I64, P, I64, P, P, P, SZ, P, P], I),
+            "laplex_apply_sym_noalloc": ([P, P, I64, P, I64, P, P, P], I),
             "laplex_apply_general": ([P, P, I64, P, P, I64, P, I64, P, P, P, SZ, P, P], I),
             "laplex_apply_transpose": ([P, P, I64, P, P, I64, P, I64, P, P, P, SZ, P, P], I),
             "laplex_apply_phased": ([P, P, I64, P, P, P, I64, P, I, P, I64, P, P, P, SZ, P, P], I),
@@ -72,7 +73,8 @@ def lib():
 def exported_symbols() -> list:
     """Names of the C entry points this binding calls."""
     return ["laplex_status_string", "laplex_read_status", "laplex_sort_workspace_size", "laplex_sort_anchors",
-            "laplex_workspace_size", "laplex_saved_size", "laplex_apply_sym", "laplex_apply_general",
+            "laplex_workspace_size", "laplex_saved_size", "laplex_apply_sym", "laplex_apply_sym_noalloc",
+            "laplex_apply_general",
             "laplex_apply_transpose", "laplex_apply_phased", "laplex_backward", "laplex_gram_apply",
             "laplex_profile_enable", "laplex_profile_report"]
 
@@ -186,6 +188,17 @@ def apply_sym(a_sorted, perm, x, saved=None):
     ws = workspace(workspace_size(OP_SYM, n, 1, B), d)
     _ok(lib().laplex_apply_sym(_p(a_sorted), _p(perm), n, _p(xr), B, _p(y), _p(saved), _p(ws), ws.numel(),
                                _p(status_word(d)), _stream(d)), "apply_sym")
+    return back(y)
+
+
+def apply_sym_noalloc(a_sorted, perm, x):
+    """y = K x on the library's static scratch: no workspace (n * padded B <= 2^20)."""
+    xr, sq = _rows(x)
+    n, B = xr.shape
+    d = _dev(x)
+    y, back = _out_like_rows(n, B, sq, x.device)
+    _ok(lib().laplex_apply_sym_noalloc(_p(a_sorted), _p(perm), n, _p(xr), B, _p(y), _p(status_word(d)), _stream(d)),
+        "apply_sym_noalloc")
     return back(y)
 
 

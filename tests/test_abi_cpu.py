@@ -85,5 +85,8 @@ def test_bad_arguments_are_rejected_before_launch(L):
     # backward of an unknown op
     assert L.laplex_backward(42, fake, fake, 8, None, fake, fake, 4, None, fake, fake, 1, None, ws, None, None,
                              None, None, ws, 1 << 30, None, None) == 1
+    # static-scratch product: beyond its size limit (n * padded B > 2^20)
+    assert L.laplex_apply_sym_noalloc(fake, fake, 65537, fake, 16, P(1 << 24), None, None) == 3
+    assert L.laplex_apply_sym_noalloc(fake, fake, 4097, fake, 257, P(1 << 24), None, None) == 3
     # sort: n too large
     assert L.laplex_sort_anchors(fake, 1 << 33, fake, fake, ws, 1 << 30, None, None) == 1
