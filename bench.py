@@ -99,9 +99,9 @@ def kernel_bytes_per_launch(kernel: str, w) -> float | None:
     n, B, k = w.n, w.B, w.k
     if w.op == "sym":
         table = {
-            "sym_bwd": (8 + 4 * B + 4 * B + 4 * B + 4) * n,   # s, perm, x, g -> gx, ga
-            "sym_left": (8 + 4 * B + 4 * B) * n,             # s, perm, x -> y
-            "sym_right": (8 + 4 * B) * n,                    # s, perm, x (carries only)
+            "sym_agg": (8 + 4 * B + 4 * B) * n,              # s, perm, x rows gathered -> sorted copy of x
+            "sym_fwd": (8 + 4 * B + 4 * B) * n,              # s, perm, sorted copy of x -> y rows scattered
+            "sym_bwd": (8 + 4 * B + 4 * B + 4 * B + 4) * n,  # s, perm, sorted x, sorted g -> gx rows, ga
             "radix_pass": (12 * n + 3 * 16 * n) / 4.0,       # pass 0 reads a; passes 1-3 read+write key,value
             "radix_hist": 4 * n,
         }
@@ -275,7 +275,7 @@ def cpu_model() -> str:
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="sym2p24",
@@ -378,7 +378,7 @@ def main():
 
     for _ in range(2):
         e2e_step()
-    ms_e2e = timed(e2e_step, max(2, args.steps // 2))
+    ms_e2e = timed(e2e_step, max(2, min(10, args.steps // 2)))
     peak_mem = torch.cuda.max_memory_allocated(device) / 1e9
 
     units = elements(w) * world
