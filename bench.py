@@ -46,14 +46,15 @@ FALLBACK_HBM_GBS = 6650.0
 
 def make_workload(name: str, rank: int, n: int | None = None):
     """Inputs of the named workload; anchors (parameters) identical on every rank,
-    vectors drawn per rank.  n overrides the symmetric workload's size (same recipe:
-    a ~ U[0, 0.05 n], B = 16), for profiling captures of a smaller case."""
+    vectors drawn per rank.  n overrides the large-side size of the symmetric,
+    phased-head and Gram workloads (same recipe otherwise), for profiling captures
+    of a smaller case."""
     gen = {
         "sym2p24": lambda s: inputs.sym_2p24_b16(s, n=n or (1 << 24)),
         "small": lambda s: inputs.sym_small_ties(s),
         "sym1e9": lambda s: inputs.sym_extreme(s),
-        "phased_head": lambda s: inputs.phased_head_2p22(s),
-        "gram_image": lambda s: inputs.gram_image(s),
+        "phased_head": lambda s: inputs.phased_head_2p22(s, n=n or (1 << 22)),
+        "gram_image": lambda s: inputs.gram_image(s, n=n or 3 * 1024 * 1024),
     }[name]
     w = gen(rank)
     if rank != 0:
@@ -281,7 +282,7 @@ def main():
     ap.add_argument("--workload", default="sym2p24",
                     choices=["sym2p24", "small", "phased_head", "gram_image", "sym1e9"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
-    ap.add_argument("--n", type=int, default=None, help="anchors of the symmetric workload (profiling captures)")
+    ap.add_argument("--n", type=int, default=None, help="large-side anchors (profiling captures of a smaller case)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 

@@ -316,6 +316,11 @@ __device__ __forceinline__ void store_vec(float* p, const float (&v)[VEC]) {
     }
 }
 
+// Rows per prefetch batch of k_large: as many as the registers allow next to the
+// accumulators (the phased, 4-channel variants carry twice the state).
+template <int VEC, bool PHASED, int MODE>
+constexpr int kLargeBatch = (VEC == 4 && PHASED) ? 4 : 8;
+
 // Each group of `lpr` lanes walks a contiguous range of sorted large-side rows;
 // lane gl of the group owns channels c0 .. c0+VEC-1 of every row.
 template <int VEC, bool PHASED, int MODE>
@@ -396,102 +401,229 @@ __global__ void __launch_bounds__(256) k_large(LargePass A) {
     int64_t st_m = -1, st_mp = -1;
     float Pm1[NP][VEC], Pmp[NP][VEC], Smp[NP][VEC];
 
-    for (int64_t r = r0; r < r1; ++r) {
-        const float q = __ldg(A.s + r);
-        const uint32_t pr = min(__ldg(A.perm + r), (uint32_t)(A.m - 1));
-        float w[NP], wd[NP];
-        if (PHASED) {
-            float sn, cs;
-            sincosf(__ldg(A.theta + pr), &sn, &cs);
-            w[0] = cs;
-            w[NP - 1] = sn;
-            wd[0] = -sn;
-            wd[NP - 1] = cs;
-        } else {
-            w[0] = 1.f;
-            wd[0] = 0.f;
-        }
-        while (m < ms && __ldg(A.sp + m) < q) ++m;
-        if (mp < m) mp = m;
-        while (mp < ms && __ldg(A.sp + mp) <= q) ++mp;
-        const bool tie = mp > m;
-        const float eL = (m > 0) ? expf(__ldg(A.sp + m - 1) - q) : 0.f;
-        const float eR = (mp < ms) ? expf(q - __ldg(A.sp + mp)) : 0.f;
+    // One row: q's bins m (small-side anchors < q) and mp (<= q), the decays eL / eR
+    // to the neighbouring small-side anchors, phase weights (w0, w1) = (cos, sin),
+    // the gathered row h.  Returns the row's anchor / phase gradient shares of this
+    // lane's channels in ga / gp.
+    auto row = [&](uint32_t pr, float w0, float w1, float eL, float eR, int64_t mr, int64_t mpr, const float* h,
+                   float& ga, float& gp) {
+        const float w[2] = {w0, w1};
+        const bool tie = mpr > mr;
         const float eLf = tie ? 1.f : eL;
-        float h[VEC];
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) h[v] = 0.f;
-        if (ROWS && cval) load_vec<VEC>(A.rows + (int64_t)pr * B + c0, h);
         if (ACCUM) {
-            if (m != cur) {
+            if (mr != cur) {
                 flush(cur);
-                cur = m;
+                cur = mr;
             }
+            if (!tie) {
+                // untied rows feed the interval sums u (weighted to the right
+                // neighbour) and v (to the left one)
 #pragma unroll
-            for (int p = 0; p < NP; ++p)
+                for (int p = 0; p < NP; ++p) {
+                    const float wr = eR * w[p], wl = eL * w[p];
 #pragma unroll
-                for (int v = 0; v < VEC; ++v) {
-                    const float val = w[p] * h[v];
-                    // A row tied with a run of small-side anchors enters that run only
-                    // (TL, TR); the neighbours beyond it receive it through the scan.
-                    if (!tie) {
-                        fu[p][v] = fmaf(eR, val, fu[p][v]);
-                        fv[p][v] = fmaf(eL, val, fv[p][v]);
-                    } else if (cval) {
-                        atomicAdd(A.TL + m * Cb + p * B + c0 + v, (double)val);
-                        atomicAdd(A.TR + (mp - 1) * Cb + p * B + c0 + v, (double)val);
+                    for (int v = 0; v < VEC; ++v) {
+                        fu[p][v] = fmaf(wr, h[v], fu[p][v]);
+                        fv[p][v] = fmaf(wl, h[v], fv[p][v]);
                     }
                 }
+            } else if (cval) {
+                // a row tied with a run of small-side anchors enters that run only
+                // (TL, TR); the neighbours beyond it receive it through the scan
+#pragma unroll
+                for (int p = 0; p < NP; ++p)
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) {
+                        const double val = (double)(w[p] * h[v]);
+                        atomicAdd(A.TL + mr * Cb + p * B + c0 + v, val);
+                        atomicAdd(A.TR + (mpr - 1) * Cb + p * B + c0 + v, val);
+                    }
+            }
             if (++cnt == 16) fold();
         }
         if (STATES) {
-            if (m != st_m || mp != st_mp) {
+            if (mr != st_m || mpr != st_mp) {
 #pragma unroll
                 for (int p = 0; p < NP; ++p)
 #pragma unroll
                     for (int v = 0; v < VEC; ++v) {
                         const int ch = p * B + c0 + v;
-                        Pm1[p][v] = (GRAD && cval && m > 0) ? __ldg(A.Pst + (m - 1) * Cb + ch) : 0.f;
-                        Pmp[p][v] = (cval && mp > 0) ? __ldg(A.Pst + (mp - 1) * Cb + ch) : 0.f;
-                        Smp[p][v] = (cval && mp < ms) ? __ldg(A.Sst + mp * Cb + ch) : 0.f;
+                        Pm1[p][v] = (GRAD && cval && mr > 0) ? __ldg(A.Pst + (mr - 1) * Cb + ch) : 0.f;
+                        Pmp[p][v] = (cval && mpr > 0) ? __ldg(A.Pst + (mpr - 1) * Cb + ch) : 0.f;
+                        Smp[p][v] = (cval && mpr < ms) ? __ldg(A.Sst + mpr * Cb + ch) : 0.f;
                     }
-                st_m = m;
-                st_mp = mp;
+                st_m = mr;
+                st_mp = mpr;
+            }
+            // out = sum_p w_p (eLf P_(mp-1) + eR S_mp); the strict left part of the
+            // prefix is eL P_(m-1) (ties excluded)
+            float fl[NP], fr[NP], dl[NP];
+#pragma unroll
+            for (int p = 0; p < NP; ++p) {
+                fl[p] = eLf * w[p];
+                fr[p] = eR * w[p];
+                dl[p] = eL * w[p];
             }
             float o[VEC];
-            float ga = 0.f, gp = 0.f;
 #pragma unroll
             for (int v = 0; v < VEC; ++v) {
                 o[v] = 0.f;
+                float t = 0.f;
 #pragma unroll
                 for (int p = 0; p < NP; ++p) {
-                    const float full = fmaf(eLf, Pmp[p][v], eR * Smp[p][v]);
-                    o[v] = fmaf(w[p], full, o[v]);
-                    if (GRAD) {
-                        const float diff = fmaf(eR, Smp[p][v], -eL * Pm1[p][v]);  // strict right - strict left
-                        ga = fmaf(h[v] * w[p], diff, ga);
-                        if (PHASED) gp = fmaf(h[v] * wd[p], full, gp);
+                    o[v] = fmaf(fl[p], Pmp[p][v], fmaf(fr[p], Smp[p][v], o[v]));
+                    if (GRAD) t = fmaf(fr[p], Smp[p][v], fmaf(-dl[p], Pm1[p][v], t));
+                }
+                if (GRAD) {
+                    ga = fmaf(h[v], t, ga);  // strict right - strict left
+                    if (PHASED) {
+                        // d/dtheta of (cos, sin) is (-sin, cos)
+                        const float f0 = fmaf(eLf, Pmp[0][v], eR * Smp[0][v]);
+                        const float f1 = fmaf(eLf, Pmp[NP - 1][v], eR * Smp[NP - 1][v]);
+                        gp = fmaf(h[v], fmaf(w0, f1, -w1 * f0), gp);
                     }
                 }
             }
             if (EXPAND && A.out != nullptr && cval) store_vec<VEC>(A.out + (int64_t)pr * B + c0, o);
-            if (GRAD) {
-                for (int off = lpr >> 1; off >= 1; off >>= 1) {
-                    ga += __shfl_xor_sync(gmask, ga, off);
-                    if (PHASED) gp += __shfl_xor_sync(gmask, gp, off);
+        }
+    };
+    auto put_grad = [&](float* dst, uint32_t pr, float v) {
+        if (dst == nullptr) return;
+        if (A.chunk_atomic)
+            atomicAdd(dst + pr, v);
+        else
+            dst[pr] = v;
+    };
+
+    constexpr int U = kLargeBatch<VEC, PHASED, MODE>;
+    if (lpr >= U) {
+        // Wide groups.  Rows are taken in batches of lpr: lane gl computes the
+        // scalars of row rb + gl (permutation entry, phase weights, bins, decays),
+        // so every row's scalar work is done once; the group then walks the batch in
+        // sub-batches of U rows whose gathered rows are loaded together, taking each
+        // row's scalars from the lane that computed them.  Bins are below 2^32.
+        for (int64_t rb = r0; rb < r1; rb += lpr) {
+            const int nb = (int)min((int64_t)lpr, r1 - rb);
+            const int64_t rme = rb + min(gl, nb - 1);
+            const float q_me = __ldg(A.s + rme);
+            const uint32_t pr_me = min(__ldg(A.perm + rme), (uint32_t)(A.m - 1));
+            float cs_me = 1.f, sn_me = 0.f;
+            if (PHASED) sincosf(__ldg(A.theta + pr_me), &sn_me, &cs_me);
+            int64_t mm = m;
+            while (mm < ms && __ldg(A.sp + mm) < q_me) ++mm;
+            int64_t mmp = max(mp, mm);
+            while (mmp < ms && __ldg(A.sp + mmp) <= q_me) ++mmp;
+            const float eL_me = (mm > 0) ? expf(__ldg(A.sp + mm - 1) - q_me) : 0.f;
+            const float eR_me = (mmp < ms) ? expf(q_me - __ldg(A.sp + mmp)) : 0.f;
+            const uint32_t mm32 = (uint32_t)mm, mmp32 = (uint32_t)mmp;
+            for (int j = 0; j < nb; j += U) {
+                uint32_t prv[U];
+                float hv[U][VEC];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    prv[u] = __shfl_sync(gmask, pr_me, min(j + u, nb - 1), lpr);
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) hv[u][v] = 0.f;
+                    if (ROWS && cval) load_vec<VEC>(A.rows + (int64_t)prv[u] * B + c0, hv[u]);
                 }
-                if (gl == 0) {
-                    if (A.g_anchor != nullptr) {
-                        if (A.chunk_atomic)
-                            atomicAdd(A.g_anchor + pr, ga);
-                        else
-                            A.g_anchor[pr] = ga;
+                float gpart[GRAD ? 2 * U : 1];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int src = min(j + u, nb - 1);
+                    const float w0 = __shfl_sync(gmask, cs_me, src, lpr);
+                    const float w1 = PHASED ? __shfl_sync(gmask, sn_me, src, lpr) : 0.f;
+                    const float eL = __shfl_sync(gmask, eL_me, src, lpr);
+                    const float eR = __shfl_sync(gmask, eR_me, src, lpr);
+                    m = __shfl_sync(gmask, mm32, src, lpr);
+                    mp = __shfl_sync(gmask, mmp32, src, lpr);
+                    float ga = 0.f, gp = 0.f;
+                    if (j + u < nb) row(prv[u], w0, w1, eL, eR, m, mp, hv[u], ga, gp);  // group-uniform
+                    if (GRAD) {
+                        gpart[u] = ga;
+                        gpart[U + u] = gp;
                     }
-                    if (PHASED && A.g_phase != nullptr) {
-                        if (A.chunk_atomic)
-                            atomicAdd(A.g_phase + pr, gp);
-                        else
-                            A.g_phase[pr] = gp;
+                }
+                if (GRAD) {
+                    // sum the 2U partials over the group's lanes by recursive halving
+                    // (halves fixed at compile time, the group width at run time);
+                    // lane gl ends with the totals of value indices base .. base + vc - 1
+                    constexpr int NV = 2 * U;
+                    int vc = NV, base = 0, hl = 0;
+#pragma unroll
+                    for (int L = 0; (NV >> L) > 1; ++L) {
+                        const int o = lpr >> (L + 1);
+                        if (o >= 1) {
+                            const bool upper = (gl & o) != 0;
+#pragma unroll
+                            for (int i = 0; i < (NV >> (L + 1)); ++i) {
+                                const float keep = upper ? gpart[i + (NV >> (L + 1))] : gpart[i];
+                                const float send = upper ? gpart[i] : gpart[i + (NV >> (L + 1))];
+                                gpart[i] = keep + __shfl_xor_sync(gmask, send, o, lpr);
+                            }
+                            if (upper) base += NV >> (L + 1);
+                            vc = NV >> (L + 1);
+                            hl = L + 1;
+                        }
+                    }
+                    // the remaining levels add whole totals: lanes that differ only in
+                    // those bits hold the same totals, and the lowest of them writes
+                    const int dup = lpr >> hl;
+                    for (int o = dup >> 1; o >= 1; o >>= 1) gpart[0] += __shfl_xor_sync(gmask, gpart[0], o, lpr);
+                    const bool writer = (gl & (dup - 1)) == 0;
+#pragma unroll
+                    for (int i = 0; i < NV; ++i) {
+                        if (i >= vc) break;
+                        const int idx = base + i, u = idx % U;
+                        const uint32_t pr = __shfl_sync(gmask, pr_me, min(j + u, nb - 1), lpr);
+                        if (writer && j + u < nb) put_grad(idx < U ? A.g_anchor : (PHASED ? A.g_phase : nullptr), pr,
+                                                          gpart[i]);
+                    }
+                }
+            }
+        }
+    } else {
+        // Narrow groups: the group walks its rows in batches of U, loading the
+        // batch's anchors and permutation entries, then its phases and gathered rows
+        // (U rows in flight), then processing the rows in order.  Rows past r1 in
+        // the last batch repeat row r1-1 for the loads and are skipped.
+        for (int64_t rb = r0; rb < r1; rb += U) {
+            float qv[U], tv[U];
+            uint32_t pv[U];
+            float hv[U][VEC];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t r = min(rb + u, r1 - 1);
+                qv[u] = __ldg(A.s + r);
+                pv[u] = min(__ldg(A.perm + r), (uint32_t)(A.m - 1));
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                tv[u] = PHASED ? __ldg(A.theta + pv[u]) : 0.f;
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) hv[u][v] = 0.f;
+                if (ROWS && cval) load_vec<VEC>(A.rows + (int64_t)pv[u] * B + c0, hv[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (rb + u >= r1) break;
+                const float q = qv[u];
+                float sn = 0.f, cs = 1.f;
+                if (PHASED) sincosf(tv[u], &sn, &cs);
+                while (m < ms && __ldg(A.sp + m) < q) ++m;
+                if (mp < m) mp = m;
+                while (mp < ms && __ldg(A.sp + mp) <= q) ++mp;
+                const float eL = (m > 0) ? expf(__ldg(A.sp + m - 1) - q) : 0.f;
+                const float eR = (mp < ms) ? expf(q - __ldg(A.sp + mp)) : 0.f;
+                float ga = 0.f, gp = 0.f;
+                row(pv[u], cs, sn, eL, eR, m, mp, hv[u], ga, gp);
+                if (GRAD) {
+                    for (int off = lpr >> 1; off >= 1; off >>= 1) {
+                        ga += __shfl_xor_sync(gmask, ga, off);
+                        if (PHASED) gp += __shfl_xor_sync(gmask, gp, off);
+                    }
+                    if (gl == 0) {
+                        put_grad(A.g_anchor, pv[u], ga);
+                        if (PHASED) put_grad(A.g_phase, pv[u], gp);
                     }
                 }
             }
@@ -666,17 +798,48 @@ cudaError_t side_scan(const RectPlan& p, SideScan a, bool bins, int32_t* status,
 #undef SIDE_CASE
 }
 
+#define LAPLEX_TRY(expr)                     \
+    do {                                     \
+        cudaError_t e_ = (expr);             \
+        if (e_ != cudaSuccess) return e_;    \
+    } while (0)
+
+// One launch of k_large<VEC, PHASED, MODE>: a grid of one wave at the kernel's
+// occupancy (resident blocks per SM are queried once per instantiation), each
+// group walking an equal contiguous run of rows, at least kLargeMinRows of them.
+constexpr int64_t kLargeMinRows = 64;
+
+template <int VEC, bool PHASED, int MODE>
+cudaError_t launch_large(LargePass A, int chunks, const char* name, cudaStream_t st) {
+    static int occ = 0;
+    if (occ == 0) {
+        int o = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large<VEC, PHASED, MODE>, 256, 0) != cudaSuccess)
+            o = 1;
+        occ = std::max(o, 1);
+    }
+    const int64_t groups_per_block = 8 * (32 / A.lpr);
+    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ / chunks);
+    const int64_t need = (A.m + groups_per_block * kLargeMinRows - 1) / (groups_per_block * kLargeMinRows);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
+    A.rows_per_group = (A.m + blocks * groups_per_block - 1) / (blocks * groups_per_block);
+    const dim3 grid((unsigned)blocks, (unsigned)chunks);
+    LAPLEX_TIMED(name, st, k_large<VEC, PHASED, MODE><<<grid, 256, 0, st>>>(A));
+    return cudaGetLastError();
+}
+
 template <int VEC, bool PHASED>
-cudaError_t large_mode(LargePass A, int mode, dim3 grid, cudaStream_t st) {
+cudaError_t large_mode(LargePass A, int mode, int chunks, cudaStream_t st) {
     switch (mode) {
-        case kLmExpand: LAPLEX_TIMED("large_expand", st, k_large<VEC, PHASED, kLmExpand><<<grid, 256, 0, st>>>(A)); break;
-        case kLmAccum: LAPLEX_TIMED("large_accum", st, k_large<VEC, PHASED, kLmAccum><<<grid, 256, 0, st>>>(A)); break;
-        case kLmGrad: LAPLEX_TIMED("large_grad", st, k_large<VEC, PHASED, kLmGrad><<<grid, 256, 0, st>>>(A)); break;
-        case kLmExpand | kLmGrad: LAPLEX_TIMED("large_expand_grad", st, k_large<VEC, PHASED, kLmExpand | kLmGrad><<<grid, 256, 0, st>>>(A)); break;
-        case kLmAccum | kLmGrad: LAPLEX_TIMED("large_accum_grad", st, k_large<VEC, PHASED, kLmAccum | kLmGrad><<<grid, 256, 0, st>>>(A)); break;
+        case kLmExpand: return launch_large<VEC, PHASED, kLmExpand>(A, chunks, "large_expand", st);
+        case kLmAccum: return launch_large<VEC, PHASED, kLmAccum>(A, chunks, "large_accum", st);
+        case kLmGrad: return launch_large<VEC, PHASED, kLmGrad>(A, chunks, "large_grad", st);
+        case kLmExpand | kLmGrad:
+            return launch_large<VEC, PHASED, kLmExpand | kLmGrad>(A, chunks, "large_expand_grad", st);
+        case kLmAccum | kLmGrad:
+            return launch_large<VEC, PHASED, kLmAccum | kLmGrad>(A, chunks, "large_accum_grad", st);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
@@ -687,20 +850,12 @@ cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
     const int chunks = (A.B + lpr * vec - 1) / (lpr * vec);
     A.lpr = lpr;
     A.chunk_atomic = chunks > 1 ? 1 : 0;
-    const int64_t groups_per_block = 8 * (32 / lpr);
-    // enough groups to fill the GPU, each walking a contiguous run of rows
-    const int64_t min_rows = 64;
-    int64_t blocks = std::min<int64_t>((int64_t)sm_count() * 4, (A.m + groups_per_block * min_rows - 1) /
-                                                                     (groups_per_block * min_rows));
-    blocks = std::max<int64_t>(blocks, 1);
-    A.rows_per_group = (A.m + blocks * groups_per_block - 1) / (blocks * groups_per_block);
     if ((mode & kLmGrad) && A.chunk_atomic) {
-        if (A.g_anchor) cudaMemsetAsync(A.g_anchor, 0, sizeof(float) * A.m, st);
-        if (A.g_phase) cudaMemsetAsync(A.g_phase, 0, sizeof(float) * A.m, st);
+        if (A.g_anchor) LAPLEX_TRY(cudaMemsetAsync(A.g_anchor, 0, sizeof(float) * A.m, st));
+        if (A.g_phase) LAPLEX_TRY(cudaMemsetAsync(A.g_phase, 0, sizeof(float) * A.m, st));
     }
-    const dim3 grid((unsigned)blocks, (unsigned)chunks);
-    if (vec == 4) return phased ? large_mode<4, true>(A, mode, grid, st) : large_mode<4, false>(A, mode, grid, st);
-    return phased ? large_mode<1, true>(A, mode, grid, st) : large_mode<1, false>(A, mode, grid, st);
+    if (vec == 4) return phased ? large_mode<4, true>(A, mode, chunks, st) : large_mode<4, false>(A, mode, chunks, st);
+    return phased ? large_mode<1, true>(A, mode, chunks, st) : large_mode<1, false>(A, mode, chunks, st);
 }
 
 cudaError_t finish(Finish F, cudaStream_t st) {
@@ -760,11 +915,6 @@ LargePass large_args(Side L, Side Sm, const RectPlan& p, int64_t B) {
     return A;
 }
 
-#define LAPLEX_TRY(expr)                     \
-    do {                                     \
-        cudaError_t e_ = (expr);             \
-        if (e_ != cudaSuccess) return e_;    \
-    } while (0)
 
 // Reduce path of the forward: interval sums of x (at I) into O's bins, scan over
 // O, parts written to ZL/ZR/ZF.
