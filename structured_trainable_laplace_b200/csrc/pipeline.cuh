@@ -238,6 +238,17 @@ __device__ __forceinline__ LP lp_step_d(LP s, float dv, float l, float t) {
     return o;
 }
 
+// One step with a single input t sitting at the row (no interval part): the
+// common case of the symmetric scans.  Written without the zero interval input so
+// that no addition of +0 (which IEEE arithmetic may not drop) is issued.
+__device__ __forceinline__ LP lp_step_x(LP s, float dv, float t) {
+    const float d = fabsf(dv);
+    LP o;
+    o.P = fmaf(d, s.P, t);
+    o.L = (dv >= 0.f) ? d * s.P : s.L;
+    return o;
+}
+
 // A then B with the decay e = exp(u_A - u_B) and the break flag u_B > u_A given.
 __device__ __forceinline__ LP combine_e(LP A, LP B, float e, bool brk) {
     LP o;

@@ -160,8 +160,15 @@ struct ChainSet {
 // t+1, t+2, ... when REV).  Called by one full warp; lane c < C handles channel c.
 // tot: this lane's tile total (anchored at u_tile_end).  u_before_tile: oriented
 // anchor of the last row of the predecessor tile.  Returns the incoming carry
-// (anchored at u_before_tile) and whether one exists.  Waits are bounded: past
-// kSpinLimit polls the tile records kStatusTimeout and proceeds.
+// (anchored at u_before_tile) and whether one exists.
+//
+// The predecessors are read 32 at a time: lane i polls the flag of the i-th
+// predecessor of the window, a ballot finds the nearest one that holds an
+// inclusive state, and once every tile up to it has published, the channel lanes
+// prepend the window's states in order (their loads are independent).  A window
+// without an inclusive state is prepended whole and the next one is read.  Waits
+// are bounded: past kSpinLimit polls the tile records kStatusTimeout and
+// proceeds with what it has.
 template <int C, bool REV>
 __device__ __forceinline__ double2 lookback(Chain ch, int64_t t, int64_t T, const float* s, int64_t n, int64_t R, LP tot,
                                             float u_tile_end, float u_before_tile, int32_t* status, bool& has_carry) {
@@ -181,36 +188,50 @@ __device__ __forceinline__ double2 lookback(Chain ch, int64_t t, int64_t T, cons
     __threadfence();
     __syncwarp();
     if (lane == 0) st_release(&ch.flags[t], 1);
-    if (lane < C) {
-        int64_t j = REV ? t + 1 : t - 1;
-        bool have = false;
-        while (true) {
-            int f;
-            uint32_t spins = 0;
-            while ((f = ld_acquire(&ch.flags[j])) == 0) {
-                if (++spins > kSpinLimit) {
-                    raise_status(status, kStatusTimeout);
-                    f = 3;
-                    break;
-                }
+    bool have = false;
+    int64_t jb = REV ? t + 1 : t - 1;  // nearest predecessor of the window
+    uint32_t spins = 0;
+    bool timed_out = false;
+    while (true) {
+        const int64_t jl = REV ? jb + lane : jb - lane;  // this lane's predecessor
+        const bool exists = REV ? (jl < T) : (jl >= 0);
+        // 3 marks a slot past the end tile (which always publishes an inclusive
+        // state, so the window never takes one)
+        int f = exists ? ld_acquire(&ch.flags[jl]) : 3;
+        unsigned incl = __ballot_sync(0xffffffffu, f >= 2);
+        unsigned zero = __ballot_sync(0xffffffffu, f == 0);
+        const int stop = incl ? __ffs(incl) - 1 : 31;           // last window slot to take
+        const unsigned need = (stop == 31) ? 0xffffffffu : ((2u << stop) - 1u);
+        if ((zero & need) != 0u && !timed_out) {
+            if (++spins > kSpinLimit) {
+                if (lane == 0) raise_status(status, kStatusTimeout);
+                timed_out = true;
+            } else {
                 __nanosleep(64);
             }
-            double2 v = make_double2(0.0, 0.0);
-            if (f == 1) v = __ldcg(&ch.agg[j * C + lane]);
-            if (f == 2) v = __ldcg(&ch.inc[j * C + lane]);
-            const float uj = REV ? -s[j * R] : s[min(n, (j + 1) * R) - 1];
-            run = have ? lpd_combine(v, uj, run, u_before_tile) : v;
-            have = true;
-            if (f != 1) break;
-            j = REV ? j + 1 : j - 1;
-            if (j < 0 || j >= T) break;  // the end tile always publishes inclusive; never walk past it
+            continue;
         }
-        ch.inc[t * C + lane] = lpd_combine(run, u_before_tile, totd, u_tile_end);
+        // a slot still unpublished after the bound counts as zero
+        const float uj = exists ? (REV ? -s[jl * R] : s[min(n, (jl + 1) * R) - 1]) : 0.f;
+        for (int i = 0; i <= stop; ++i) {
+            const int fi = __shfl_sync(0xffffffffu, f, i);
+            const float ui = __shfl_sync(0xffffffffu, uj, i);
+            const int64_t ji = REV ? jb + i : jb - i;
+            const bool take = (fi == 1 || fi == 2);
+            if (lane < C && take) {
+                const double2 v = (fi == 1) ? __ldcg(&ch.agg[ji * C + lane]) : __ldcg(&ch.inc[ji * C + lane]);
+                run = have ? lpd_combine(v, ui, run, u_before_tile) : v;
+            }
+            have = have || take;
+        }
+        if (incl != 0u || timed_out) break;
+        jb = REV ? jb + 32 : jb - 32;
     }
+    if (lane < C) ch.inc[t * C + lane] = have ? lpd_combine(run, u_before_tile, totd, u_tile_end) : totd;
     __threadfence();
     __syncwarp();
     if (lane == 0) st_release(&ch.flags[t], 2);
-    has_carry = true;
+    has_carry = have;
     return run;
 }
 

@@ -62,7 +62,18 @@ struct SymGeo {
     static constexpr int R = G::R;  // rows per tile (SK * E)
 };
 
-inline int64_t rows_per_tile(int C) { return C <= 8 ? 32 * kE : (32 * kE * 8) / C; }
+// Single channel (B = 1): tiles of k1NT threads x k1E rows, loaded straight into
+// registers (see the one-channel kernels below).
+constexpr int k1NT = 256, k1E = 16, k1NW = k1NT / 32, k1R = k1NT * k1E;
+
+inline int64_t rows_per_tile(int C) {
+    return C == 1 ? k1R : (C <= 8 ? 32 * kE : (32 * kE * 8) / C);
+}
+
+template <int C>
+__host__ __device__ constexpr int tile_rows() {
+    return C == 1 ? k1R : SymGeo<C>::R;
+}
 
 __host__ __device__ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 
@@ -379,9 +390,9 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
         }
         LP sr[1] = {{0.f, 0.f}}, sl[1] = {{0.f, 0.f}};
 #pragma unroll
-        for (int e = E - 1; e >= 0; --e) sr[0] = lp_step_d(sr[0], dk[e + 1], 0.f, xv[e]);
+        for (int e = E - 1; e >= 0; --e) sr[0] = lp_step_x(sr[0], dk[e + 1], xv[e]);
 #pragma unroll
-        for (int e = 0; e < E; ++e) sl[0] = lp_step_d(sl[0], dk[e], 0.f, xv[e]);
+        for (int e = 0; e < E; ++e) sl[0] = lp_step_x(sl[0], dk[e], xv[e]);
         group_scan<SK, 1>(sl, sr, tb, k);
         const LP tl = shfl_lp(sl[0], SK - 1, SK);  // tile totals: left at the last segment, right at the first
         if (k == 0) {
@@ -401,73 +412,69 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
 
 // ------------------------------------------------------------------ pass B
 
-// One CTA of kCarryThreads per channel group.  Thread (c, q) owns block q of PS
-// consecutive ranges: it folds their aggregates in both directions (loads issued
-// kCarryBatch at a time, ahead of the dependent folds), the NB block aggregates
-// are scanned in shared memory by doubling (log2 NB steps), and each thread then
-// re-walks its block, writing the carry entering every range.
-constexpr int kCarryThreads = 512;
-constexpr int kCarryBatch = 8;
+// One CTA of kCarryThreads per channel group.  First every thread computes the
+// fp64 decays between consecutive range ends (shared by all channels) into
+// shared memory, so that the scans below are chains of fused multiply-adds only.
+// Thread (c, q) owns block q of PS consecutive ranges: it folds their aggregates
+// in both directions, the NB block aggregates are scanned in shared memory by
+// doubling (log2 NB steps), and each thread then re-walks its block, writing the
+// carry entering every range.
+constexpr int kCarryThreads = 1024;
+
+// Decay between the end anchors of two consecutive ranges, encoded with its break
+// flag: exp(uA - uB) when uB > uA, -1 for a tie (decay 1, no break).
+__device__ __forceinline__ double enc_decay_d(float uA, float uB) {
+    return (uB > uA) ? exp((double)uA - (double)uB) : -1.0;
+}
+
+__device__ __forceinline__ double2 fold_d(double2 A, double2 B, double ev) {
+    return combine_ed(A, B, fabs(ev), ev >= 0.0);
+}
 
 template <int C>
 __global__ void __launch_bounds__(kCarryThreads) k_sym_carry(SymScan a, RangeState st) {
-    constexpr int QS = kCarryThreads / C, U = kCarryBatch;
+    constexpr int QS = kCarryThreads / C;
     __shared__ double2 sL[QS][C], sR[QS][C];
-    __shared__ float eL[QS], eR[QS];  // oriented end anchor of each block, per direction
+    extern __shared__ double s_dec[];  // [2][P]: left decay into range j (from j-1), right decay into j (from j+1)
     const int grp = blockIdx.x;
     const int c = threadIdx.x % C, q = threadIdx.x / C;
     const int P = a.P;
     const int PS = (P + QS - 1) / QS, NB = (P + PS - 1) / PS;
     const int j0 = min(P, q * PS), j1 = min(P, j0 + PS);
-    const int64_t RR = a.tpr * (int64_t)SymGeo<C>::R;  // rows per range
+    const int64_t RR = a.tpr * (int64_t)tile_rows<C>();  // rows per range
     auto uL = [&](int jj) { return __ldg(a.s + min(a.n, (jj + 1) * RR) - 1); };  // left anchor of range jj
     auto uR = [&](int jj) { return -__ldg(a.s + jj * RR); };                    // right anchor of range jj
+    double* dL = s_dec;
+    double* dR = s_dec + P;
+    for (int jj = threadIdx.x; jj < P; jj += kCarryThreads) {
+        dL[jj] = jj > 0 ? enc_decay_d(uL(jj - 1), uL(jj)) : 0.0;
+        dR[jj] = jj + 1 < P ? enc_decay_d(uR(jj + 1), uR(jj)) : 0.0;
+    }
     const double2* Lagg = st.Lagg + (int64_t)grp * P * C + c;
     const double2* Ragg = st.Ragg + (int64_t)grp * P * C + c;
     const bool mine = q < NB;  // blocks q >= NB are empty
+    __syncthreads();
 
     // block aggregates (left: ranges j0 .. j1-1 in order; right: j1-1 .. j0)
-    double2 fl = make_double2(0.0, 0.0), fr = make_double2(0.0, 0.0);
-    float ufl = 0.f, ufr = 0.f;
     if (mine) {
-        for (int jb = j0; jb < j1; jb += U) {
-            double2 vl[U], vr[U];
-            float ul[U], ur[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int jl = jb + u, jr = j1 - 1 - (jb - j0) - u;
-                if (jl < j1) {
-                    vl[u] = Lagg[(int64_t)jl * C];
-                    ul[u] = uL(jl);
-                    vr[u] = Ragg[(int64_t)jr * C];
-                    ur[u] = uR(jr);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                if (jb + u < j1) {
-                    const bool first = (jb + u == j0);
-                    fl = first ? vl[u] : lpd_combine(fl, ufl, vl[u], ul[u]);
-                    fr = first ? vr[u] : lpd_combine(fr, ufr, vr[u], ur[u]);
-                    ufl = ul[u];
-                    ufr = ur[u];
-                }
-            }
+        double2 fl = Lagg[(int64_t)j0 * C], fr = Ragg[(int64_t)(j1 - 1) * C];
+        for (int u = 1; u < j1 - j0; ++u) {
+            const int jl = j0 + u, jr = j1 - 1 - u;
+            fl = fold_d(fl, Lagg[(int64_t)jl * C], dL[jl]);
+            fr = fold_d(fr, Ragg[(int64_t)jr * C], dR[jr]);
         }
         sL[q][c] = fl;
         sR[q][c] = fr;
-        if (c == 0) {
-            eL[q] = ufl;
-            eR[q] = ufr;
-        }
     }
     __syncthreads();
-    // inclusive scans over the blocks: left over 0..q, right over q..NB-1
+    // inclusive scans over the blocks: left over 0..q, right over q..NB-1; the decay
+    // between block q-off's end and block q's end is the product of the range
+    // decays between them, taken here as exp of the anchor difference
     for (int off = 1; off < NB; off <<= 1) {
         const bool dl = mine && q >= off, dr = mine && q + off < NB;
         double2 nl, nr;
-        if (dl) nl = lpd_combine(sL[q - off][c], eL[q - off], sL[q][c], eL[q]);
-        if (dr) nr = lpd_combine(sR[q + off][c], eR[q + off], sR[q][c], eR[q]);
+        if (dl) nl = fold_d(sL[q - off][c], sL[q][c], enc_decay_d(uL(min(P, (q - off + 1) * PS) - 1), uL(j1 - 1)));
+        if (dr) nr = fold_d(sR[q + off][c], sR[q][c], enc_decay_d(uR((q + off) * PS), uR(j0)));
         __syncthreads();
         if (dl) sL[q][c] = nl;
         if (dr) sR[q][c] = nr;
@@ -475,38 +482,18 @@ __global__ void __launch_bounds__(kCarryThreads) k_sym_carry(SymScan a, RangeSta
     }
     if (!mine) return;
     // carries entering the block, then entering each of its ranges
-    bool hl = q >= 1, hr = q + 1 < NB;
-    double2 cl = hl ? sL[q - 1][c] : make_double2(0.0, 0.0);
-    double2 cr = hr ? sR[q + 1][c] : make_double2(0.0, 0.0);
-    float ucl = hl ? eL[q - 1] : 0.f, ucr = hr ? eR[q + 1] : 0.f;
     double2* Lin = st.Lin + (int64_t)grp * P * C + c;
     double2* Rin = st.Rin + (int64_t)grp * P * C + c;
-    for (int jb = j0; jb < j1; jb += U) {
-        double2 vl[U], vr[U];
-        float ul[U], ur[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int jl = jb + u, jr = j1 - 1 - (jb - j0) - u;
-            if (jl < j1) {
-                vl[u] = Lagg[(int64_t)jl * C];
-                ul[u] = uL(jl);
-                vr[u] = Ragg[(int64_t)jr * C];
-                ur[u] = uR(jr);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int jl = jb + u, jr = j1 - 1 - (jb - j0) - u;
-            if (jl < j1) {
-                Lin[(int64_t)jl * C] = cl;  // zero (unused) for the first range
-                Rin[(int64_t)jr * C] = cr;  // zero (unused) for the last range
-                cl = hl ? lpd_combine(cl, ucl, vl[u], ul[u]) : vl[u];
-                cr = hr ? lpd_combine(cr, ucr, vr[u], ur[u]) : vr[u];
-                ucl = ul[u];
-                ucr = ur[u];
-                hl = hr = true;
-            }
-        }
+    const bool hl = q >= 1, hr = q + 1 < NB;
+    double2 cl = hl ? sL[q - 1][c] : make_double2(0.0, 0.0);
+    double2 cr = hr ? sR[q + 1][c] : make_double2(0.0, 0.0);
+    for (int u = 0; u < j1 - j0; ++u) {
+        const int jl = j0 + u, jr = j1 - 1 - u;
+        Lin[(int64_t)jl * C] = cl;  // zero (unused) for the first range
+        Rin[(int64_t)jr * C] = cr;  // zero (unused) for the last range
+        const double2 vl = Lagg[(int64_t)jl * C], vr = Ragg[(int64_t)jr * C];
+        cl = (hl || u > 0) ? fold_d(cl, vl, dL[jl]) : vl;
+        cr = (hr || u > 0) ? fold_d(cr, vr, dR[jr]) : vr;
     }
 }
 
@@ -682,9 +669,9 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 sr[w] = LP{0.f, 0.f};
                 sl[w] = LP{0.f, 0.f};
 #pragma unroll
-                for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_d(sr[w], dk[e + 1], 0.f, xr[w][e]);
+                for (int e = E - 1; e >= 0; --e) sr[w] = lp_step_x(sr[w], dk[e + 1], xr[w][e]);
 #pragma unroll
-                for (int e = 0; e < E; ++e) sl[w] = lp_step_d(sl[w], dk[e], 0.f, xr[w][e]);
+                for (int e = 0; e < E; ++e) sl[w] = lp_step_x(sl[w], dk[e], xr[w][e]);
             }
             group_scan<SK, NV>(sl, sr, tb, k);  // now inclusive over segments 0..k (left) / k..SK-1 (right)
             LP cL[NV], cR[NV];
@@ -722,8 +709,8 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
                 const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e + 1];
-                ax = lp_step_d(ax, dv, 0.f, xe);
-                ag = lp_step_d(ag, dv, 0.f, ge);
+                ax = lp_step_x(ax, dv, xe);
+                ag = lp_step_x(ag, dv, ge);
                 ob[e * C] = ag.P - ge;               // gx, right part
                 gap[e] = fmaf(ge, ax.L, xe * ag.L);  // strict right sums
             }
@@ -732,10 +719,10 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
 #pragma unroll
             for (int e = 0; e < E; ++e) {
                 const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e];
-                ax = lp_step_d(ax, dv, 0.f, xe);
-                ag = lp_step_d(ag, dv, 0.f, ge);
+                ax = lp_step_x(ax, dv, xe);
+                ag = lp_step_x(ag, dv, ge);
                 ob[e * C] += ag.P;                            // gx
-                gap[e] = gap[e] - fmaf(ge, ax.L, xe * ag.L);  // this channel's share of ga
+                gap[e] = fmaf(-ge, ax.L, fmaf(-xe, ag.L, gap[e]));  // this channel's share of ga
             }
             // sum over the warp's channels, then one padded row per warp in shared memory
             reduce_scatter<CW, SK>(gap, cs);
@@ -761,6 +748,350 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                     st_hint(ga + row, acc, pol_l);  // kept in L2 until its lines are complete
             }
         }
+    }
+}
+
+// ------------------------------------------------------- one channel (B = 1)
+//
+// With a single channel every row carries 4 bytes, so staging tiles in shared
+// memory would cost as much as the rows themselves and would cap the CTAs per
+// SM.  Instead thread q of a tile owns rows lo + q*k1E .. + k1E - 1: it loads
+// their anchors and permutation entries with 16-byte loads, gathers (aggregate
+// pass) or streams (sweeps) their values into registers, and scatters its
+// outputs through the permutation itself; many tiles' gathers are in flight per
+// SM.  The tile's scans: a sequential pass per thread, a shuffle scan over the
+// warp's 32 segments, and a pass over the k1NW warp totals in shared memory.
+// The base ranges, range aggregates, carries and the saved state are those of
+// the multi-channel kernels with C = 1 and tiles of k1R rows.
+
+struct Rows1 {
+    float a[k1E];       // anchors, kHighAnchor past n
+    uint32_t p[k1E];    // permutation entries (clamped), 0 past n
+    float ap, an;       // anchors of the rows just before / after the segment
+    int64_t row0;
+};
+
+__device__ __forceinline__ void load_rows1(const float* __restrict__ s, const uint32_t* __restrict__ perm, int64_t n,
+                                           int64_t row0, Rows1& r) {
+    r.row0 = row0;
+    const uint32_t last = (uint32_t)(n - 1);
+    if (row0 + k1E <= n) {
+#pragma unroll
+        for (int q = 0; q < k1E / 4; ++q) {
+            const float4 av = __ldg(reinterpret_cast<const float4*>(s + row0) + q);
+            const uint4 pv = __ldg(reinterpret_cast<const uint4*>(perm + row0) + q);
+            r.a[4 * q] = av.x, r.a[4 * q + 1] = av.y, r.a[4 * q + 2] = av.z, r.a[4 * q + 3] = av.w;
+            r.p[4 * q] = min(pv.x, last), r.p[4 * q + 1] = min(pv.y, last);
+            r.p[4 * q + 2] = min(pv.z, last), r.p[4 * q + 3] = min(pv.w, last);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < k1E; ++e) {
+            const bool in = row0 + e < n;
+            r.a[e] = in ? __ldg(s + row0 + e) : kHighAnchor;
+            r.p[e] = in ? min(__ldg(perm + row0 + e), last) : 0u;
+        }
+    }
+    r.ap = (row0 == 0) ? kLowAnchor : (row0 - 1 < n ? __ldg(s + row0 - 1) : kHighAnchor);
+    r.an = (row0 + k1E < n) ? __ldg(s + row0 + k1E) : kHighAnchor;
+}
+
+// Encoded decays into each row from the row before it (d[0] from ap), and d[k1E]
+// from the last row to the row after the segment (see enc_decay).
+__device__ __forceinline__ void decays1(const Rows1& r, float (&d)[k1E + 1]) {
+    d[0] = enc_decay(r.ap, r.a[0]);
+#pragma unroll
+    for (int e = 1; e < k1E; ++e) d[e] = enc_decay(r.a[e - 1], r.a[e]);
+    d[k1E] = enc_decay(r.a[k1E - 1], r.an);
+}
+
+// Inclusive shuffle scans over the 32 segments of a warp, left (over lanes
+// 0..lane, anchored at the lane's last row) and right (lanes lane..31, anchored
+// at -its first row), NV vectors.
+template <int NV>
+__device__ __forceinline__ void warp_scan1(LP (&l)[NV], LP (&rr)[NV], float ul, float ur) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float uo_l = __shfl_up_sync(0xffffffffu, ul, off);
+        const float uo_r = __shfl_down_sync(0xffffffffu, ur, off);
+        const float evl = enc_decay(uo_l, ul), evr = enc_decay(uo_r, ur);
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            LP ol, orr;
+            ol.L = __shfl_up_sync(0xffffffffu, l[v].L, off);
+            ol.P = __shfl_up_sync(0xffffffffu, l[v].P, off);
+            orr.L = __shfl_down_sync(0xffffffffu, rr[v].L, off);
+            orr.P = __shfl_down_sync(0xffffffffu, rr[v].P, off);
+            if (lane >= off) l[v] = combine_v(ol, l[v], evl);
+            if (lane + off < 32) rr[v] = combine_v(orr, rr[v], evr);
+        }
+    }
+}
+
+// Cross-warp scratch of one tile.
+template <int NV>
+struct Cross1 {
+    LP wl[NV][k1NW], wr[NV][k1NW];  // warp inclusive totals
+    float ul[k1NW], ur[k1NW];       // left: anchor of the warp's last row; right: -anchor of its first row
+    LP xl[NV][k1NW], xr[NV][k1NW];  // exclusive states entering each warp (from the warps before / after)
+    LP tl[NV], tr[NV];              // tile totals
+    LP cl[NV], cr[NV];              // tile carries (sweeps)
+    bool hl, hr;                    // carries present
+};
+
+// Warp totals -> exclusive states per warp and the tile totals.  Threads 0 ..
+// k1NW-1 each serve one warp; one __syncthreads inside, the caller syncs after.
+template <int NV>
+__device__ __forceinline__ void cross_warps1(Cross1<NV>& cx) {
+    __syncthreads();
+    const int w = threadIdx.x;
+    if (w < k1NW) {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+            LP acc = {0.f, 0.f};
+            float ua = 0.f;
+            for (int j = 0; j < w; ++j) {
+                acc = (j == 0) ? cx.wl[v][0] : lp_combine(acc, ua, cx.wl[v][j], cx.ul[j]);
+                ua = cx.ul[j];
+            }
+            cx.xl[v][w] = acc;
+            if (w == k1NW - 1) cx.tl[v] = (w == 0) ? cx.wl[v][w] : lp_combine(acc, ua, cx.wl[v][w], cx.ul[w]);
+            acc = LP{0.f, 0.f};
+            for (int j = k1NW - 1; j > w; --j) {
+                acc = (j == k1NW - 1) ? cx.wr[v][j] : lp_combine(acc, ua, cx.wr[v][j], cx.ur[j]);
+                ua = cx.ur[j];
+            }
+            cx.xr[v][w] = acc;
+            if (w == 0) cx.tr[v] = (k1NW == 1) ? cx.wr[v][0] : lp_combine(acc, ua, cx.wr[v][0], cx.ur[0]);
+        }
+    }
+}
+
+// Aggregate pass for one channel: walks its base ranges' tiles right to left,
+// writes the sorted copy, RS and the range aggregates (as k_sym_agg).
+__global__ void __launch_bounds__(k1NT, 3) k_sym1_agg(SymScan a, const float* __restrict__ v, RangeState st,
+                                                     float* __restrict__ vs) {
+    __shared__ Cross1<1> cx;
+    const CtaTiles w = cta_tiles(a);
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    auto range_end = [&](int64_t J) { return __ldg(a.s + min(a.n, (J + 1) * a.tpr * (int64_t)k1R) - 1); };
+    double2 runR = make_double2(0.0, 0.0), runL = make_double2(0.0, 0.0);
+    for (int64_t t = w.te - 1; t >= w.tb; --t) {
+        const int64_t lo = t * (int64_t)k1R, J = t / a.tpr;
+        Rows1 r;
+        load_rows1(a.s, a.perm, a.n, lo + threadIdx.x * k1E, r);
+        float x[k1E];
+#pragma unroll
+        for (int e = 0; e < k1E; ++e) x[e] = (r.row0 + e < a.n) ? __ldg(v + r.p[e]) : 0.f;
+        {
+            float4* dst = reinterpret_cast<float4*>(vs + r.row0);
+#pragma unroll
+            for (int q = 0; q < k1E / 4; ++q) __stcs(dst + q, make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
+        }
+        float d[k1E + 1];
+        decays1(r, d);
+        LP sl[1] = {{0.f, 0.f}}, sr[1] = {{0.f, 0.f}};
+#pragma unroll
+        for (int e = k1E - 1; e >= 0; --e) sr[0] = lp_step_x(sr[0], d[e + 1], x[e]);
+#pragma unroll
+        for (int e = 0; e < k1E; ++e) sl[0] = lp_step_x(sl[0], d[e], x[e]);
+        warp_scan1<1>(sl, sr, r.a[k1E - 1], -r.a[0]);
+        if (lane == 31) {
+            cx.wl[0][wp] = sl[0];
+            cx.ul[wp] = r.a[k1E - 1];
+        }
+        if (lane == 0) {
+            cx.wr[0][wp] = sr[0];
+            cx.ur[wp] = -r.a[0];
+        }
+        cross_warps1<1>(cx);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const float f0 = __ldg(a.s + lo);                                    // the tile's first row
+            const float fa = (lo + k1R < a.n) ? __ldg(a.s + lo + k1R) : kHighAnchor;  // the row after it
+            const float fl = (lo + k1R <= a.n) ? __ldg(a.s + lo + k1R - 1) : kHighAnchor;  // its last row
+            const float ue = range_end(J);
+            const bool last_of_range = (t + 1 == min(a.T, (J + 1) * a.tpr));
+            const double2 trd = to_d2(cx.tr[0]), tld = to_d2(cx.tl[0]);
+            const bool br = fa > f0, bl = ue > fl;
+            runR = last_of_range ? trd : combine_ed(runR, trd, br ? exp((double)f0 - (double)fa) : 1.0, br);
+            st.RS[t] = runR;
+            runL = last_of_range ? tld : combine_ed(tld, runL, bl ? exp((double)fl - (double)ue) : 1.0, bl);
+            if (t == J * a.tpr) {
+                st.Lagg[J] = runL;
+                st.Ragg[J] = runR;
+            }
+        }
+        __syncthreads();  // cx is rewritten by the next tile
+    }
+}
+
+// Sweep for one channel: NV = 1 forward (xs -> y), NV = 2 backward (xs, gs -> gx,
+// ga), from the sorted copies, RS and the range carries (as k_sym_sweep).
+template <int NV>
+__global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a, const float* __restrict__ xs,
+                                                       const float* __restrict__ gs, RangeState sx, RangeState sg,
+                                                       float* __restrict__ out, float* __restrict__ ga) {
+    __shared__ Cross1<NV> cx;
+    __shared__ double2 s_runL[NV];
+    const CtaTiles cw = cta_tiles(a);
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    if (threadIdx.x < NV) {
+        const RangeState& sv = (threadIdx.x == 0) ? sx : sg;
+        s_runL[threadIdx.x] = (cw.J0 > 0) ? sv.Lin[cw.J0] : make_double2(0.0, 0.0);
+    }
+    bool hasL = (cw.J0 > 0);
+    __syncthreads();
+    for (int64_t t = cw.tb; t < cw.te; ++t) {
+        const int64_t lo = t * (int64_t)k1R, J = t / a.tpr;
+        const bool more = (t + 1 < min(a.T, (J + 1) * a.tpr)), hasRin = (J + 1 < a.P);
+        Rows1 r;
+        load_rows1(a.s, a.perm, a.n, lo + threadIdx.x * k1E, r);
+        float xv[NV][k1E];
+#pragma unroll
+        for (int vv = 0; vv < NV; ++vv) {
+            const float4* src = reinterpret_cast<const float4*>((vv == 0 ? xs : gs) + r.row0);
+#pragma unroll
+            for (int q = 0; q < k1E / 4; ++q) {
+                const float4 f = __ldcs(src + q);
+                xv[vv][4 * q] = f.x, xv[vv][4 * q + 1] = f.y, xv[vv][4 * q + 2] = f.z, xv[vv][4 * q + 3] = f.w;
+            }
+        }
+        // tile carries (thread 0, fp64): left = the running fold, right = RS of the
+        // next tile of the range after the range's own right carry
+        if (threadIdx.x == 0) {
+            const float fa = (lo + k1R < a.n) ? __ldg(a.s + lo + k1R) : kHighAnchor;
+            const float ur = -__ldg(a.s + min(a.n - 1, (J + 1) * a.tpr * (int64_t)k1R));
+            const bool brr = -fa > ur;
+            const double er = brr ? exp((double)ur + (double)fa) : 1.0;
+#pragma unroll
+            for (int vv = 0; vv < NV; ++vv) {
+                const RangeState& sv = (vv == 0) ? sx : sg;
+                double2 crd = hasRin ? sv.Rin[J] : make_double2(0.0, 0.0);
+                if (more) {
+                    const double2 rsn = sv.RS[t + 1];
+                    crd = hasRin ? combine_ed(crd, rsn, er, brr) : rsn;
+                }
+                cx.cr[vv] = LP{(float)crd.x, (float)crd.y};
+                cx.cl[vv] = LP{(float)s_runL[vv].x, (float)s_runL[vv].y};
+            }
+            cx.hl = hasL;
+            cx.hr = hasRin || more;
+        }
+        float d[k1E + 1];
+        decays1(r, d);
+        LP sl[NV], sr[NV];
+#pragma unroll
+        for (int vv = 0; vv < NV; ++vv) {
+            sl[vv] = LP{0.f, 0.f};
+            sr[vv] = LP{0.f, 0.f};
+#pragma unroll
+            for (int e = k1E - 1; e >= 0; --e) sr[vv] = lp_step_x(sr[vv], d[e + 1], xv[vv][e]);
+#pragma unroll
+            for (int e = 0; e < k1E; ++e) sl[vv] = lp_step_x(sl[vv], d[e], xv[vv][e]);
+        }
+        warp_scan1<NV>(sl, sr, r.a[k1E - 1], -r.a[0]);
+        if (lane == 31) {
+#pragma unroll
+            for (int vv = 0; vv < NV; ++vv) cx.wl[vv][wp] = sl[vv];
+            cx.ul[wp] = r.a[k1E - 1];
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int vv = 0; vv < NV; ++vv) cx.wr[vv][wp] = sr[vv];
+            cx.ur[wp] = -r.a[0];
+        }
+        cross_warps1<NV>(cx);
+        __syncthreads();
+        // incoming states of this thread's segment: tile carry, then the warps
+        // before (after), then the lanes before (after) in this warp
+        const float u_tile_l = (lo > 0) ? __ldg(a.s + lo - 1) : kLowAnchor;          // row before the tile
+        const float u_tile_r = -((lo + k1R < a.n) ? __ldg(a.s + lo + k1R) : kHighAnchor);  // -row after it
+        const float u_warp_l = (wp > 0) ? cx.ul[wp - 1] : u_tile_l;
+        const float u_warp_r = (wp + 1 < k1NW) ? cx.ur[wp + 1] : u_tile_r;
+        LP inL[NV], inR[NV];
+#pragma unroll
+        for (int vv = 0; vv < NV; ++vv) {
+            // left
+            bool h = cx.hl;
+            LP acc = cx.cl[vv];
+            if (wp > 0) {
+                acc = h ? lp_combine(acc, u_tile_l, cx.xl[vv][wp], u_warp_l) : cx.xl[vv][wp];
+                h = true;
+            }
+            const LP exl = shfl_lp(sl[vv], (lane - 1) & 31, 32);
+            if (lane > 0) {
+                acc = h ? lp_combine(acc, u_warp_l, exl, r.ap) : exl;
+                h = true;
+            }
+            inL[vv] = h ? acc : LP{0.f, 0.f};
+            // right
+            h = cx.hr;
+            acc = cx.cr[vv];
+            if (wp + 1 < k1NW) {
+                acc = h ? lp_combine(acc, u_tile_r, cx.xr[vv][wp], u_warp_r) : cx.xr[vv][wp];
+                h = true;
+            }
+            const LP exr = shfl_lp(sr[vv], (lane + 1) & 31, 32);
+            if (lane < 31) {
+                acc = h ? lp_combine(acc, u_warp_r, exr, -r.an) : exr;
+                h = true;
+            }
+            inR[vv] = h ? acc : LP{0.f, 0.f};
+        }
+        // the fold of the tile's left total into the running carry (thread 0, after
+        // every thread has read the carries above)
+        const LP tl0 = cx.tl[0], tl1 = cx.tl[NV - 1];
+        if (NV == 1) {
+            float pr = inR[0].P, pl = inL[0].P;
+            float yv[k1E];
+#pragma unroll
+            for (int e = k1E - 1; e >= 0; --e) {
+                pr = fmaf(fabsf(d[e + 1]), pr, xv[0][e]);
+                yv[e] = pr - xv[0][e];
+            }
+#pragma unroll
+            for (int e = 0; e < k1E; ++e) {
+                pl = fmaf(fabsf(d[e]), pl, xv[0][e]);
+                if (r.row0 + e < a.n) __stcs(out + r.p[e], yv[e] + pl);
+            }
+        } else {
+            LP ax = inR[0], ag = inR[NV - 1];
+            float gxr[k1E], gap[k1E];
+#pragma unroll
+            for (int e = k1E - 1; e >= 0; --e) {
+                const float xe = xv[0][e], ge = xv[NV - 1][e], dv = d[e + 1];
+                ax = lp_step_x(ax, dv, xe);
+                ag = lp_step_x(ag, dv, ge);
+                gxr[e] = ag.P - ge;
+                gap[e] = fmaf(ge, ax.L, xe * ag.L);  // strict right sums
+            }
+            ax = inL[0];
+            ag = inL[NV - 1];
+#pragma unroll
+            for (int e = 0; e < k1E; ++e) {
+                const float xe = xv[0][e], ge = xv[NV - 1][e], dv = d[e];
+                ax = lp_step_x(ax, dv, xe);
+                ag = lp_step_x(ag, dv, ge);
+                if (r.row0 + e < a.n) {
+                    if (out != nullptr) __stcs(out + r.p[e], gxr[e] + ag.P);
+                    if (ga != nullptr) __stcs(ga + r.p[e], fmaf(-ge, ax.L, fmaf(-xe, ag.L, gap[e])));
+                }
+            }
+        }
+        if (threadIdx.x == 0) {
+            const float fl = (lo + k1R <= a.n) ? __ldg(a.s + lo + k1R - 1) : kHighAnchor;
+            const bool bl = fl > u_tile_l;
+            const double el = bl ? exp((double)u_tile_l - (double)fl) : 1.0;
+#pragma unroll
+            for (int vv = 0; vv < NV; ++vv) {
+                const LP tlv = (vv == 0) ? tl0 : tl1;
+                s_runL[vv] = hasL ? combine_ed(s_runL[vv], to_d2(tlv), el, bl) : to_d2(tlv);
+            }
+        }
+        hasL = true;
+        __syncthreads();  // cx and s_runL are rewritten by the next tile
     }
 }
 
@@ -845,14 +1176,53 @@ SymScan scan_args(const SymPlan& p, const float* s, const uint32_t* perm, int64_
 template <int C>
 cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms,
                          const float* v, RangeState st, float* vs, cudaStream_t stream) {
-    using SM = AggSmem<C, kAheadAgg>;
-    static int occ_cache = 0;
-    const int occ = prepare(k_sym_agg<C, kAheadAgg>, SymGeo<C>::NT, sizeof(SM), occ_cache);
-    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
-    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
-    LAPLEX_TIMED("sym_agg", stream,
-                 k_sym_agg<C, kAheadAgg><<<grid, SymGeo<C>::NT, sizeof(SM), stream>>>(a, v, st, vs));
-    LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, kCarryThreads, 0, stream>>>(a, st));
+    if constexpr (C == 1) {
+        static int occ_cache = 0;
+        const int occ = prepare(k_sym1_agg, k1NT, 0, occ_cache);
+        const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+        const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
+        LAPLEX_TIMED("sym_agg", stream, k_sym1_agg<<<grid, k1NT, 0, stream>>>(a, v, st, vs));
+    } else {
+        using SM = AggSmem<C, kAheadAgg>;
+        static int occ_cache = 0;
+        const int occ = prepare(k_sym_agg<C, kAheadAgg>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+        const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+        const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
+        LAPLEX_TIMED("sym_agg", stream,
+                     k_sym_agg<C, kAheadAgg><<<grid, SymGeo<C>::NT, sizeof(SM), stream>>>(a, v, st, vs));
+    }
+    const SymScan a = scan_args(p, s, perm, n, B, sms, 1);
+    const size_t dsm = sizeof(double) * 2 * (size_t)p.P;
+    static int carry_ready = 0;
+    if (!carry_ready) {
+        cudaFuncSetAttribute(k_sym_carry<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(sizeof(double) * 2 * kMaxRanges));
+        carry_ready = 1;
+    }
+    LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, kCarryThreads, dsm, stream>>>(a, st));
+    return cudaGetLastError();
+}
+
+// The forward sweep (y from the sorted copy, RS and the range carries).
+template <int C>
+cudaError_t launch_sym_sweep_fwd(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms,
+                                 const float* xs, const RangeState& sx, float* y, cudaStream_t st) {
+    if constexpr (C == 1) {
+        static int occ_cache = 0;
+        const int occ = prepare(k_sym1_sweep<1>, k1NT, 0, occ_cache);
+        const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+        const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
+        LAPLEX_TIMED("sym_fwd", st, k_sym1_sweep<1><<<grid, k1NT, 0, st>>>(a, xs, nullptr, sx, sx, y, nullptr));
+    } else {
+        using SM = SweepSmem<C, 1, kAheadFwd>;
+        static int occ_cache = 0;
+        const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+        const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+        const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
+        LAPLEX_TIMED("sym_fwd", st,
+                     k_sym_sweep<C, 1, kAheadFwd>
+                     <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, nullptr, sx, sx, y, nullptr, 0));
+    }
     return cudaGetLastError();
 }
 
@@ -872,15 +1242,7 @@ cudaError_t sym_forward_t(const float* s, const uint32_t* perm, int64_t n, const
     }
     cudaError_t e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
     if (e != cudaSuccess) return e;
-    using SM = SweepSmem<C, 1, kAheadFwd>;
-    static int occ_cache = 0;
-    const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
-    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
-    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
-    LAPLEX_TIMED("sym_fwd", st,
-                 k_sym_sweep<C, 1, kAheadFwd>
-                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, nullptr, sx, sx, y, nullptr, 0));
-    return cudaGetLastError();
+    return launch_sym_sweep_fwd<C>(p, s, perm, n, B, sms, xs, sx, y, st);
 }
 
 template <int C>
@@ -910,14 +1272,22 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
     }
     e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, gs, st);
     if (e != cudaSuccess) return e;
-    using SM = SweepSmem<C, 2, kAheadBwd>;
-    static int occ_cache = 0;
-    const int occ = prepare(k_sym_sweep<C, 2, kAheadBwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
-    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
-    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
-    LAPLEX_TIMED("sym_bwd", st,
-                 k_sym_sweep<C, 2, kAheadBwd>
-                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, gs, sx, sg, gx, ga, p.G > 1 ? 1 : 0));
+    if constexpr (C == 1) {
+        static int occ_cache = 0;
+        const int occ = prepare(k_sym1_sweep<2>, k1NT, 0, occ_cache);
+        const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+        const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
+        LAPLEX_TIMED("sym_bwd", st, k_sym1_sweep<2><<<grid, k1NT, 0, st>>>(a, xs, gs, sx, sg, gx, ga));
+    } else {
+        using SM = SweepSmem<C, 2, kAheadBwd>;
+        static int occ_cache = 0;
+        const int occ = prepare(k_sym_sweep<C, 2, kAheadBwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+        const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
+        const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
+        LAPLEX_TIMED("sym_bwd", st,
+                     k_sym_sweep<C, 2, kAheadBwd>
+                     <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, gs, sx, sg, gx, ga, p.G > 1 ? 1 : 0));
+    }
     return cudaGetLastError();
 }
 
@@ -1009,15 +1379,7 @@ cudaError_t sym_forward_static_t(const float* s, const uint32_t* perm, int64_t n
     float* xs = (float*)((char*)scratch + state);
     e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
     if (e != cudaSuccess) return e;
-    using SM = SweepSmem<C, 1, kAheadFwd>;
-    static int occ_cache = 0;
-    const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
-    const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
-    const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
-    LAPLEX_TIMED("sym_fwd", st,
-                 k_sym_sweep<C, 1, kAheadFwd>
-                 <<<grid, SymGeo<C>::NT, sizeof(SM), st>>>(a, xs, nullptr, sx, sx, y, nullptr, 0));
-    return cudaGetLastError();
+    return launch_sym_sweep_fwd<C>(p, s, perm, n, B, sms, xs, sx, y, st);
 }
 
 }  // namespace
