@@ -5,8 +5,8 @@
 // Keys are the order-preserving uint32 images of the anchors (-0 folded onto
 // +0), values the original indices.  Least-significant digit first, 4 passes of
 // 8 bits.  Each pass is one kernel over tiles of 4096 keys claimed in order from
-// an atomic counter: the tile ranks its keys stably inside each warp (match-any
-// over the digit), publishes its per-digit counts, looks back over the tiles
+// an atomic counter: the tile ranks its keys stably inside each warp (the lanes
+// sharing a digit found by ballots over its bits), publishes its per-digit counts, looks back over the tiles
 // before it for their per-digit prefixes (bounded waits), and scatters through
 // shared memory so that runs of equal digits leave as contiguous stores.
 // A histogram kernel computes the four global digit histograms in one read of
@@ -142,13 +142,23 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
     }
     // stable rank inside the warp, items in (i, lane) order = index order.  The
     // masks of lanes holding the same digit do not depend on the running counts,
-    // so all are formed first (independent match operations); only the count
-    // updates form a chain.  rank[] holds the mask until the rank replaces it.
+    // so all are formed first; only the count updates form a chain.  Each mask is
+    // the AND over the digit's 8 bits of the ballot of lanes agreeing on that bit
+    // (plus the ballot of valid lanes, so that rows past n group apart).  rank[]
+    // holds the mask until the rank replaces it.
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
         const bool valid = wbase + i * 32 + lane < n;
         const uint32_t d = (key[i] >> shift) & 0xffu;
-        rank[i] = __match_any_sync(0xffffffffu, valid ? d : 0x100u);  // rows past n group apart
+        const uint32_t vb = __ballot_sync(0xffffffffu, valid);
+        uint32_t peers = valid ? vb : ~vb;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const bool bit = (d >> b) & 1u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, bit);
+            peers &= bit ? bal : ~bal;
+        }
+        rank[i] = peers;
     }
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
