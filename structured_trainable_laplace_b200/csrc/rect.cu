@@ -316,15 +316,14 @@ __device__ __forceinline__ void store_vec(float* p, const float (&v)[VEC]) {
     }
 }
 
-// Rows per prefetch batch of k_large: as many as the registers allow next to the
-// accumulators (the phased, 4-channel variants carry twice the state).
+// Rows per prefetch batch of k_large (gathered rows in flight per group).
 template <int VEC, bool PHASED, int MODE>
-constexpr int kLargeBatch = (VEC == 4 && PHASED) ? 4 : 8;
+constexpr int kLargeBatch = 8;
 
 // Each group of `lpr` lanes walks a contiguous range of sorted large-side rows;
 // lane gl of the group owns channels c0 .. c0+VEC-1 of every row.
 template <int VEC, bool PHASED, int MODE>
-__global__ void __launch_bounds__(256) k_large(LargePass A) {
+__global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
     constexpr int NP = PHASED ? 2 : 1;
     constexpr bool EXPAND = (MODE & kLmExpand) != 0;
     constexpr bool ACCUM = (MODE & kLmAccum) != 0;
@@ -349,23 +348,30 @@ __global__ void __launch_bounds__(256) k_large(LargePass A) {
     const int64_t m_first = m;
     const int64_t m_last = ACCUM ? lower_bound_f(A.sp, ms, __ldg(A.s + r1 - 1)) : 0;
 
-    // interval sums of the current bin: fp32 for up to 16 rows, then folded into fp64
+    // interval sums of the current bin: fp32 for up to 16 rows, then folded into
+    // fp64 partials kept in shared memory (slot i of thread t at [i][t]: touched
+    // only at folds and flushes, so they cost no registers)
+    constexpr int ND = ACCUM ? 2 * NP * VEC : 1;
+    __shared__ double s_dacc[ND][256];
     int64_t cur = m;
     float fu[NP][VEC], fv[NP][VEC];
-    double du[NP][VEC], dv[NP][VEC];
-    int cnt = 0;
+    int cnt = 0;  // rows in the fp32 partials (wide groups: the same in every lane)
 #pragma unroll
     for (int p = 0; p < NP; ++p)
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) fu[p][v] = fv[p][v] = 0.f, du[p][v] = dv[p][v] = 0.0;
+        for (int v = 0; v < VEC; ++v) fu[p][v] = fv[p][v] = 0.f;
+#pragma unroll
+    for (int i = 0; i < ND; ++i) s_dacc[i][threadIdx.x] = 0.0;
+    auto du = [&](int p, int v) -> double& { return s_dacc[(p * VEC + v) % ND][threadIdx.x]; };
+    auto dv = [&](int p, int v) -> double& { return s_dacc[(NP * VEC + p * VEC + v) % ND][threadIdx.x]; };
 
     auto fold = [&]() {
 #pragma unroll
         for (int p = 0; p < NP; ++p)
 #pragma unroll
             for (int v = 0; v < VEC; ++v) {
-                du[p][v] += (double)fu[p][v];
-                dv[p][v] += (double)fv[p][v];
+                du(p, v) += (double)fu[p][v];
+                dv(p, v) += (double)fv[p][v];
                 fu[p][v] = fv[p][v] = 0.f;
             }
         cnt = 0;
@@ -379,27 +385,32 @@ __global__ void __launch_bounds__(256) k_large(LargePass A) {
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) {
                     const int ch = p * B + c0 + v;
+                    const double su = du(p, v), sv = dv(p, v);
                     if (bin < ms) {
                         double* dst = A.U + bin * Cb + ch;
                         if (owner)
-                            *dst = du[p][v];
-                        else if (du[p][v] != 0.0)
-                            atomicAdd(dst, du[p][v]);
+                            *dst = su;
+                        else if (su != 0.0)
+                            atomicAdd(dst, su);
                     }
                     if (bin >= 1) {
                         double* dst = A.V + (bin - 1) * Cb + ch;
                         if (owner)
-                            *dst = dv[p][v];
-                        else if (dv[p][v] != 0.0)
-                            atomicAdd(dst, dv[p][v]);
+                            *dst = sv;
+                        else if (sv != 0.0)
+                            atomicAdd(dst, sv);
                     }
-                    du[p][v] = dv[p][v] = 0.0;
+                    du(p, v) = 0.0;
+                    dv(p, v) = 0.0;
                 }
         }
     };
 
     int64_t st_m = -1, st_mp = -1;
     float Pm1[NP][VEC], Pmp[NP][VEC], Smp[NP][VEC];
+
+    constexpr int U = kLargeBatch<VEC, PHASED, MODE>;
+    const bool wide = lpr >= U;  // group-uniform, and warp-uniform when wide
 
     // One row: q's bins m (small-side anchors < q) and mp (<= q), the decays eL / eR
     // to the neighbouring small-side anchors, phase weights (w0, w1) = (cos, sin),
@@ -439,7 +450,7 @@ __global__ void __launch_bounds__(256) k_large(LargePass A) {
                         atomicAdd(A.TR + (mpr - 1) * Cb + p * B + c0 + v, val);
                     }
             }
-            if (++cnt == 16) fold();
+            if (wide && ++cnt == 16) fold();  // narrow groups fold on a fixed schedule instead
         }
         if (STATES) {
             if (mr != st_m || mpr != st_mp) {
@@ -495,8 +506,7 @@ __global__ void __launch_bounds__(256) k_large(LargePass A) {
             dst[pr] = v;
     };
 
-    constexpr int U = kLargeBatch<VEC, PHASED, MODE>;
-    if (lpr >= U) {
+    if (wide) {
         // Wide groups.  Rows are taken in batches of lpr: lane gl computes the
         // scalars of row rb + gl (permutation entry, phase weights, bins, decays),
         // so every row's scalar work is done once; the group then walks the batch in
@@ -627,6 +637,9 @@ __global__ void __launch_bounds__(256) k_large(LargePass A) {
                     }
                 }
             }
+            // fp32 interval partials cover at most 16 rows; the schedule is the same
+            // for every group of the warp, so the fold never diverges
+            if (ACCUM && (((rb - r0) / U) & 1)) fold();
         }
     }
     if (ACCUM) flush(cur);

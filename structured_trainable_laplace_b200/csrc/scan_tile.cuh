@@ -211,18 +211,40 @@ __device__ __forceinline__ double2 lookback(Chain ch, int64_t t, int64_t T, cons
             }
             continue;
         }
-        // a slot still unpublished after the bound counts as zero
+        // Every state taken is weighted to the same anchor (the end of the nearest
+        // predecessor), so the carry is a plain sum of independent terms: slot i
+        // adds e_i P_i to P and, to L, e_i P_i when its end lies strictly before
+        // that anchor, else its own strict part L_i.  Lane i computes slot i's
+        // fp64 decay; a slot still unpublished after the bound counts as zero.
         const float uj = exists ? (REV ? -s[jl * R] : s[min(n, (jl + 1) * R) - 1]) : 0.f;
-        for (int i = 0; i <= stop; ++i) {
-            const int fi = __shfl_sync(0xffffffffu, f, i);
-            const float ui = __shfl_sync(0xffffffffu, uj, i);
-            const int64_t ji = REV ? jb + i : jb - i;
-            const bool take = (fi == 1 || fi == 2);
-            if (lane < C && take) {
-                const double2 v = (fi == 1) ? __ldcg(&ch.agg[ji * C + lane]) : __ldcg(&ch.inc[ji * C + lane]);
-                run = have ? lpd_combine(v, ui, run, u_before_tile) : v;
+        const bool brk_me = u_before_tile > uj;
+        const double e_me = brk_me ? exp((double)uj - (double)u_before_tile) : 1.0;
+        // slots are taken 4 at a time: their loads are issued together
+        for (int i0 = 0; i0 <= stop; i0 += 4) {
+            int fk[4];
+            double2 vk[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = (i0 + k) & 31;
+                fk[k] = __shfl_sync(0xffffffffu, f, i);
+                if (i0 + k > stop) fk[k] = 0;
+                const int64_t ji = REV ? jb + i : jb - i;
+                vk[k] = make_double2(0.0, 0.0);
+                if (lane < C && (fk[k] == 1 || fk[k] == 2))
+                    vk[k] = (fk[k] == 1) ? __ldcg(&ch.agg[ji * C + lane]) : __ldcg(&ch.inc[ji * C + lane]);
             }
-            have = have || take;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = (i0 + k) & 31;
+                const double ei = __shfl_sync(0xffffffffu, e_me, i);
+                const bool bi = __shfl_sync(0xffffffffu, brk_me, i);
+                const bool take = (fk[k] == 1 || fk[k] == 2);
+                if (lane < C && take) {
+                    run.y = fma(ei, vk[k].y, run.y);
+                    run.x = bi ? fma(ei, vk[k].y, run.x) : run.x + vk[k].x;
+                }
+                have = have || take;
+            }
         }
         if (incl != 0u || timed_out) break;
         jb = REV ? jb + 32 : jb - 32;
