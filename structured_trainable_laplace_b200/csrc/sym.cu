@@ -330,10 +330,21 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
     // fp64 decays of the tile folds, negative for a tie (decay 1, no break): [0] right
     // fold (-row after the tile -> -its first row), [1] left fold (the tile's last row
     // -> its base range's last row)
+    // Thread 0 computes [0], thread 32 (another warp) [1], in parallel; thread 32
+    // keeps the current range's end anchor and reloads it only when the range changes.
+    int64_t J_ue = -1;
+    float ue_c = 0.f;
     auto tile_ed = [&](const float* sb, int64_t t, double* ed) {
-        const float ue = range_end(t / a.tpr);
-        ed[0] = (sb[4 + R] > sb[4]) ? exp((double)sb[4] - (double)sb[4 + R]) : -1.0;
-        ed[1] = (ue > sb[4 + R - 1]) ? exp((double)sb[4 + R - 1] - (double)ue) : -1.0;
+        if (threadIdx.x == 0) {
+            ed[0] = (sb[4 + R] > sb[4]) ? exp((double)sb[4] - (double)sb[4 + R]) : -1.0;
+        } else if (threadIdx.x == 32) {
+            const int64_t J = t / a.tpr;
+            if (J != J_ue) {
+                J_ue = J;
+                ue_c = range_end(J);
+            }
+            ed[1] = (ue_c > sb[4 + R - 1]) ? exp((double)sb[4 + R - 1] - (double)ue_c) : -1.0;
+        }
     };
     // cp.async groups, in commit order: anchors+permutation of tiles 0 .. MA-1
     // (waited for at once), rows of tiles 0 .. AHEAD-1, then per iteration j the
@@ -356,7 +367,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
         cp_async_commit();
     }
     seg_tables<SK, SG::NT>(sm.s[0], sm.tab[0]);
-    if (threadIdx.x == 0) tile_ed(sm.s[0], tile_of(0), sm.ed[0]);
+    tile_ed(sm.s[0], tile_of(0), sm.ed[0]);
     double2 runR = make_double2(0.0, 0.0), runL = make_double2(0.0, 0.0);
     for (int i = 0; i < nt; ++i) {
         const int64_t t = tile_of(i);
@@ -373,7 +384,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
         cp_async_commit();
         if (i + 1 < nt) {
             seg_tables<SK, SG::NT>(sm.s[(i + 1) % MS], sm.tab[(i + 1) & 1]);
-            if (threadIdx.x == 0) tile_ed(sm.s[(i + 1) % MS], tile_of(i + 1), sm.ed[(i + 1) & 1]);
+            tile_ed(sm.s[(i + 1) % MS], tile_of(i + 1), sm.ed[(i + 1) & 1]);
         }
         const float* sb = sm.s[i % MS];
         const SegTab<SK>& tb = sm.tab[i & 1];
@@ -539,10 +550,21 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
     // fp64 decays of the tile folds, negative for a tie (decay 1, no break):
     // [0] left fold (row before the tile -> its last row), [1] right carry (the row
     // after the base range -> the row after the tile)
+    // Thread 0 computes [0], thread 32 (another warp) [1], in parallel; thread 32
+    // keeps the current range's right anchor and reloads it only when the range changes.
+    int64_t J_ur = -1;
+    float ur_c = 0.f;
     auto tile_ed = [&](const float* sb, int64_t t, double* ed) {
-        const float ur = u_rin(t / a.tpr);
-        ed[0] = (sb[4 + R - 1] > sb[3]) ? exp((double)sb[3] - (double)sb[4 + R - 1]) : -1.0;
-        ed[1] = (-sb[4 + R] > ur) ? exp((double)ur + (double)sb[4 + R]) : -1.0;
+        if (threadIdx.x == 0) {
+            ed[0] = (sb[4 + R - 1] > sb[3]) ? exp((double)sb[3] - (double)sb[4 + R - 1]) : -1.0;
+        } else if (threadIdx.x == 32) {
+            const int64_t J = t / a.tpr;
+            if (J != J_ur) {
+                J_ur = J;
+                ur_c = u_rin(J);
+            }
+            ed[1] = (-sb[4 + R] > ur_c) ? exp((double)ur_c + (double)sb[4 + R]) : -1.0;
+        }
     };
     // everything but the scattered 4-byte ga rows streams through L2 once
     const uint64_t pol_f = l2_evict_first(), pol_l = l2_evict_last();
@@ -572,7 +594,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         cp_async_commit();
     }
     seg_tables<SK, NT>(sm.s[0], sm.tab[0]);
-    if (threadIdx.x == 0) tile_ed(sm.s[0], cw.tb, sm.ed[0]);
+    tile_ed(sm.s[0], cw.tb, sm.ed[0]);
 
     // fp64 left folds of channel c, kept by the channel's first lane (k == 0)
     double2 runL[NV];
@@ -597,7 +619,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
         cp_async_commit();
         if (i + 1 < nt) {
             seg_tables<SK, NT>(sm.s[(i + 1) % MS], sm.tab[(i + 1) & 1]);
-            if (threadIdx.x == 0) tile_ed(sm.s[(i + 1) % MS], t + 1, sm.ed[(i + 1) & 1]);
+            tile_ed(sm.s[(i + 1) % MS], t + 1, sm.ed[(i + 1) & 1]);
         }
         const SegTab<SK>& tb = sm.tab[i & 1];
         const float* dk = tb.d[k];
@@ -704,14 +726,14 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 inR[w] = seg_in(hr_tile, cR[w], k + 1 < SK, exR, evr);
             }
             // pass 2: gx to the output rows, ga to the per-warp sums
-            float gap[E];
+            float gap[E], gxr[E];
             LP ax = inR[0], ag = inR[NV - 1];
 #pragma unroll
             for (int e = E - 1; e >= 0; --e) {
                 const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e + 1];
                 ax = lp_step_x(ax, dv, xe);
                 ag = lp_step_x(ag, dv, ge);
-                ob[e * C] = ag.P - ge;               // gx, right part
+                gxr[e] = ag.P - ge;                  // gx, right part
                 gap[e] = fmaf(ge, ax.L, xe * ag.L);  // strict right sums
             }
             ax = inL[0];
@@ -721,7 +743,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? (NV == 
                 const float xe = xr[0][e], ge = xr[NV - 1][e], dv = dk[e];
                 ax = lp_step_x(ax, dv, xe);
                 ag = lp_step_x(ag, dv, ge);
-                ob[e * C] += ag.P;                            // gx
+                ob[e * C] = gxr[e] + ag.P;                    // gx
                 gap[e] = fmaf(-ge, ax.L, fmaf(-xe, ag.L, gap[e]));  // this channel's share of ga
             }
             // sum over the warp's channels, then one padded row per warp in shared memory
