@@ -251,7 +251,9 @@ struct LargePass {
     int64_t m;
     const float* sp;  // small side, sorted anchors
     int64_t ms;
-    const float* rows;  // [m][B] original order: accumulated (accum) and h (grad)
+    const float* rows;   // [m][Bs] original order: accumulated (accum) and h (grad)
+    const float* rows2;  // nullptr, or the source of channels [Bs, B) ([m][Bs]) of a paired pass
+    int Bs;              // row stride of rows / rows2: B, or B / 2 for a paired pass
     int B;
     int Cb;
     const float* Pst;  // small side states [ms][Cb]
@@ -411,6 +413,12 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
 
     constexpr int U = kLargeBatch<VEC, PHASED, MODE>;
     const bool wide = lpr >= U;  // group-uniform, and warp-uniform when wide
+    // this lane's channels of gathered row pr (a paired pass takes channels past Bs
+    // from the second source; Bs is a multiple of VEC, so no chunk straddles)
+    auto row_src = [&](uint32_t pr) -> const float* {
+        return (A.rows2 != nullptr && c0 >= A.Bs) ? A.rows2 + (int64_t)pr * A.Bs + (c0 - A.Bs)
+                                                  : A.rows + (int64_t)pr * A.Bs + c0;
+    };
 
     // One row: q's bins m (small-side anchors < q) and mp (<= q), the decays eL / eR
     // to the neighbouring small-side anchors, phase weights (w0, w1) = (cos, sin),
@@ -534,7 +542,7 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
                     prv[u] = __shfl_sync(gmask, pr_me, min(j + u, nb - 1), lpr);
 #pragma unroll
                     for (int v = 0; v < VEC; ++v) hv[u][v] = 0.f;
-                    if (ROWS && cval) load_vec<VEC>(A.rows + (int64_t)prv[u] * B + c0, hv[u]);
+                    if (ROWS && cval) load_vec<VEC>(row_src(prv[u]), hv[u]);
                 }
                 float gpart[GRAD ? 2 * U : 1];
 #pragma unroll
@@ -611,7 +619,7 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
                 tv[u] = PHASED ? __ldg(A.theta + pv[u]) : 0.f;
 #pragma unroll
                 for (int v = 0; v < VEC; ++v) hv[u][v] = 0.f;
-                if (ROWS && cval) load_vec<VEC>(A.rows + (int64_t)pv[u] * B + c0, hv[u]);
+                if (ROWS && cval) load_vec<VEC>(row_src(pv[u]), hv[u]);
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -706,22 +714,29 @@ __global__ void __launch_bounds__(256) k_finish(Finish F) {
     }
 }
 
-__global__ void k_scale_rows(const float* __restrict__ D, const float* __restrict__ w, float* __restrict__ out,
-                             int64_t k, int B) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < k * B) out[i] = __ldg(D + i / B) * __ldg(w + i);
-}
-
-__global__ void k_row_dot(const float* __restrict__ a, const float* __restrict__ b, float* __restrict__ out, int64_t k,
-                          int B) {
+// The middle of the Gram apply, one warp per small-side row j: w2 = D_j w_j (the
+// input of the second pass), w_saved = w_j (optional), and gD_j = <wg_j, w_j> when
+// wg is given.  w and wg are rows of ld floats (a paired pass stores them side by
+// side in one [k][2B] array).
+__global__ void __launch_bounds__(256) k_gram_mid(const float* __restrict__ D, const float* __restrict__ w, int ld,
+                                                  const float* __restrict__ wg, float* __restrict__ w2,
+                                                  float* __restrict__ w_saved, float* __restrict__ gD, int64_t k, int B) {
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= k) return;
     const int lane = threadIdx.x & 31;
+    const float d = __ldg(D + r);
     float acc = 0.f;
-    for (int c = lane; c < B; c += 32) acc = fmaf(__ldg(a + r * B + c), __ldg(b + r * B + c), acc);
+    for (int c = lane; c < B; c += 32) {
+        const float wv = __ldg(w + r * ld + c);
+        w2[r * B + c] = d * wv;
+        if (w_saved != nullptr) w_saved[r * B + c] = wv;
+        if (wg != nullptr) acc = fmaf(__ldg(wg + r * ld + c), wv, acc);
+    }
+    if (gD != nullptr) {
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) out[r] = acc;
+        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) gD[r] = acc;
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -857,7 +872,8 @@ cudaError_t large_mode(LargePass A, int mode, int chunks, cudaStream_t st) {
 
 cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
     const bool phased = A.theta != nullptr;
-    const int vec = (A.B % 4 == 0) ? 4 : 1;
+    if (A.Bs == 0) A.Bs = A.B;
+    const int vec = (A.B % 4 == 0 && A.Bs % 4 == 0) ? 4 : 1;
     int lpr = 1;
     while (lpr < 32 && lpr * vec < A.B) lpr <<= 1;
     const int chunks = (A.B + lpr * vec - 1) / (lpr * vec);
@@ -919,6 +935,8 @@ LargePass large_args(Side L, Side Sm, const RectPlan& p, int64_t B) {
     A.sp = Sm.s;
     A.ms = Sm.m;
     A.B = (int)B;
+    A.Bs = (int)B;
+    A.rows2 = nullptr;
     A.Cb = p.Cb;
     const int64_t sz = p.ms * (int64_t)p.Cb;
     A.U = p.bins;
@@ -932,10 +950,14 @@ LargePass large_args(Side L, Side Sm, const RectPlan& p, int64_t B) {
 // Reduce path of the forward: interval sums of x (at I) into O's bins, scan over
 // O, parts written to ZL/ZR/ZF.
 cudaError_t reduce_parts(const RectPlan& p, Side O, Side I, const float* x, int64_t B, float* ZL, float* ZR, float* ZF,
-                         int32_t* status, cudaStream_t st) {
+                         int32_t* status, cudaStream_t st, const float* x2 = nullptr) {
     LAPLEX_TRY(cudaMemsetAsync(p.bins, 0, sizeof(double) * 4 * p.ms * p.Cb, st));
     LargePass A = large_args(I, O, p, B);
     A.rows = x;
+    if (x2 != nullptr) {  // paired pass: channels [0, B/2) from x, [B/2, B) from x2
+        A.rows2 = x2;
+        A.Bs = (int)(B / 2);
+    }
     LAPLEX_TRY(large_pass(A, kLmAccum, st));
     return side_scan(p, bins_scan(O, p, B, ZL, ZR, ZF), true, status, st);
 }
@@ -1084,27 +1106,49 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
     return cudaSuccess;
 }
 
+// Workspace of the Gram apply: the rectangular scratch sized for the paired pass
+// (2B channels), then three [k][B] row buffers.
 size_t gram_workspace_bytes(int64_t n, int64_t k, int64_t B) {
-    return plan_rect(n, k, B, false, nullptr, k).total;
+    return plan_rect(n, k, 2 * B, false, nullptr, k).total;
 }
 
 cudaError_t launch_gram(Side A, Side Bs, const float* D, const float* v, int64_t B, float* y, float* w_saved,
                         const float* g, float* gD, void* ws, int32_t* status, cudaStream_t st) {
-    const RectPlan p = plan_rect(A.m, Bs.m, B, false, ws, Bs.m);
+    const RectPlan p2 = plan_rect(A.m, Bs.m, 2 * B, false, ws, Bs.m);  // layout: rows3 after the paired scratch
     const int64_t kb = Bs.m * B;
-    float* w = w_saved ? w_saved : p.rows3;
-    float* w2 = p.rows3 + kb;
-    float* wg = p.rows3 + 2 * kb;
-    LAPLEX_TRY(launch_rect_forward(Bs, A, v, B, w, nullptr, ws, status, st));  // w = A^T v
-    LAPLEX_TIMED("scale_rows", st, k_scale_rows<<<(unsigned)((kb + 255) / 256), 256, 0, st>>>(D, w, w2, Bs.m, (int)B));
-    LAPLEX_TRY(cudaGetLastError());
-    LAPLEX_TRY(launch_rect_forward(A, Bs, w2, B, y, nullptr, ws, status, st));  // y = A (D w)
-    if (g != nullptr && gD != nullptr) {
-        LAPLEX_TRY(launch_rect_forward(Bs, A, g, B, wg, nullptr, ws, status, st));  // A^T g
-        LAPLEX_TIMED("row_dot", st, k_row_dot<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(wg, w, gD, Bs.m, (int)B));
+    float* wpair = p2.rows3;      // [k][2B]: A^T v | A^T g (paired pass)
+    float* w2 = p2.rows3 + 2 * kb;  // [k][B]: D (A^T v)
+    if (g != nullptr && gD != nullptr && A.m > Bs.m) {
+        // A^T v and A^T g in one reduce pass over the pixel side (2B channels)
+        const RectPlan pp = plan_rect(Bs.m, A.m, 2 * B, false, ws);
+        const int64_t sz = pp.ms * (int64_t)pp.Cb;
+        LAPLEX_TRY(reduce_parts(pp, Bs, A, v, 2 * B, pp.bufA, pp.bufA + sz, pp.bufA + 2 * sz, status, st, g));
+        Finish F{};
+        F.perm = Bs.perm;
+        F.m = Bs.m;
+        F.ZL = pp.bufA;
+        F.ZR = pp.bufA + sz;
+        F.ZF = pp.bufA + 2 * sz;
+        F.B = (int)(2 * B);
+        F.Cb = pp.Cb;
+        F.out = wpair;
+        LAPLEX_TRY(finish(F, st));
+        LAPLEX_TIMED("gram_mid", st,
+                     k_gram_mid<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, wpair, 2 * B, wpair + B, w2, w_saved,
+                                                                           gD, Bs.m, (int)B));
         LAPLEX_TRY(cudaGetLastError());
+        return launch_rect_forward(A, Bs, w2, B, y, nullptr, ws, status, st);  // y = A (D w)
     }
-    return cudaSuccess;
+    float* w = w_saved ? w_saved : wpair;
+    float* wg = wpair + kb;
+    LAPLEX_TRY(launch_rect_forward(Bs, A, v, B, w, nullptr, ws, status, st));  // w = A^T v
+    if (g != nullptr && gD != nullptr)
+        LAPLEX_TRY(launch_rect_forward(Bs, A, g, B, wg, nullptr, ws, status, st));  // A^T g
+    LAPLEX_TIMED("gram_mid", st,
+                 k_gram_mid<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, w, B, (g && gD) ? wg : nullptr, w2,
+                                                                       nullptr, (g && gD) ? gD : nullptr, Bs.m, (int)B));
+    LAPLEX_TRY(cudaGetLastError());
+    return launch_rect_forward(A, Bs, w2, B, y, nullptr, ws, status, st);  // y = A (D w)
 }
 
 }  // namespace laplex

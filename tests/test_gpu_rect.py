@@ -99,10 +99,25 @@ def compare_gram(L, a, b, D, v, g, tag=""):
                  f"gram gD {tag}")
 
 
-@pytest.mark.parametrize("n,k,B", [(5000, 200, 3), (200, 5000, 2), (3000, 3000, 8), (1, 1, 1)])
+@pytest.mark.parametrize("n,k,B", [(5000, 200, 3), (200, 5000, 2), (3000, 3000, 8), (1, 1, 1), (9000, 700, 4),
+                                   (6000, 500, 6), (7001, 64, 16)])
 def test_gram_small(L, n, k, B):
+    # n > k takes the paired reduce pass (A^T v and A^T g together, 2B channels)
     w = inputs.gram(n, k, B, seed=n + k, span=30.0)
     compare_gram(L, w["a"], w["b"], w["D"], w["v"], w["g"], tag=f"n{n} k{k}")
+
+
+@pytest.mark.parametrize("n,k,B", [(5000, 200, 3), (300, 4000, 8)])
+def test_gram_without_gradient(L, n, k, B):
+    w = inputs.gram(n, k, B, seed=n * 3 + k, span=30.0)
+    sa, pa = L.sort_anchors(dev(w["a"]))
+    sb, pb = L.sort_anchors(dev(w["b"]))
+    y, wv = L.gram_apply(sa, pa, sb, pb, dev(w["D"]), dev(w["v"]), return_w=True)
+    L.check()
+    y_ref, w_ref = oracle.gram_apply(w["a"], w["b"], w["D"], w["v"], return_w=True)
+    assert_close(host(y), y_ref, oracle.gram_apply(w["a"], w["b"], w["D"], w["v"], twin=True), "gram y (no g)")
+    assert_close(host(wv), w_ref, oracle.rect_apply(w["a"], w["b"], w["v"], transpose=True, twin=True),
+                 "gram w (no g)")
 
 
 def test_gram_full_size(L):
