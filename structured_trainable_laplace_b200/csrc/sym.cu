@@ -431,6 +431,7 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
 // doubling (log2 NB steps), and each thread then re-walks its block, writing the
 // carry entering every range.
 constexpr int kCarryThreads = 1024;
+constexpr int kCarryBatch = 4;
 
 // Decay between the end anchors of two consecutive ranges, encoded with its break
 // flag: exp(uA - uB) when uB > uA, -1 for a tie (decay 1, no break).
@@ -466,13 +467,25 @@ __global__ void __launch_bounds__(kCarryThreads) k_sym_carry(SymScan a, RangeSta
     const bool mine = q < NB;  // blocks q >= NB are empty
     __syncthreads();
 
-    // block aggregates (left: ranges j0 .. j1-1 in order; right: j1-1 .. j0)
+    // block aggregates (left: ranges j0 .. j1-1 in order; right: j1-1 .. j0); the
+    // aggregates are loaded kCarryBatch at a time, ahead of the dependent folds
     if (mine) {
-        double2 fl = Lagg[(int64_t)j0 * C], fr = Ragg[(int64_t)(j1 - 1) * C];
-        for (int u = 1; u < j1 - j0; ++u) {
-            const int jl = j0 + u, jr = j1 - 1 - u;
-            fl = fold_d(fl, Lagg[(int64_t)jl * C], dL[jl]);
-            fr = fold_d(fr, Ragg[(int64_t)jr * C], dR[jr]);
+        double2 fl = make_double2(0.0, 0.0), fr = make_double2(0.0, 0.0);
+        for (int ub = 0; ub < j1 - j0; ub += kCarryBatch) {
+            double2 vl[kCarryBatch], vr[kCarryBatch];
+#pragma unroll
+            for (int u = 0; u < kCarryBatch; ++u) {
+                const int uu = min(ub + u, j1 - j0 - 1);
+                vl[u] = Lagg[(int64_t)(j0 + uu) * C];
+                vr[u] = Ragg[(int64_t)(j1 - 1 - uu) * C];
+            }
+#pragma unroll
+            for (int u = 0; u < kCarryBatch; ++u) {
+                const int uu = ub + u;
+                if (uu >= j1 - j0) break;
+                fl = uu ? fold_d(fl, vl[u], dL[j0 + uu]) : vl[u];
+                fr = uu ? fold_d(fr, vr[u], dR[j1 - 1 - uu]) : vr[u];
+            }
         }
         sL[q][c] = fl;
         sR[q][c] = fr;
@@ -498,13 +511,24 @@ __global__ void __launch_bounds__(kCarryThreads) k_sym_carry(SymScan a, RangeSta
     const bool hl = q >= 1, hr = q + 1 < NB;
     double2 cl = hl ? sL[q - 1][c] : make_double2(0.0, 0.0);
     double2 cr = hr ? sR[q + 1][c] : make_double2(0.0, 0.0);
-    for (int u = 0; u < j1 - j0; ++u) {
-        const int jl = j0 + u, jr = j1 - 1 - u;
-        Lin[(int64_t)jl * C] = cl;  // zero (unused) for the first range
-        Rin[(int64_t)jr * C] = cr;  // zero (unused) for the last range
-        const double2 vl = Lagg[(int64_t)jl * C], vr = Ragg[(int64_t)jr * C];
-        cl = (hl || u > 0) ? fold_d(cl, vl, dL[jl]) : vl;
-        cr = (hr || u > 0) ? fold_d(cr, vr, dR[jr]) : vr;
+    for (int ub = 0; ub < j1 - j0; ub += kCarryBatch) {
+        double2 vl[kCarryBatch], vr[kCarryBatch];
+#pragma unroll
+        for (int u = 0; u < kCarryBatch; ++u) {
+            const int uu = min(ub + u, j1 - j0 - 1);
+            vl[u] = Lagg[(int64_t)(j0 + uu) * C];
+            vr[u] = Ragg[(int64_t)(j1 - 1 - uu) * C];
+        }
+#pragma unroll
+        for (int u = 0; u < kCarryBatch; ++u) {
+            const int uu = ub + u;
+            if (uu >= j1 - j0) break;
+            const int jl = j0 + uu, jr = j1 - 1 - uu;
+            Lin[(int64_t)jl * C] = cl;  // zero (unused) for the first range
+            Rin[(int64_t)jr * C] = cr;  // zero (unused) for the last range
+            cl = (hl || uu > 0) ? fold_d(cl, vl[u], dL[jl]) : vl[u];
+            cr = (hr || uu > 0) ? fold_d(cr, vr[u], dR[jr]) : vr[u];
+        }
     }
 }
 
