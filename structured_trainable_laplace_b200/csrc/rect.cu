@@ -29,7 +29,7 @@
 //   k_finish  per small-side row: combine the cos/sin parts into outputs and
 //       gradients.
 #include "laplex_internal.h"
-#include "scan_tile.cuh"
+#include "pipeline.cuh"
 
 namespace laplex {
 
@@ -354,7 +354,11 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
     // fp64 partials kept in shared memory (slot i of thread t at [i][t]: touched
     // only at folds and flushes, so they cost no registers)
     constexpr int ND = ACCUM ? 2 * NP * VEC : 1;
-    __shared__ double s_dacc[ND][256];
+    // dynamic shared memory: the fp64 partials [ND][256], then (wide groups in
+    // modes that gather rows) the per-warp ring of two sub-batch slots
+    extern __shared__ __align__(16) unsigned char large_smem[];
+    double(*s_dacc)[256] = reinterpret_cast<double(*)[256]>(large_smem);
+    float* s_rows = reinterpret_cast<float*>(large_smem + sizeof(double) * ND * 256);
     int64_t cur = m;
     float fu[NP][VEC], fv[NP][VEC];
     int cnt = 0;  // rows in the fp32 partials (wide groups: the same in every lane)
@@ -518,32 +522,73 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
         // Wide groups.  Rows are taken in batches of lpr: lane gl computes the
         // scalars of row rb + gl (permutation entry, phase weights, bins, decays),
         // so every row's scalar work is done once; the group then walks the batch in
-        // sub-batches of U rows whose gathered rows are loaded together, taking each
-        // row's scalars from the lane that computed them.  Bins are below 2^32.
-        for (int64_t rb = r0; rb < r1; rb += lpr) {
-            const int nb = (int)min((int64_t)lpr, r1 - rb);
+        // sub-batches of U rows, taking each row's scalars from the lane that
+        // computed them.  Bins are below 2^32.  The gathered rows go through a
+        // per-warp ring of two sub-batch slots in shared memory: each lane copies
+        // its own VEC floats of the next sub-batch's rows with cp.async while the
+        // current one is processed (and reads back only what it copied, so no
+        // warp barrier is needed).  The next batch's scalars are computed one
+        // sub-batch early, from the bins reached so far (a lower bound).
+        struct Scal {
+            uint32_t pr, mm, mmp;
+            float cs, sn, eL, eR;
+        };
+        auto batch_scalars = [&](int64_t rb, int nb, Scal& S) {
             const int64_t rme = rb + min(gl, nb - 1);
             const float q_me = __ldg(A.s + rme);
-            const uint32_t pr_me = min(__ldg(A.perm + rme), (uint32_t)(A.m - 1));
-            float cs_me = 1.f, sn_me = 0.f;
-            if (PHASED) sincosf(__ldg(A.theta + pr_me), &sn_me, &cs_me);
+            S.pr = min(__ldg(A.perm + rme), (uint32_t)(A.m - 1));
+            S.cs = 1.f;
+            S.sn = 0.f;
+            if (PHASED) sincosf(__ldg(A.theta + S.pr), &S.sn, &S.cs);
             int64_t mm = m;
             while (mm < ms && __ldg(A.sp + mm) < q_me) ++mm;
             int64_t mmp = max(mp, mm);
             while (mmp < ms && __ldg(A.sp + mmp) <= q_me) ++mmp;
-            const float eL_me = (mm > 0) ? expf(__ldg(A.sp + mm - 1) - q_me) : 0.f;
-            const float eR_me = (mmp < ms) ? expf(q_me - __ldg(A.sp + mmp)) : 0.f;
-            const uint32_t mm32 = (uint32_t)mm, mmp32 = (uint32_t)mmp;
-            for (int j = 0; j < nb; j += U) {
-                uint32_t prv[U];
-                float hv[U][VEC];
+            S.eL = (mm > 0) ? expf(__ldg(A.sp + mm - 1) - q_me) : 0.f;
+            S.eR = (mmp < ms) ? expf(q_me - __ldg(A.sp + mmp)) : 0.f;
+            S.mm = (uint32_t)mm;
+            S.mmp = (uint32_t)mmp;
+        };
+        float* ring = s_rows + (threadIdx.x >> 5) * (2 * U * 32 * VEC) + lane * VEC;  // this lane's slots
+        auto stage = [&](const Scal& S, int j, int nb, int slot) {
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    prv[u] = __shfl_sync(gmask, pr_me, min(j + u, nb - 1), lpr);
-#pragma unroll
-                    for (int v = 0; v < VEC; ++v) hv[u][v] = 0.f;
-                    if (ROWS && cval) load_vec<VEC>(row_src(prv[u]), hv[u]);
+            for (int u = 0; u < U; ++u) {
+                const uint32_t pr = __shfl_sync(gmask, S.pr, min(j + u, nb - 1), lpr);
+                if (ROWS && cval) {
+                    float* dst = ring + (slot * U + u) * (32 * VEC);
+                    if constexpr (VEC == 4)
+                        cp_async16(dst, row_src(pr));
+                    else
+                        cp_async4(dst, row_src(pr));
                 }
+            }
+            cp_async_commit();
+        };
+        Scal S;
+        int slot = 0;
+        batch_scalars(r0, (int)min((int64_t)lpr, r1 - r0), S);
+        stage(S, 0, (int)min((int64_t)lpr, r1 - r0), 0);
+        for (int64_t rb = r0; rb < r1; rb += lpr) {
+            const int nb = (int)min((int64_t)lpr, r1 - rb);
+            Scal Sn = S;
+            for (int j = 0; j < nb; j += U) {
+                if (j + U < nb) {
+                    stage(S, j + U, nb, slot ^ 1);
+                } else if (rb + lpr < r1) {
+                    const int nbn = (int)min((int64_t)lpr, r1 - rb - lpr);
+                    batch_scalars(rb + lpr, nbn, Sn);
+                    stage(Sn, 0, nbn, slot ^ 1);
+                } else {
+                    cp_async_commit();  // keep one group per sub-batch
+                }
+                cp_async_wait<1>();  // this sub-batch's copies are in
+                // the rows are read from the ring inside the row body (lanes past B
+                // read zeros)
+                const float zeros[VEC] = {};
+                const float* hrow0 = (ROWS && cval) ? ring + slot * U * (32 * VEC) : zeros;
+                const int hstep = (ROWS && cval) ? 32 * VEC : 0;
+                const float cs_me = S.cs, sn_me = S.sn, eL_me = S.eL, eR_me = S.eR;
+                const uint32_t mm32 = S.mm, mmp32 = S.mmp;
                 float gpart[GRAD ? 2 * U : 1];
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
@@ -555,7 +600,8 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
                     m = __shfl_sync(gmask, mm32, src, lpr);
                     mp = __shfl_sync(gmask, mmp32, src, lpr);
                     float ga = 0.f, gp = 0.f;
-                    if (j + u < nb) row(prv[u], w0, w1, eL, eR, m, mp, hv[u], ga, gp);  // group-uniform
+                    const uint32_t pru = __shfl_sync(gmask, S.pr, src, lpr);
+                    if (j + u < nb) row(pru, w0, w1, eL, eR, m, mp, hrow0 + u * hstep, ga, gp);  // group-uniform
                     if (GRAD) {
                         gpart[u] = ga;
                         gpart[U + u] = gp;
@@ -592,13 +638,16 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
                     for (int i = 0; i < NV; ++i) {
                         if (i >= vc) break;
                         const int idx = base + i, u = idx % U;
-                        const uint32_t pr = __shfl_sync(gmask, pr_me, min(j + u, nb - 1), lpr);
+                        const uint32_t pr = __shfl_sync(gmask, S.pr, min(j + u, nb - 1), lpr);
                         if (writer && j + u < nb) put_grad(idx < U ? A.g_anchor : (PHASED ? A.g_phase : nullptr), pr,
                                                           gpart[i]);
                     }
                 }
+                slot ^= 1;
             }
+            S = Sn;
         }
+        cp_async_wait_all();
     } else {
         // Narrow groups: the group walks its rows in batches of U, loading the
         // batch's anchors and permutation entries, then its phases and gathered rows
@@ -837,22 +886,44 @@ cudaError_t side_scan(const RectPlan& p, SideScan a, bool bins, int32_t* status,
 // group walking an equal contiguous run of rows, at least kLargeMinRows of them.
 constexpr int64_t kLargeMinRows = 64;
 
+// One warp as tile 1 of a two-tile chain whose tile 0 never publishes: the
+// lookback must give up after its bound and record the timeout.
+__global__ void k_check_wait_bound(Chain ch, const float* s, int32_t* status) {
+    bool has = false;
+    (void)lookback<1, false>(ch, 1, 2, s, 2, 1, LP{1.f, 1.f}, s[1], s[0], status, has);
+}
+
+// Dynamic shared memory of k_large<VEC, PHASED, MODE>: the fp64 partials, plus the
+// staging ring when the groups are wide and the mode gathers rows.
+template <int VEC, bool PHASED, int MODE>
+size_t large_smem_bytes(bool wide) {
+    constexpr int NP = PHASED ? 2 : 1;
+    constexpr int ND = (MODE & kLmAccum) ? 2 * NP * VEC : 1;
+    constexpr bool ROWS = (MODE & (kLmAccum | kLmGrad)) != 0;
+    const size_t ring = (wide && ROWS) ? sizeof(float) * 8 * 2 * kLargeBatch<VEC, PHASED, MODE> * 32 * VEC : 0;
+    return sizeof(double) * ND * 256 + ring;
+}
+
 template <int VEC, bool PHASED, int MODE>
 cudaError_t launch_large(LargePass A, int chunks, const char* name, cudaStream_t st) {
-    static int occ = 0;
-    if (occ == 0) {
+    const bool wide = A.lpr >= kLargeBatch<VEC, PHASED, MODE>;
+    const size_t smem = large_smem_bytes<VEC, PHASED, MODE>(wide);
+    static int occ[2] = {0, 0};
+    if (occ[wide] == 0) {
         int o = 1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large<VEC, PHASED, MODE>, 256, 0) != cudaSuccess)
+        cudaFuncSetAttribute(k_large<VEC, PHASED, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)large_smem_bytes<VEC, PHASED, MODE>(true));
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large<VEC, PHASED, MODE>, 256, smem) != cudaSuccess)
             o = 1;
-        occ = std::max(o, 1);
+        occ[wide] = std::max(o, 1);
     }
     const int64_t groups_per_block = 8 * (32 / A.lpr);
-    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ / chunks);
+    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ[wide] / chunks);
     const int64_t need = (A.m + groups_per_block * kLargeMinRows - 1) / (groups_per_block * kLargeMinRows);
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
     A.rows_per_group = (A.m + blocks * groups_per_block - 1) / (blocks * groups_per_block);
     const dim3 grid((unsigned)blocks, (unsigned)chunks);
-    LAPLEX_TIMED(name, st, k_large<VEC, PHASED, MODE><<<grid, 256, 0, st>>>(A));
+    LAPLEX_TIMED(name, st, k_large<VEC, PHASED, MODE><<<grid, 256, smem, st>>>(A));
     return cudaGetLastError();
 }
 
@@ -1108,6 +1179,16 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
 
 // Workspace of the Gram apply: the rectangular scratch sized for the paired pass
 // (2B channels), then three [k][B] row buffers.
+cudaError_t launch_check_wait_bound(void* ws, int32_t* status, cudaStream_t st) {
+    // ws: flags [2] | agg [2] | inc [2] | anchors [2]
+    char* b = (char*)ws;
+    LAPLEX_TRY(cudaMemsetAsync(b, 0, 256, st));
+    Chain ch{(int*)b, (double2*)(b + 64), (double2*)(b + 128)};
+    const float* s = (const float*)(b + 192);  // anchors 0, 0 (zeroed)
+    LAPLEX_TIMED("check_wait_bound", st, k_check_wait_bound<<<1, 32, 0, st>>>(ch, s, status));
+    return cudaGetLastError();
+}
+
 size_t gram_workspace_bytes(int64_t n, int64_t k, int64_t B) {
     return plan_rect(n, k, 2 * B, false, nullptr, k).total;
 }
