@@ -205,6 +205,22 @@ laplex_status laplex_gram_apply(const float* a_sorted, const uint32_t* perm_a, i
                                 float* y, float* w_saved, const float* g, float* gD, void* ws, size_t ws_bytes,
                                 int32_t* d_status, laplex_stream_t stream);
 
+/* -------------------------------------------------------- diagnostics */
+
+/* Bytes of device workspace laplex_check_wait_bound needs. */
+#define LAPLEX_CHECK_WAIT_WS_BYTES 1024
+
+/* Failure-detection self-check (no counterpart on the pages).  Runs one warp of the
+ * small-side scan's lookback against a predecessor whose status flag nothing ever
+ * sets: the bounded wait must give up (after about 2^20 polls, well under a second
+ * on a B200), write LAPLEX_ERR_TIMEOUT to *d_status and let the kernel finish, so
+ * the context stays usable.  ws: at least LAPLEX_CHECK_WAIT_WS_BYTES of device
+ * memory (overwritten); d_status: required, zeroed by the caller.  Returns
+ * LAPLEX_ERR_ARG / LAPLEX_ERR_ALIGN / LAPLEX_ERR_WORKSPACE for bad arguments,
+ * LAPLEX_ERR_CUDA if the launch fails, else LAPLEX_OK (read the outcome with
+ * laplex_read_status). */
+laplex_status laplex_check_wait_bound(void* ws, size_t ws_bytes, int32_t* d_status, laplex_stream_t stream);
+
 /* ------------------------------------------------------------- tracing */
 
 /* Per-kernel timing aid (no counterpart on the pages; a measurement tool).

@@ -113,6 +113,14 @@ laplex_status laplex_read_status(const int32_t* d_status, laplex_stream_t stream
     return (laplex_status)*h_status;
 }
 
+laplex_status laplex_check_wait_bound(void* ws, size_t ws_bytes, int32_t* d_status, laplex_stream_t stream) {
+    if (!ws || !d_status) return LAPLEX_ERR_ARG;
+    if (ws_bytes < LAPLEX_CHECK_WAIT_WS_BYTES) return LAPLEX_ERR_WORKSPACE;
+    laplex_status s = check_ranges({}, {{ws, ws_bytes}, {d_status, 4}});
+    if (s != LAPLEX_OK) return s;
+    return cuda_status(launch_check_wait_bound(ws, d_status, (cudaStream_t)stream));
+}
+
 size_t laplex_sort_workspace_size(int64_t n) { return size_ok(n) ? sort_workspace_bytes(n) : 0; }
 
 laplex_status laplex_sort_anchors(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws,

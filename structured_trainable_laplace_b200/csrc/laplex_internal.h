@@ -70,6 +70,10 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
                                  float* gx, float* gO, float* gI, float* gtO, float* gtI, void* ws, int32_t* status,
                                  cudaStream_t stream);
 
+// The bounded lookback against a predecessor that never publishes (failure-
+// detection self-check): ws holds the chain, zeroed here.
+cudaError_t launch_check_wait_bound(void* ws, int32_t* status, cudaStream_t stream);
+
 size_t gram_workspace_bytes(int64_t n, int64_t k, int64_t B);
 cudaError_t launch_gram(Side A, Side Bs, const float* D, const float* v, int64_t B, float* y, float* w_saved,
                         const float* g, float* gD, void* ws, int32_t* status, cudaStream_t stream);

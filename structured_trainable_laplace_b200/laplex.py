@@ -59,6 +59,7 @@ def lib():
             "laplex_apply_phased": ([P, P, I64, P, P, P, I64, P, I, P, I64, P, P, P, SZ, P, P], I),
             "laplex_backward": ([I, P, P, I64, P, P, P, I64, P, P, P, I64, P, P, P, P, P, P, P, SZ, P, P], I),
             "laplex_gram_apply": ([P, P, I64, P, P, I64, P, P, I64, P, P, P, P, P, SZ, P, P], I),
+            "laplex_check_wait_bound": ([P, SZ, P, P], I),
             "laplex_profile_enable": ([I], None),
             "laplex_profile_report": ([I, P, I, P, P], I),
         }
@@ -76,7 +77,7 @@ def exported_symbols() -> list:
             "laplex_workspace_size", "laplex_saved_size", "laplex_apply_sym", "laplex_apply_sym_noalloc",
             "laplex_apply_general",
             "laplex_apply_transpose", "laplex_apply_phased", "laplex_backward", "laplex_gram_apply",
-            "laplex_profile_enable", "laplex_profile_report"]
+            "laplex_check_wait_bound", "laplex_profile_enable", "laplex_profile_report"]
 
 
 # ---------------------------------------------------------------- plumbing
@@ -299,6 +300,21 @@ def gram_apply(a_sorted, perm_a, b_sorted, perm_b, D, v, g=None, return_w=False)
     if g is not None:
         res += (gD,)
     return res[0] if len(res) == 1 else res
+
+
+# ---------------------------------------------------------------- diagnostics
+
+def check_wait_bound(device: int | None = None) -> int:
+    """Run the failure-detection self-check (a bounded lookback wait on a flag that
+    nothing sets) on its own status word and return the status it recorded (5 =
+    the wait gave up, as it must)."""
+    device = torch.cuda.current_device() if device is None else device
+    ws = torch.empty(1024, dtype=torch.uint8, device=f"cuda:{device}")
+    st = torch.zeros(1, dtype=torch.int32, device=f"cuda:{device}")
+    _ok(lib().laplex_check_wait_bound(_p(ws), ws.numel(), _p(st), _stream(device)), "check_wait_bound")
+    h = ctypes.c_int32(0)
+    lib().laplex_read_status(ctypes.c_void_p(st.data_ptr()), _stream(device), ctypes.byref(h))
+    return int(h.value)
 
 
 # ---------------------------------------------------------------- tracing
