@@ -554,12 +554,17 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const uint32_t pr = __shfl_sync(gmask, S.pr, min(j + u, nb - 1), lpr);
-                if (ROWS && cval) {
+                if (ROWS) {
                     float* dst = ring + (slot * U + u) * (32 * VEC);
-                    if constexpr (VEC == 4)
-                        cp_async16(dst, row_src(pr));
-                    else
-                        cp_async4(dst, row_src(pr));
+                    if (cval) {
+                        if constexpr (VEC == 4)
+                            cp_async16(dst, row_src(pr));
+                        else
+                            cp_async4(dst, row_src(pr));
+                    } else {
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) dst[v] = 0.f;  // channels past B read as zero
+                    }
                 }
             }
             cp_async_commit();
@@ -582,11 +587,9 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
                     cp_async_commit();  // keep one group per sub-batch
                 }
                 cp_async_wait<1>();  // this sub-batch's copies are in
-                // the rows are read from the ring inside the row body (lanes past B
-                // read zeros)
-                const float zeros[VEC] = {};
-                const float* hrow0 = (ROWS && cval) ? ring + slot * U * (32 * VEC) : zeros;
-                const int hstep = (ROWS && cval) ? 32 * VEC : 0;
+                // the rows are read from the ring inside the row body
+                const float* hrow0 = ring + slot * U * (32 * VEC);
+                constexpr int hstep = 32 * VEC;
                 const float cs_me = S.cs, sn_me = S.sn, eL_me = S.eL, eR_me = S.eR;
                 const uint32_t mm32 = S.mm, mmp32 = S.mmp;
                 float gpart[GRAD ? 2 * U : 1];
