@@ -45,7 +45,7 @@ namespace {
 constexpr int kE = 16;
 constexpr int kMaxRanges = 8192;   // base ranges per channel group
 constexpr int kRangesPerSM = 6;    // base ranges per SM (divisible by the usual occupancies)
-constexpr int kAheadAgg = 3;       // prefetch distance of the gathered rows (aggregate pass)
+constexpr int kAheadAgg = 2;       // prefetch distance of the gathered rows (aggregate pass)
 constexpr int kAheadFwd = 1;       // of the streamed sorted tiles: forward sweep
 constexpr int kAheadBwd = 1;       // backward sweep (two streamed vectors)
 
@@ -308,7 +308,7 @@ __device__ __forceinline__ CtaTiles cta_tiles(const SymScan& a) {
 // aggregate; both restart at each base range's last tile and are written out at
 // its first.
 template <int C, int AHEAD>
-__global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 2 : 1))
+__global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
     k_sym_agg(SymScan a, const float* __restrict__ v, RangeState st, float* __restrict__ vs) {
     using SG = SymGeo<C>;
     using G = typename SG::G;
