@@ -177,6 +177,27 @@ def gram_backward_D(a, b, v, g, twin=False):
     return gD
 
 
+def gram_backward(a, b, D, v, g, twin=False):
+    """Every gradient of <g, A diag(D) A^T v>, from the C scans: with w = A^T v and
+    u = A^T g (transposed products), gv = A (D u) (a general product), gD = sum_c u w,
+    and ga, gb the anchor gradients of the two general products A (D w) read by g
+    and A (D u) read by v (dl/dA_ij = D_j sum_c (g_ic w_jc + v_ic u_jc)).
+    Returns dict gv, ga, gb, gD (fp64).  ``twin=True`` composes the companions."""
+    D = _f32(D).astype(np.float64)
+    w = rect_apply(a, b, v, transpose=True, twin=twin)
+    u = rect_apply(a, b, g, transpose=True, twin=twin)
+    Dm = np.abs(D) if twin else D
+    x1, x2 = Dm[:, None] * w, Dm[:, None] * u
+    r1 = rect_backward(a, b, x1, g, twin=twin)
+    r2 = rect_backward(a, b, x2, v, twin=twin)
+    return {
+        "gv": rect_apply(a, b, x2, twin=twin),
+        "ga": r1["ga"] + r2["ga"],
+        "gb": r1["gb"] + r2["gb"],
+        "gD": (u * w).sum(axis=1),
+    }
+
+
 def sym_sampled(a, x, samples, g=None, window=100.0):
     """Windowed direct evaluation of the symmetric operator at sample indices.
     Returns dict y, y_twin [m][B], dropped [B] (and ga, ga_twin [m] if g given)."""

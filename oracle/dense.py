@@ -167,3 +167,30 @@ def gram_backward_D(a, b, v, g):
     v, g = _rows(v), _rows(g)
     A = kernel(a, b)
     return ((A.T @ g) * (A.T @ v)).sum(axis=1)
+
+
+def gram_backward(a, b, D, v, g, twin=False):
+    """Every gradient of l = <g, A diag(D) A^T v> (A_ij = exp(-|a_i - b_j|)), entry by
+    entry.  With w = A^T v and u = A^T g, l = sum_jc D_j u_jc w_jc, and
+    dl/dA_ij = D_j M_ij with M_ij = sum_c (g_ic w_jc + v_ic u_jc); with the entry
+    derivatives of the module docstring:
+      gv = A (D u) (the operator is symmetric),  gD_j = sum_c u_jc w_jc,
+      ga_i = sum_j -S_ij A_ij D_j M_ij,  gb_j = sum_i S_ij A_ij D_j M_ij.
+    ``twin=True``: every factor (and w, u) replaced by its magnitude companion."""
+    v, g = _rows(v), _rows(g)
+    A = kernel(a, b)
+    S = sign_matrix(a, b)
+    Dv = _f64(D)
+    sg = 1.0
+    if twin:
+        v, g, S, Dv, sg = np.abs(v), np.abs(g), np.abs(S), np.abs(Dv), -1.0
+    w, u = A.T @ v, A.T @ g
+    M = g @ w.T + v @ u.T
+    W = A * Dv[None, :] * M
+    return {
+        "gv": A @ (Dv[:, None] * u),
+        "ga": (sg * -S * W).sum(axis=1),
+        "gb": (S * W).sum(axis=0),
+        "gD": (u * w).sum(axis=1),
+    }
+

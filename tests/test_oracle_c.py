@@ -86,6 +86,23 @@ def test_gram_matches_dense():
     assert rel(oracle.gram_backward_D(a, b, v, g), dense.gram_backward_D(a, b, v, g)) < 1e-13
 
 
+def test_gram_full_backward_matches_dense():
+    """The composed C evaluation of every Gram gradient against the dense
+    definition, with ties inside a, inside b and between them.  The composition
+    rounds A^T v and A^T g to fp32 between its passes (relative 6e-8)."""
+    rng = np.random.default_rng(22)
+    a, b = tied(rng, 50, 0.25, 30), tied(rng, 11, 0.25, 30)
+    D = rng.uniform(0.1, 2, 11).astype(np.float32)
+    v, g = rng.standard_normal((50, 2)).astype(np.float32), rng.standard_normal((50, 2)).astype(np.float32)
+    got, ref = oracle.gram_backward(a, b, D, v, g), dense.gram_backward(a, b, D, v, g)
+    tw = dense.gram_backward(a, b, D, v, g, twin=True)
+    for key in ("gv", "ga", "gb", "gD"):
+        assert np.all(np.abs(got[key] - ref[key]) <= 1e-6 * tw[key] + 1e-12), key
+    got_tw = oracle.gram_backward(a, b, D, v, g, twin=True)
+    for key in ("gv", "ga", "gb", "gD"):
+        assert np.all(got_tw[key] >= np.abs(ref[key]) * (1 - 1e-6) - 1e-12), key
+
+
 def test_sort_matches_numpy_stable_argsort():
     rng = np.random.default_rng(21)
     a = tied(rng, 5000, 0.125, 64)

@@ -170,6 +170,50 @@ def test_gram_D_gradient_matches_finite_differences():
     np.testing.assert_allclose(gD, fd_grad(lambda t: np.sum(g * dense.gram_apply(a, b, t, v)), D), rtol=1e-7)
 
 
+def test_gram_full_backward_matches_finite_differences():
+    """gv, ga, gb and gD of <g, A diag(D) A^T v> against central differences of the
+    dense forward (anchors kept 1e-3 apart, so no |a_i - b_j| crosses zero)."""
+    rng = np.random.default_rng(15)
+    n, k, B = 14, 6, 2
+    a, b = separated(rng, n, 0, 6, 1e-3), separated(rng, k, 0.01, 6.01, 1e-3)
+    while np.min(np.abs(a[:, None] - b[None, :])) < 1e-3:
+        b = separated(rng, k, 0.01, 6.01, 1e-3)
+    D = rng.uniform(0.1, 2, k)
+    v, g = rng.standard_normal((n, B)), rng.standard_normal((n, B))
+    gr = dense.gram_backward(a, b, D, v, g)
+
+    def loss(a_=a, b_=b, D_=D, v_=v):
+        return np.sum(g * dense.gram_apply(a_, b_, D_, v_))
+
+    np.testing.assert_allclose(gr["ga"], fd_grad(lambda t: loss(a_=t), a), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(gr["gb"], fd_grad(lambda t: loss(b_=t), b), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(gr["gD"], fd_grad(lambda t: loss(D_=t), D), rtol=1e-7, atol=1e-9)
+    np.testing.assert_allclose(gr["gv"], fd_grad(lambda t: loss(v_=t.reshape(v.shape)), v.reshape(-1)).reshape(v.shape),
+                               rtol=1e-7, atol=1e-9)
+    # the operator is symmetric, so gv is the operator applied to g
+    np.testing.assert_allclose(gr["gv"], dense.gram_apply(a, b, D, g), rtol=1e-12)
+    # shifting every anchor leaves the loss unchanged (ties included): sum ga + sum gb = 0
+    assert abs(gr["ga"].sum() + gr["gb"].sum()) < 1e-10 * (np.abs(gr["ga"]).sum() + np.abs(gr["gb"]).sum())
+
+
+def test_planted_gram_gradient_mistake_fails_the_fd_pin():
+    """A gradient that forgets the dependence of w = A^T v on the anchors (keeping
+    only the outer A) is caught by the finite-difference pin."""
+    rng = np.random.default_rng(16)
+    n, k = 12, 5
+    a, b = separated(rng, n, 0, 5, 1e-3), separated(rng, k, 0.01, 5.01, 1e-3)
+    while np.min(np.abs(a[:, None] - b[None, :])) < 1e-3:
+        b = separated(rng, k, 0.01, 5.01, 1e-3)
+    D = rng.uniform(0.1, 2, k)
+    v, g = rng.standard_normal((n, 1)), rng.standard_normal((n, 1))
+    A, S = dense.kernel(a, b), dense.sign_matrix(a, b)
+    w = A.T @ v
+    wrong_ga = (-S * A * D[None, :] * (g @ w.T)).sum(axis=1)  # the v u^T term dropped
+    fd = fd_grad(lambda t: np.sum(g * dense.gram_apply(t, b, D, v)), a)
+    assert not np.allclose(wrong_ga, fd, rtol=1e-4, atol=1e-6)
+    np.testing.assert_allclose(dense.gram_backward(a, b, D, v, g)["ga"], fd, rtol=1e-6, atol=1e-8)
+
+
 def test_gram_is_positive_semidefinite_and_symmetric():
     rng = np.random.default_rng(13)
     a, b = rng.uniform(0, 8, 40), rng.uniform(0, 8, 7)
