@@ -205,6 +205,23 @@ laplex_status laplex_gram_apply(const float* a_sorted, const uint32_t* perm_a, i
                                 float* y, float* w_saved, const float* g, float* gD, void* ws, size_t ws_bytes,
                                 int32_t* d_status, laplex_stream_t stream);
 
+/* Every gradient of the Gram apply (section 2.2, "Gram operators"; the covariance
+ * factor is trainable, abstract and section 4.2): for l = <g, A diag(D) A^T v>,
+ * A_ij = exp(-|a_i - b_j|), with w = A^T v and u = A^T g,
+ *   gv [n][B] = A diag(D) A^T g                 (the operator is symmetric),
+ *   ga [n]    = sum_c g_ic (R - L)[D w]_ic + v_ic (R - L)[D u]_ic,
+ *   gb [k]    = D_j sum_c w_jc (R' - L')[g]_jc + u_jc (R' - L')[v]_jc,
+ *   gD [k]    = sum_c u_jc w_jc,
+ * where (R - L)[z]_i is the sum over the b anchors strictly right of a_i minus the
+ * sum over those strictly left, each weighted exp(-|a_i - b_j|) (sign(0) = 0), and
+ * (R' - L')[h]_j the same over the a anchors relative to b_j.  Any output may be
+ * NULL to skip it (at least one must be set); v, g [n][B] in original order.
+ * Workspace: laplex_workspace_size(LAPLEX_OP_GRAM, n, k, B). */
+laplex_status laplex_gram_backward(const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* b_sorted,
+                                   const uint32_t* perm_b, int64_t k, const float* D, const float* v, const float* g,
+                                   int64_t B, float* gv, float* ga, float* gb, float* gD, void* ws, size_t ws_bytes,
+                                   int32_t* d_status, laplex_stream_t stream);
+
 /* -------------------------------------------------------- diagnostics */
 
 /* Bytes of device workspace laplex_check_wait_bound needs. */

@@ -257,4 +257,23 @@ laplex_status laplex_gram_apply(const float* a_sorted, const uint32_t* perm_a, i
     return cuda_status(launch_gram(A, Bs, D, v, B, y, w_saved, g, gD, ws, d_status, (cudaStream_t)stream));
 }
 
+
+laplex_status laplex_gram_backward(const float* a_sorted, const uint32_t* perm_a, int64_t n, const float* b_sorted,
+                                   const uint32_t* perm_b, int64_t k, const float* D, const float* v, const float* g,
+                                   int64_t B, float* gv, float* ga, float* gb, float* gD, void* ws, size_t ws_bytes,
+                                   int32_t* d_status, laplex_stream_t stream) {
+    if (!size_ok(n) || !size_ok(k) || !batch_ok(B)) return LAPLEX_ERR_ARG;
+    if (!a_sorted || !perm_a || !b_sorted || !perm_b || !D || !v || !g || !ws) return LAPLEX_ERR_ARG;
+    if (!gv && !ga && !gb && !gD) return LAPLEX_ERR_ARG;
+    if (ws_bytes < gram_workspace_bytes(n, k, B)) return LAPLEX_ERR_WORKSPACE;
+    laplex_status s = check_ranges({{a_sorted, fbytes(n)}, {perm_a, fbytes(n)}, {b_sorted, fbytes(k)},
+                                    {perm_b, fbytes(k)}, {D, fbytes(k)}, {v, fbytes(n * B)}, {g, fbytes(n * B)}},
+                                   {{gv, fbytes(n * B)}, {ga, fbytes(n)}, {gb, fbytes(k)}, {gD, fbytes(k)},
+                                    {ws, ws_bytes}, {d_status, 4}});
+    if (s != LAPLEX_OK) return s;
+    Side A{a_sorted, perm_a, nullptr, n}, Bs{b_sorted, perm_b, nullptr, k};
+    return cuda_status(
+        launch_gram_backward(A, Bs, D, v, g, B, gv, ga, gb, gD, ws, d_status, (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -66,15 +66,22 @@ cudaError_t launch_rect_forward(Side O, Side I, const float* x, int64_t B, float
                                 int32_t* status, cudaStream_t stream);
 // Gradients of <g, out> for launch_rect_forward (g at O):
 //   gx [n_in][B], gO/gI anchor gradients, gtO/gtI phase gradients (each nullable).
+// accumulate: add the anchor and phase gradients into gO, gI, gtO, gtI instead of
+// writing them (gx is always written).
 cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g, int64_t B, const void* saved,
                                  float* gx, float* gO, float* gI, float* gtO, float* gtI, void* ws, int32_t* status,
-                                 cudaStream_t stream);
+                                 cudaStream_t stream, bool accumulate = false);
 
 // The bounded lookback against a predecessor that never publishes (failure-
 // detection self-check): ws holds the chain, zeroed here.
 cudaError_t launch_check_wait_bound(void* ws, int32_t* status, cudaStream_t stream);
 
 size_t gram_workspace_bytes(int64_t n, int64_t k, int64_t B);
+// Every gradient of <g, A diag(D) A^T v> (each output nullable): gv [n][B] = A D A^T g,
+// ga [n], gb [k] the anchor gradients, gD [k].
+cudaError_t launch_gram_backward(Side A, Side Bs, const float* D, const float* v, const float* g, int64_t B,
+                                 float* gv, float* ga, float* gb, float* gD, void* ws, int32_t* status,
+                                 cudaStream_t stream);
 cudaError_t launch_gram(Side A, Side Bs, const float* D, const float* v, int64_t B, float* y, float* w_saved,
                         const float* g, float* gD, void* ws, int32_t* status, cudaStream_t stream);
 

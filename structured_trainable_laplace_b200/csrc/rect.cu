@@ -268,6 +268,7 @@ struct LargePass {
     int64_t rows_per_group;
     int lpr;
     int chunk_atomic;
+    int accumulate;  // add the anchor / phase gradients into g_anchor / g_phase
 };
 
 __device__ __forceinline__ int64_t lower_bound_f(const float* a, int64_t n, float v) {
@@ -514,6 +515,8 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
         if (dst == nullptr) return;
         if (A.chunk_atomic)
             atomicAdd(dst + pr, v);
+        else if (A.accumulate)
+            dst[pr] += v;  // every row is visited once per launch
         else
             dst[pr] = v;
     };
@@ -720,6 +723,7 @@ struct Finish {
     float* out;      // [m][B] original order: sum_p w_p ZF
     float* g_anchor;  // sum_c h sum_p w_p (ZR - ZL)
     float* g_phase;   // sum_c h sum_p w'_p ZF
+    int accumulate;   // add into g_anchor / g_phase instead of writing
 };
 
 template <bool PHASED>
@@ -761,8 +765,8 @@ __global__ void __launch_bounds__(256) k_finish(Finish F) {
         gp += __shfl_xor_sync(0xffffffffu, gp, off);
     }
     if (lane == 0) {
-        if (F.g_anchor) F.g_anchor[pr] = ga;
-        if (PHASED && F.g_phase) F.g_phase[pr] = gp;
+        if (F.g_anchor) F.g_anchor[pr] = F.accumulate ? F.g_anchor[pr] + ga : ga;
+        if (PHASED && F.g_phase) F.g_phase[pr] = F.accumulate ? F.g_phase[pr] + gp : gp;
     }
 }
 
@@ -953,7 +957,7 @@ cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
     const int chunks = (A.B + lpr * vec - 1) / (lpr * vec);
     A.lpr = lpr;
     A.chunk_atomic = chunks > 1 ? 1 : 0;
-    if ((mode & kLmGrad) && A.chunk_atomic) {
+    if ((mode & kLmGrad) && A.chunk_atomic && !A.accumulate) {
         if (A.g_anchor) LAPLEX_TRY(cudaMemsetAsync(A.g_anchor, 0, sizeof(float) * A.m, st));
         if (A.g_phase) LAPLEX_TRY(cudaMemsetAsync(A.g_phase, 0, sizeof(float) * A.m, st));
     }
@@ -1078,7 +1082,7 @@ cudaError_t launch_rect_forward(Side O, Side I, const float* x, int64_t B, float
 
 cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g, int64_t B, const void* saved,
                                  float* gx, float* gO, float* gI, float* gtO, float* gtI, void* ws, int32_t* status,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool accumulate) {
     const bool phased = O.theta != nullptr;
     const RectPlan p = plan_rect(O.m, I.m, B, phased, ws);
     const int64_t sz = p.ms * (int64_t)p.Cb;
@@ -1097,6 +1101,7 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
             A.out = gx;
             A.g_anchor = gI;
             A.g_phase = gtI;
+            A.accumulate = accumulate;
             const int mode = (gx ? kLmExpand : 0) | ((gI || gtI) ? kLmGrad : 0);
             LAPLEX_TRY(large_pass(A, mode, st));
         }
@@ -1119,6 +1124,7 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
                 F.h = g;
                 F.g_anchor = gO;
                 F.g_phase = gtO;
+                F.accumulate = accumulate;
                 if (gO == nullptr) {
                     // k_finish keys the anchor sums on g_anchor; phase-only still needs a target
                     F.g_anchor = nullptr;
@@ -1136,6 +1142,7 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
                 A.Sst = Pst + sz;
                 A.g_anchor = gO;
                 A.g_phase = gtO;
+                A.accumulate = accumulate;
                 LAPLEX_TRY(large_pass(A, kLmGrad, st));
             }
         }
@@ -1157,6 +1164,7 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
         A.Sst = Pst ? Pst + sz : nullptr;
         A.g_anchor = gO;
         A.g_phase = gtO;
+        A.accumulate = accumulate;
         LAPLEX_TRY(large_pass(A, mode, st));
     }
     if (needI) {
@@ -1175,13 +1183,12 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
         F.out = gx;
         F.g_anchor = gI;
         F.g_phase = gtI;
+        F.accumulate = accumulate;
         LAPLEX_TRY(finish(F, st));
     }
     return cudaSuccess;
 }
 
-// Workspace of the Gram apply: the rectangular scratch sized for the paired pass
-// (2B channels), then three [k][B] row buffers.
 cudaError_t launch_check_wait_bound(void* ws, int32_t* status, cudaStream_t st) {
     // ws: flags [2] | agg [2] | inc [2] | anchors [2]
     char* b = (char*)ws;
@@ -1192,6 +1199,32 @@ cudaError_t launch_check_wait_bound(void* ws, int32_t* status, cudaStream_t st) 
     return cudaGetLastError();
 }
 
+// The middle of the Gram backward, one warp per small-side row j: x1 = D_j w_j,
+// x2 = D_j u_j (the inputs of the general products A (D w) and A (D u)) and
+// gD_j = <u_j, w_j>.  w and u are rows of ld floats.
+__global__ void __launch_bounds__(256) k_gram_mid2(const float* __restrict__ D, const float* __restrict__ w,
+                                                   const float* __restrict__ u, int ld, float* __restrict__ x1,
+                                                   float* __restrict__ x2, float* __restrict__ gD, int64_t k, int B) {
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= k) return;
+    const int lane = threadIdx.x & 31;
+    const float d = __ldg(D + r);
+    float acc = 0.f;
+    for (int c = lane; c < B; c += 32) {
+        const float wv = __ldg(w + r * ld + c), uv = __ldg(u + r * ld + c);
+        x1[r * B + c] = d * wv;
+        x2[r * B + c] = d * uv;
+        acc = fmaf(uv, wv, acc);
+    }
+    if (gD != nullptr) {
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) gD[r] = acc;
+    }
+}
+
+// Workspace of the Gram apply: the rectangular scratch sized for the paired pass
+// (2B channels), then three [k][2B] row buffers.
 size_t gram_workspace_bytes(int64_t n, int64_t k, int64_t B) {
     return plan_rect(n, k, 2 * B, false, nullptr, k).total;
 }
@@ -1233,6 +1266,58 @@ cudaError_t launch_gram(Side A, Side Bs, const float* D, const float* v, int64_t
                                                                        nullptr, (g && gD) ? gD : nullptr, Bs.m, (int)B));
     LAPLEX_TRY(cudaGetLastError());
     return launch_rect_forward(A, Bs, w2, B, y, nullptr, ws, status, st);  // y = A (D w)
+}
+
+// Every gradient of l = <g, A diag(D) A^T v>: with w = A^T v and u = A^T g,
+// gv = A (D u), gD = sum_c u w, and ga, gb the anchor gradients of the general
+// products A (D w) read by g and A (D u) read by v (dl/dA_ij = D_j sum_c (g_ic w_jc
+// + v_ic u_jc)); the second backward adds into the first's ga, gb.
+cudaError_t launch_gram_backward(Side A, Side Bs, const float* D, const float* v, const float* g, int64_t B,
+                                 float* gv, float* ga, float* gb, float* gD, void* ws, int32_t* status,
+                                 cudaStream_t st) {
+    const RectPlan p2 = plan_rect(A.m, Bs.m, 2 * B, false, ws, Bs.m);
+    const int64_t kb = Bs.m * B;
+    float* wpair = p2.rows3;           // [k][2B] (paired) or w | u ([k][B] each)
+    float* x1 = p2.rows3 + 2 * kb;     // [k][B]  D w
+    float* x2 = p2.rows3 + 3 * kb;     // [k][B]  D u
+    const float* w;
+    const float* u;
+    int ld;
+    if (A.m > Bs.m) {  // A^T v and A^T g in one paired reduce pass
+        const RectPlan pp = plan_rect(Bs.m, A.m, 2 * B, false, ws);
+        const int64_t sz = pp.ms * (int64_t)pp.Cb;
+        LAPLEX_TRY(reduce_parts(pp, Bs, A, v, 2 * B, pp.bufA, pp.bufA + sz, pp.bufA + 2 * sz, status, st, g));
+        Finish F{};
+        F.perm = Bs.perm;
+        F.m = Bs.m;
+        F.ZL = pp.bufA;
+        F.ZR = pp.bufA + sz;
+        F.ZF = pp.bufA + 2 * sz;
+        F.B = (int)(2 * B);
+        F.Cb = pp.Cb;
+        F.out = wpair;
+        LAPLEX_TRY(finish(F, st));
+        w = wpair;
+        u = wpair + B;
+        ld = (int)(2 * B);
+    } else {
+        LAPLEX_TRY(launch_rect_forward(Bs, A, v, B, wpair, nullptr, ws, status, st));       // w = A^T v
+        LAPLEX_TRY(launch_rect_forward(Bs, A, g, B, wpair + kb, nullptr, ws, status, st));  // u = A^T g
+        w = wpair;
+        u = wpair + kb;
+        ld = (int)B;
+    }
+    LAPLEX_TIMED("gram_mid", st,
+                 k_gram_mid2<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, w, u, ld, x1, x2, gD, Bs.m, (int)B));
+    LAPLEX_TRY(cudaGetLastError());
+    if (gv != nullptr) LAPLEX_TRY(launch_rect_forward(A, Bs, x2, B, gv, nullptr, ws, status, st));  // gv = A (D u)
+    if (ga != nullptr || gb != nullptr) {
+        LAPLEX_TRY(launch_rect_backward(A, Bs, x1, g, B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
+                                        false));
+        LAPLEX_TRY(launch_rect_backward(A, Bs, x2, v, B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
+                                        true));
+    }
+    return cudaSuccess;
 }
 
 }  // namespace laplex

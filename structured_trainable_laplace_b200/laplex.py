@@ -59,6 +59,7 @@ def lib():
             "laplex_apply_phased": ([P, P, I64, P, P, P, I64, P, I, P, I64, P, P, P, SZ, P, P], I),
             "laplex_backward": ([I, P, P, I64, P, P, P, I64, P, P, P, I64, P, P, P, P, P, P, P, SZ, P, P], I),
             "laplex_gram_apply": ([P, P, I64, P, P, I64, P, P, I64, P, P, P, P, P, SZ, P, P], I),
+            "laplex_gram_backward": ([P, P, I64, P, P, I64, P, P, P, I64, P, P, P, P, P, SZ, P, P], I),
             "laplex_check_wait_bound": ([P, SZ, P, P], I),
             "laplex_profile_enable": ([I], None),
             "laplex_profile_report": ([I, P, I, P, P], I),
@@ -77,7 +78,7 @@ def exported_symbols() -> list:
             "laplex_workspace_size", "laplex_saved_size", "laplex_apply_sym", "laplex_apply_sym_noalloc",
             "laplex_apply_general",
             "laplex_apply_transpose", "laplex_apply_phased", "laplex_backward", "laplex_gram_apply",
-            "laplex_check_wait_bound", "laplex_profile_enable", "laplex_profile_report"]
+            "laplex_gram_backward", "laplex_check_wait_bound", "laplex_profile_enable", "laplex_profile_report"]
 
 
 # ---------------------------------------------------------------- plumbing
@@ -300,6 +301,33 @@ def gram_apply(a_sorted, perm_a, b_sorted, perm_b, D, v, g=None, return_w=False)
     if g is not None:
         res += (gD,)
     return res[0] if len(res) == 1 else res
+
+
+def gram_backward(a_sorted, perm_a, b_sorted, perm_b, D, v, g, need=("gv", "ga", "gb", "gD")):
+    """Gradients of <g, A diag(D) A^T v>: a dict with the requested entries among
+    gv [n][B], ga [n], gb [k], gD [k]."""
+    vr, sq = _rows(v)
+    gr, _ = _rows(g)
+    n, B = vr.shape
+    k = b_sorted.numel()
+    d = _dev(v)
+    dev = v.device
+    out = {}
+    if "gv" in need:
+        out["gv"] = torch.empty_like(vr)
+    if "ga" in need:
+        out["ga"] = torch.empty(n, dtype=torch.float32, device=dev)
+    if "gb" in need:
+        out["gb"] = torch.empty(k, dtype=torch.float32, device=dev)
+    if "gD" in need:
+        out["gD"] = torch.empty(k, dtype=torch.float32, device=dev)
+    ws = workspace(workspace_size(OP_GRAM, n, k, B), d)
+    _ok(lib().laplex_gram_backward(_p(a_sorted), _p(perm_a), n, _p(b_sorted), _p(perm_b), k, _p(D), _p(vr), _p(gr), B,
+                                   _p(out.get("gv")), _p(out.get("ga")), _p(out.get("gb")), _p(out.get("gD")), _p(ws),
+                                   ws.numel(), _p(status_word(d)), _stream(d)), "gram_backward")
+    if "gv" in out and sq:
+        out["gv"] = out["gv"].reshape(-1)
+    return out
 
 
 # ---------------------------------------------------------------- diagnostics

@@ -124,3 +124,35 @@ def test_gram_full_size(L):
     """Flattened 3x1024x1024 image: n = 3,145,728, k = 65,536, B = 8."""
     w = inputs.gram_image(0)
     compare_gram(L, w["a"], w["b"], w["D"], w["v"], w["g"], tag="image")
+
+
+def compare_gram_backward(L, a, b, D, v, g, ref_fn, tag=""):
+    sa, pa = L.sort_anchors(dev(a))
+    sb, pb = L.sort_anchors(dev(b))
+    got = L.gram_backward(sa, pa, sb, pb, dev(D), dev(v), dev(g))
+    L.check()
+    ref, tw = ref_fn(a, b, D, v, g), ref_fn(a, b, D, v, g, twin=True)
+    for key in ("gv", "ga", "gb", "gD"):
+        assert_close(host(got[key]), ref[key], tw[key], f"gram {key} {tag}")
+
+
+@pytest.mark.parametrize("n,k,B,quant", [(4000, 150, 3, None), (150, 4000, 2, None), (2000, 2000, 4, 0.05),
+                                         (1, 1, 1, None), (6001, 64, 16, 0.02), (777, 900, 8, 0.25)])
+def test_gram_full_backward_small(L, n, k, B, quant):
+    """gv, ga, gb, gD of <g, A diag(D) A^T v> against the dense definition (ties
+    inside a, inside b and between them when quantised)."""
+    rng = np.random.default_rng(n * 5 + k + B)
+    a, b = rng.uniform(0, 25, n), rng.uniform(0, 25, k)
+    if quant:
+        a, b = np.round(a / quant) * quant, np.round(b / quant) * quant
+    a, b = a.astype(np.float32), b.astype(np.float32)
+    D = np.log1p(np.exp(rng.standard_normal(k))).astype(np.float32)
+    v = rng.standard_normal((n, B)).astype(np.float32)
+    g = rng.standard_normal((n, B)).astype(np.float32)
+    compare_gram_backward(L, a, b, D, v, g, oracle.dense.gram_backward, tag=f"n{n} k{k} B{B} q{quant}")
+
+
+def test_gram_full_backward_image(L):
+    """Flattened 3x1024x1024 image: every gradient against the composed C oracle."""
+    w = inputs.gram_image(0)
+    compare_gram_backward(L, w["a"], w["b"], w["D"], w["v"], w["g"], oracle.gram_backward, tag="image")
