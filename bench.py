@@ -55,6 +55,7 @@ def make_workload(name: str, rank: int, n: int | None = None):
         "sym1e9": lambda s: inputs.sym_extreme(s),
         "phased_head": lambda s: inputs.phased_head_2p22(s, n=n or (1 << 22)),
         "gram_image": lambda s: inputs.gram_image(s, n=n or 3 * 1024 * 1024),
+        "gram_image_full": lambda s: _full_gram(inputs.gram_image(s, n=n or 3 * 1024 * 1024)),
     }[name]
     w = gen(rank)
     if rank != 0:
@@ -62,6 +63,13 @@ def make_workload(name: str, rank: int, n: int | None = None):
         for key in ("a", "b", "phi", "psi", "D"):
             if key in w0:
                 w.arrays[key] = w0[key]
+    return w
+
+
+def _full_gram(w):
+    """The Gram workload stepped with every gradient (gv, ga, gb, gD)."""
+    w.op = "gram_full"
+    w.name = w.name + "_full_backward"
     return w
 
 
@@ -90,6 +98,11 @@ def compulsory_bytes(w) -> int:
         fwd = 8 * n + 4 * n * B + 4 * n * B + 4 * k
         bwd = 8 * n + 4 * n * B + 4 * k
         return sort + fwd + bwd
+    if w.op == "gram_full":
+        sort = 12 * n + 12 * k
+        fwd = 8 * n + 4 * n * B + 4 * n * B + 4 * k
+        bwd = 8 * n + 8 * n * B + 4 * n * B + 4 * n + 8 * k  # v, g in; gv, ga out; gb, gD
+        return sort + fwd + bwd
     raise ValueError(w.op)
 
 
@@ -114,10 +127,11 @@ def kernel_bytes_per_launch(kernel: str, w) -> float | None:
             "radix_pass": (12 * n + 3 * 16 * n) / 4.0,
         }
         return table.get(kernel)
-    if w.op == "gram":
+    if w.op in ("gram", "gram_full"):
         table = {
-            "large_accum": (8 + 4 * B) * n,
+            "large_accum": (8 + 8 * B) * n,                  # paired pass: s, perm, v and g rows
             "large_expand": (8 + 4 * B) * n,
+            "large_accum_grad": (8 + 4 * B + 4) * n,         # s, perm, upstream rows, ga
             "radix_pass": (12 * n + 3 * 16 * n) / 4.0,
         }
         return table.get(kernel)
@@ -162,6 +176,10 @@ class Step:
         if w.op == "gram":
             y, gD = L.gram_apply(sa, pa, sb[0], sb[1], t["D"], t["v"], g=t["g"])
             return {"y": y, "gD": gD}
+        if w.op == "gram_full":
+            y = L.gram_apply(sa, pa, sb[0], sb[1], t["D"], t["v"])
+            gr = L.gram_backward(sa, pa, sb[0], sb[1], t["D"], t["v"], t["g"])
+            return {"y": y, **gr}
         raise ValueError(w.op)
 
 
@@ -253,7 +271,10 @@ def oracle_sample(w, budget_s: float):
             k_s = max(1, int(round(w.k * n_s / w.n)))
             ws = inputs.gram(n_s, k_s, w.B, seed=123)
             oracle.gram_apply(ws["a"], ws["b"], ws["D"], ws["v"])
-            oracle.gram_backward_D(ws["a"], ws["b"], ws["v"], ws["g"])
+            if w.op == "gram_full":
+                oracle.gram_backward(ws["a"], ws["b"], ws["D"], ws["v"], ws["g"])
+            else:
+                oracle.gram_backward_D(ws["a"], ws["b"], ws["v"], ws["g"])
             units = n_s * w.B
         dt = time.perf_counter() - t0
         if dt >= budget_s or n_s >= w.n:
@@ -280,7 +301,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="sym2p24",
-                    choices=["sym2p24", "small", "phased_head", "gram_image", "sym1e9"])
+                    choices=["sym2p24", "small", "phased_head", "gram_image", "gram_image_full", "sym1e9"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
     ap.add_argument("--n", type=int, default=None, help="large-side anchors (profiling captures of a smaller case)")
     args = ap.parse_args()
