@@ -34,6 +34,11 @@ size_t sort_workspace_bytes(int64_t n);
 cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
                         cudaStream_t stream);
 
+// out[perm[r]] = v[r] (4-byte rows) through destination buckets (sort.cu); v is
+// overwritten (it holds the regrouped values of the last split).
+size_t unpermute_workspace_bytes(int64_t n);
+cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* out, void* ws, cudaStream_t stream);
+
 // sym.cu
 size_t sym_workspace_bytes(int64_t n, int64_t B);
 size_t sym_saved_bytes(int64_t n, int64_t B);

@@ -250,7 +250,172 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
     }
 }
 
+// ---------------------------------------------------------- unpermute
+//
+// out[perm[r]] = v[r] for vectors whose rows are single floats and too large for
+// the L2.  A direct scatter makes every 4-byte store a separate sector request
+// (about 23 G stores/s fully random on a B200, 34 G/s inside 16 MB windows,
+// 93 G/s inside 64 KB windows), so the (destination, value) pairs are regrouped
+// instead: two split passes group them by 16 bits of the destination (8 bits
+// each), so that window q holds exactly the destinations [q << s, (q + 1) << s)
+// (its size and where its pairs go follow from n alone: no histogram, no lookback,
+// and the order inside a window is free), then one CTA per window places its
+// values in shared memory and writes the window out contiguously.
+
+constexpr int kSplitItems = 16;
+constexpr int kSplitTile = kNT * kSplitItems;
+constexpr int kPlaceMaxWindow = 1 << 14;  // floats of a window placed in shared memory
+
+// One tile of pairs: the bucket of p is p >> shift; the tile's pairs all share
+// its bits above the lowest 8 (the first pass has at most 256 buckets, and the
+// second pass's tiles lie inside one first-pass bucket).  Per-bucket counts
+// (shared atomics), a block scan into per-bucket starts, one global cursor claim
+// per bucket, then runs of equal buckets leave as contiguous stores.
+__global__ void __launch_bounds__(kNT) k_bucket_split(const uint32_t* __restrict__ p_in, const float* __restrict__ v_in,
+                                                      int64_t n, int shift, uint32_t* cursor, uint32_t* __restrict__ p_out,
+                                                      float* __restrict__ v_out) {
+    __shared__ uint32_t s_cnt[kRadix], s_start[kRadix], s_base[kRadix], s_scan[kNW];
+    __shared__ uint32_t s_p[kSplitTile];
+    __shared__ float s_v[kSplitTile];
+    const int tid = threadIdx.x;
+    const int64_t base = (int64_t)blockIdx.x * kSplitTile;
+    s_cnt[tid] = 0;
+    __syncthreads();
+    const uint32_t last = (uint32_t)(n - 1);
+    uint32_t pv[kSplitItems], rk[kSplitItems];
+    float vv[kSplitItems];
+#pragma unroll
+    for (int i = 0; i < kSplitItems; ++i) {
+        const int64_t idx = base + i * kNT + tid;
+        if (idx < n) {
+            pv[i] = min(__ldcs(p_in + idx), last);
+            vv[i] = __ldcs(v_in + idx);
+            rk[i] = atomicAdd(&s_cnt[(pv[i] >> shift) & 0xffu], 1u);
+        }
+    }
+    __syncthreads();
+    const uint32_t hi = ((min(__ldg(p_in + base), last)) >> shift) & ~0xffu;  // the tile's common upper bits
+    uint32_t tot;
+    const uint32_t cnt = s_cnt[tid];
+    s_start[tid] = block_excl_scan_256(cnt, s_scan, &tot);
+    if (cnt) s_base[tid] = atomicAdd(cursor + (hi | tid), cnt);
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kSplitItems; ++i) {
+        const int64_t idx = base + i * kNT + tid;
+        if (idx < n) {
+            const uint32_t q = s_start[(pv[i] >> shift) & 0xffu] + rk[i];
+            s_p[q] = pv[i];
+            s_v[q] = vv[i];
+        }
+    }
+    __syncthreads();
+    const int count = (n - base) < kSplitTile ? (int)(n - base) : kSplitTile;
+    for (int q = tid; q < count; q += kNT) {
+        const uint32_t p = s_p[q], b = (p >> shift) & 0xffu;
+        const int64_t dst = (int64_t)s_base[b] + (q - (int)s_start[b]);
+        if (dst < n) {  // always, for a permutation; a bad perm never writes out of range
+            p_out[dst] = p;
+            v_out[dst] = s_v[q];
+        }
+    }
+}
+
+__global__ void k_bucket_cursors(uint32_t* cursor, int64_t count, int shift) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < count) cursor[i] = (uint32_t)(i << shift);
+}
+
+// One CTA per window of W = 1 << shift destinations: its pairs (contiguous after
+// the splits) go to a shared-memory copy of the window, which then leaves with
+// contiguous stores.
+__global__ void __launch_bounds__(kNT) k_place_window(const uint32_t* __restrict__ p, const float* __restrict__ v,
+                                                      int64_t n, int shift, float* __restrict__ out) {
+    extern __shared__ float s_win[];
+    const int64_t w0 = (int64_t)blockIdx.x << shift;
+    const int cnt = (int)min((int64_t)1 << shift, n - w0);
+    for (int i = threadIdx.x; i < cnt; i += kNT) {
+        const int64_t d = (int64_t)__ldcs(p + w0 + i) - w0;
+        if (d >= 0 && d < cnt) s_win[d] = __ldcs(v + w0 + i);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += kNT) __stcs(out + w0 + i, s_win[i]);
+}
+
+// out[p[i]] = v[i], i in order, for windows too large for shared memory.
+__global__ void __launch_bounds__(kNT) k_scatter_pairs(const uint32_t* __restrict__ p, const float* __restrict__ v,
+                                                       int64_t n, float* __restrict__ out) {
+    const int64_t stride = (int64_t)gridDim.x * kNT * 4;
+    for (int64_t i0 = (int64_t)blockIdx.x * kNT * 4 + threadIdx.x; i0 < n; i0 += stride) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t i = i0 + u * kNT;
+            if (i < n) {
+                const uint32_t d = __ldcs(p + i);
+                if ((int64_t)d < n) out[d] = __ldcs(v + i);
+            }
+        }
+    }
+}
+
 }  // namespace
+
+size_t unpermute_workspace_bytes(int64_t n) {
+    return 3 * align_up((size_t)n * 4, 256) + (size_t)4 * 65536;
+}
+
+cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* out, void* ws, cudaStream_t stream) {
+    if (n <= 0) return cudaSuccess;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const auto scatter_grid = [&](int64_t m) {
+        return (int)std::max<int64_t>(1, std::min<int64_t>((m + kNT * 4 - 1) / (kNT * 4), (int64_t)sms * 8));
+    };
+    int bits = 0;
+    while ((1ll << bits) < n) ++bits;
+    // two 8-bit levels above the window bits s2 (windows of 2^s2 destinations)
+    const int s2 = bits > 16 ? bits - 16 : 0, s1 = s2 + 8;
+    if (s1 < 12) {  // second-level tiles would straddle first-level buckets: one plain scatter
+        LAPLEX_TIMED("unpermute_place", stream,
+                     k_scatter_pairs<<<scatter_grid(n), kNT, 0, stream>>>(perm, v, n, out));
+        return cudaGetLastError();
+    }
+    char* q = (char*)ws;
+    uint32_t* p1 = (uint32_t*)q;
+    q += align_up((size_t)n * 4, 256);
+    float* v1 = (float*)q;
+    q += align_up((size_t)n * 4, 256);
+    uint32_t* p2 = (uint32_t*)q;
+    q += align_up((size_t)n * 4, 256);
+    uint32_t* cursor = (uint32_t*)q;  // 65536 entries
+    float* v2 = v;                    // v is read only by the first split
+    const int64_t tiles = (n + kSplitTile - 1) / kSplitTile;
+    const int64_t nb1 = ((n - 1) >> s1) + 1, nb2 = ((n - 1) >> s2) + 1;  // buckets of each level
+    LAPLEX_TIMED("unpermute_split", stream, k_bucket_cursors<<<1, kRadix, 0, stream>>>(cursor, nb1, s1));
+    LAPLEX_TIMED("unpermute_split", stream,
+                 k_bucket_split<<<(unsigned)tiles, kNT, 0, stream>>>(perm, v, n, s1, cursor, p1, v1));
+    // bucket q of the first level fills [q << s1, (q + 1) << s1) and 2^s1 is a
+    // multiple of the tile, so every second-level tile lies inside one of them
+    LAPLEX_TIMED("unpermute_split", stream,
+                 k_bucket_cursors<<<(unsigned)((nb2 + kNT - 1) / kNT), kNT, 0, stream>>>(cursor, nb2, s2));
+    LAPLEX_TIMED("unpermute_split", stream,
+                 k_bucket_split<<<(unsigned)tiles, kNT, 0, stream>>>(p1, v1, n, s2, cursor, p2, v2));
+    if ((1ll << s2) <= kPlaceMaxWindow) {
+        static bool ready = false;
+        if (!ready) {
+            const cudaError_t e = cudaFuncSetAttribute(k_place_window, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)(sizeof(float) * kPlaceMaxWindow));
+            if (e != cudaSuccess) return e;
+            ready = true;
+        }
+        LAPLEX_TIMED("unpermute_place", stream,
+                     k_place_window<<<(unsigned)nb2, kNT, sizeof(float) << s2, stream>>>(p2, v2, n, s2, out));
+    } else {
+        LAPLEX_TIMED("unpermute_place", stream, k_scatter_pairs<<<scatter_grid(n), kNT, 0, stream>>>(p2, v2, n, out));
+    }
+    return cudaGetLastError();
+}
 
 size_t sort_workspace_bytes(int64_t n) {
     const int64_t T = (n + kTile - 1) / kTile;

@@ -65,6 +65,9 @@ struct SymGeo {
 // Single channel (B = 1): tiles of k1NT threads x k1E rows, loaded straight into
 // registers (see the one-channel kernels below).
 constexpr int k1NT = 256, k1E = 16, k1NW = k1NT / 32, k1R = k1NT * k1E;
+// Above this many rows (a 64 MB single-channel output) the one-channel sweeps
+// write sorted-order outputs and launch_unpermute places them.
+constexpr int64_t kUnpermuteMinRows = 1ll << 24;
 
 inline int64_t rows_per_tile(int C) {
     return C == 1 ? k1R : (C <= 8 ? 32 * kE : (32 * kE * 8) / C);
@@ -973,12 +976,35 @@ __global__ void __launch_bounds__(k1NT, 3) k_sym1_agg(SymScan a, const float* __
     }
 }
 
+// A thread's 16 outputs: scattered through the permutation, or (sorted_out) in
+// sorted order with 16-byte stores, for a later bucketed unpermute.
+__device__ __forceinline__ void put_rows1(float* __restrict__ dst, const float (&val)[k1E], const Rows1& r, int64_t n,
+                                          int sorted_out) {
+    if (sorted_out) {
+        if (r.row0 + k1E <= n) {
+            float4* d4 = reinterpret_cast<float4*>(dst + r.row0);
+#pragma unroll
+            for (int q = 0; q < k1E / 4; ++q)
+                __stcs(d4 + q, make_float4(val[4 * q], val[4 * q + 1], val[4 * q + 2], val[4 * q + 3]));
+        } else {
+#pragma unroll
+            for (int e = 0; e < k1E; ++e)
+                if (r.row0 + e < n) dst[r.row0 + e] = val[e];
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < k1E; ++e)
+            if (r.row0 + e < n) __stcs(dst + r.p[e], val[e]);
+    }
+}
+
 // Sweep for one channel: NV = 1 forward (xs -> y), NV = 2 backward (xs, gs -> gx,
 // ga), from the sorted copies, RS and the range carries (as k_sym_sweep).
 template <int NV>
 __global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a, const float* __restrict__ xs,
                                                        const float* __restrict__ gs, RangeState sx, RangeState sg,
-                                                       float* __restrict__ out, float* __restrict__ ga) {
+                                                       float* __restrict__ out, float* __restrict__ ga,
+                                                       int sorted_out) {
     __shared__ Cross1<NV> cx;
     __shared__ double2 s_runL[NV];
     const CtaTiles cw = cta_tiles(a);
@@ -1100,8 +1126,9 @@ __global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a,
 #pragma unroll
             for (int e = 0; e < k1E; ++e) {
                 pl = fmaf(fabsf(d[e]), pl, xv[0][e]);
-                if (r.row0 + e < a.n) __stcs(out + r.p[e], yv[e] + pl);
+                yv[e] += pl;
             }
+            put_rows1(out, yv, r, a.n, sorted_out);
         } else {
             LP ax = inR[0], ag = inR[NV - 1];
             float gxr[k1E], gap[k1E];
@@ -1120,11 +1147,11 @@ __global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a,
                 const float xe = xv[0][e], ge = xv[NV - 1][e], dv = d[e];
                 ax = lp_step_x(ax, dv, xe);
                 ag = lp_step_x(ag, dv, ge);
-                if (r.row0 + e < a.n) {
-                    if (out != nullptr) __stcs(out + r.p[e], gxr[e] + ag.P);
-                    if (ga != nullptr) __stcs(ga + r.p[e], fmaf(-ge, ax.L, fmaf(-xe, ag.L, gap[e])));
-                }
+                gxr[e] += ag.P;
+                gap[e] = fmaf(-ge, ax.L, fmaf(-xe, ag.L, gap[e]));
             }
+            if (out != nullptr) put_rows1(out, gxr, r, a.n, sorted_out);
+            if (ga != nullptr) put_rows1(ga, gap, r, a.n, sorted_out);
         }
         if (threadIdx.x == 0) {
             const float fl = (lo + k1R <= a.n) ? __ldg(a.s + lo + k1R - 1) : kHighAnchor;
@@ -1150,6 +1177,8 @@ struct SymPlan {
     size_t state_bytes;          // RS, Lin, Rin, Lagg, Ragg of one vector
     size_t saved_state_bytes;    // RS, Lin, Rin of one vector
     size_t sorted_bytes;         // sorted copy of one vector (G * T * R * C floats)
+    bool bucketed;               // one channel past the L2: outputs leave through launch_unpermute
+    size_t unperm_bytes;         // two sorted-order outputs + the unpermute scratch
     size_t total;
 };
 
@@ -1170,7 +1199,19 @@ SymPlan plan_sym(int64_t n, int64_t B, int sms) {
     p.sorted_bytes = align_up(sizeof(float) * (size_t)p.G * p.T * p.R * p.C, 256);
     // per vector (x, g): the scan state and the sorted copy
     p.total = 2 * (p.state_bytes + p.sorted_bytes);
+    // single floats scattered through the permutation into an output far larger
+    // than the L2 are written in sorted order and regrouped by destination instead
+    p.bucketed = (p.C == 1 && n > kUnpermuteMinRows);
+    p.unperm_bytes = p.bucketed ? 2 * align_up(sizeof(float) * (size_t)n, 256) + unpermute_workspace_bytes(n) : 0;
+    p.total += p.unperm_bytes;
     return p;
+}
+
+// The sorted-order outputs and the unpermute scratch (after the scan state and
+// the sorted copies in the workspace).
+float* unperm_outputs(const SymPlan& p, void* ws) { return (float*)((char*)ws + 2 * (p.state_bytes + p.sorted_bytes)); }
+void* unperm_scratch(const SymPlan& p, void* ws, int64_t n) {
+    return (char*)unperm_outputs(p, ws) + 2 * align_up(sizeof(float) * (size_t)n, 256);
 }
 
 RangeState carve(const SymPlan& p, double2* base, bool with_aggs) {
@@ -1249,16 +1290,27 @@ cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm,
     return cudaGetLastError();
 }
 
+#define LAPLEX_TRY_SYM(expr)                 \
+    do {                                     \
+        cudaError_t e_ = (expr);             \
+        if (e_ != cudaSuccess) return e_;    \
+    } while (0)
+
 // The forward sweep (y from the sorted copy, RS and the range carries).
 template <int C>
 cudaError_t launch_sym_sweep_fwd(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms,
-                                 const float* xs, const RangeState& sx, float* y, cudaStream_t st) {
+                                 const float* xs, const RangeState& sx, float* y, cudaStream_t st,
+                                 void* ws = nullptr) {
     if constexpr (C == 1) {
         static int occ_cache = 0;
         const int occ = prepare(k_sym1_sweep<1>, k1NT, 0, occ_cache);
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
-        LAPLEX_TIMED("sym_fwd", st, k_sym1_sweep<1><<<grid, k1NT, 0, st>>>(a, xs, nullptr, sx, sx, y, nullptr));
+        const bool bucketed = p.bucketed && ws != nullptr;
+        float* ys = bucketed ? unperm_outputs(p, ws) : y;
+        LAPLEX_TIMED("sym_fwd", st,
+                     k_sym1_sweep<1><<<grid, k1NT, 0, st>>>(a, xs, nullptr, sx, sx, ys, nullptr, bucketed ? 1 : 0));
+        if (bucketed) return launch_unpermute(perm, ys, n, y, unperm_scratch(p, ws, n), st);
     } else {
         using SM = SweepSmem<C, 1, kAheadFwd>;
         static int occ_cache = 0;
@@ -1288,7 +1340,7 @@ cudaError_t sym_forward_t(const float* s, const uint32_t* perm, int64_t n, const
     }
     cudaError_t e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
     if (e != cudaSuccess) return e;
-    return launch_sym_sweep_fwd<C>(p, s, perm, n, B, sms, xs, sx, y, st);
+    return launch_sym_sweep_fwd<C>(p, s, perm, n, B, sms, xs, sx, y, st, ws);
 }
 
 template <int C>
@@ -1323,7 +1375,15 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
         const int occ = prepare(k_sym1_sweep<2>, k1NT, 0, occ_cache);
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
-        LAPLEX_TIMED("sym_bwd", st, k_sym1_sweep<2><<<grid, k1NT, 0, st>>>(a, xs, gs, sx, sg, gx, ga));
+        float* gxs = p.bucketed && gx ? unperm_outputs(p, ws) : gx;
+        float* gas = p.bucketed && ga ? unperm_outputs(p, ws) + align_up((size_t)n, 64) : ga;
+        LAPLEX_TIMED("sym_bwd", st,
+                     k_sym1_sweep<2><<<grid, k1NT, 0, st>>>(a, xs, gs, sx, sg, gxs, gas, p.bucketed ? 1 : 0));
+        if (p.bucketed) {
+            void* scratch = unperm_scratch(p, ws, n);
+            if (gx) LAPLEX_TRY_SYM(launch_unpermute(perm, gxs, n, gx, scratch, st));
+            if (ga) LAPLEX_TRY_SYM(launch_unpermute(perm, gas, n, ga, scratch, st));
+        }
     } else {
         using SM = SweepSmem<C, 2, kAheadBwd>;
         static int occ_cache = 0;

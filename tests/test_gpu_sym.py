@@ -69,6 +69,13 @@ def test_wide_gaps_and_underflow(L):
     compare(L, a, x, g, tag="gaps")
 
 
+def test_single_channel_past_the_unpermute_threshold(L):
+    """B = 1 with n > 2^24: the sweeps write sorted-order outputs and the bucketed
+    unpermute places them (y, gx, ga), with ties."""
+    w = inputs.symmetric((1 << 24) + 4097, 1, seed=31, tie_frac=0.01)
+    compare(L, w["a"], w["x"], w["g"], tag="n 2^24+4097 B1")
+
+
 def test_full_size_2p24_b16(L):
     w = inputs.sym_2p24_b16(0)
     compare(L, w["a"], w["x"], w["g"], tag="2^24 x 16")
