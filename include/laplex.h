@@ -108,6 +108,35 @@ size_t laplex_sort_workspace_size(int64_t n);
 laplex_status laplex_sort_anchors(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws,
                                   size_t ws_bytes, int32_t* d_status, laplex_stream_t stream);
 
+/* Bytes of workspace laplex_resort_anchors needs for n anchors. */
+size_t laplex_resort_workspace_size(int64_t n);
+
+/* laplex_resort_anchors *d_path values. */
+#define LAPLEX_RESORT_SORTED 0   /* a[perm_prev] was already in the stable order */
+#define LAPLEX_RESORT_REPAIRED 1 /* the displaced anchors were sorted and placed */
+#define LAPLEX_RESORT_FULL 2     /* the full radix sort ran */
+
+/* Warm-start re-sort: the same output as laplex_sort_anchors(a, ...), bit for bit,
+ * starting from the permutation of an earlier sort of anchors that have moved
+ * since (trainable anchors between two steps; technical summary section 2.2:
+ * the scans run over the sorted anchors).
+ *   a          [n] fp32, original order (read only), the anchors as they are now.
+ *   perm_prev  [n] uint32 (read only): any array; the fast path applies when it
+ *              is a permutation of 0..n-1 that nearly sorts a.  Entries >= n are
+ *              clamped to n - 1 (and then send the call to the full sort).
+ *   a_sorted, perm [n] out: as laplex_sort_anchors.
+ *   d_path     optional device int32 out: LAPLEX_RESORT_SORTED / _REPAIRED / _FULL.
+ * An anchor whose composite (anchor, index) exceeds every one before it in the
+ * order perm_prev gives and is below every one after it is already at its final
+ * rank; the others (the displaced ones) are sorted by the radix sort and written
+ * into the positions they leave free.  When more than half are displaced, or
+ * perm_prev is not a permutation, the full radix sort of a runs instead.  The
+ * choice is made on the device: the call does not synchronise.  NaN or infinite
+ * anchors set LAPLEX_ERR_NONFINITE (on the fast path, those perm_prev reaches). */
+laplex_status laplex_resort_anchors(const float* a, int64_t n, const uint32_t* perm_prev, float* a_sorted,
+                                    uint32_t* perm, void* ws, size_t ws_bytes, int32_t* d_status, int32_t* d_path,
+                                    laplex_stream_t stream);
+
 /* ------------------------------------------------------------ operators */
 
 /* Bytes of workspace for the forward and the backward of `op` (the larger of

@@ -133,6 +133,19 @@ laplex_status laplex_sort_anchors(const float* a, int64_t n, float* a_sorted, ui
     return cuda_status(launch_sort(a, n, a_sorted, perm, ws, d_status, (cudaStream_t)stream));
 }
 
+size_t laplex_resort_workspace_size(int64_t n) { return size_ok(n) ? resort_workspace_bytes(n) : 0; }
+
+laplex_status laplex_resort_anchors(const float* a, int64_t n, const uint32_t* perm_prev, float* a_sorted,
+                                    uint32_t* perm, void* ws, size_t ws_bytes, int32_t* d_status, int32_t* d_path,
+                                    laplex_stream_t stream) {
+    if (!size_ok(n) || !a || !perm_prev || !a_sorted || !perm || !ws) return LAPLEX_ERR_ARG;
+    if (ws_bytes < resort_workspace_bytes(n)) return LAPLEX_ERR_WORKSPACE;
+    laplex_status s = check_ranges({{a, fbytes(n)}, {perm_prev, fbytes(n)}},
+                                   {{a_sorted, fbytes(n)}, {perm, fbytes(n)}, {ws, ws_bytes}, {d_status, 4}, {d_path, 4}});
+    if (s != LAPLEX_OK) return s;
+    return cuda_status(launch_resort(a, n, perm_prev, a_sorted, perm, ws, d_status, d_path, (cudaStream_t)stream));
+}
+
 size_t laplex_workspace_size(laplex_op op, int64_t n, int64_t k, int64_t B) {
     if (!size_ok(n) || !batch_ok(B)) return 0;
     if (op == LAPLEX_OP_SYM) return sym_workspace_bytes(n, B);

@@ -31,8 +31,17 @@ struct ProfScope {
 
 // sort.cu
 size_t sort_workspace_bytes(int64_t n);
+// n_dev (optional): the count to sort, read on the device (<= n, which sizes the
+// launches and the workspace); 0 makes every kernel return at once.
 cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
-                        cudaStream_t stream);
+                        cudaStream_t stream, const int64_t* n_dev = nullptr);
+
+// resort.cu: warm-start re-sort from a previous permutation; *path (optional,
+// device) gets which way the sorted order was reached.
+constexpr int32_t kResortSorted = 0, kResortRepaired = 1, kResortFull = 2;
+size_t resort_workspace_bytes(int64_t n);
+cudaError_t launch_resort(const float* a, int64_t n, const uint32_t* perm_prev, float* a_sorted, uint32_t* perm,
+                          void* ws, int32_t* status, int32_t* path, cudaStream_t stream);
 
 // out[perm[r]] = v[r] (4-byte rows) through destination buckets (sort.cu); v is
 // overwritten (it holds the regrouped values of the last split).

@@ -54,9 +54,12 @@ __device__ __forceinline__ uint32_t block_excl_scan_256(uint32_t v, uint32_t* s_
     return base + inc - v;
 }
 
-__global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a, int64_t n, uint32_t* hist,
-                                                    unsigned long long* look0, int64_t look_words, int32_t* status) {
+__global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a, int64_t n, const int64_t* n_dev,
+                                                    uint32_t* hist, unsigned long long* look0, int32_t* status) {
     __shared__ uint32_t s_hist[kNW][4][kRadix];  // one histogram set per warp: fewer colliding atomics
+    if (n_dev != nullptr) n = min(n, *n_dev);  // count known only on the device (<= the launch bound)
+    if (n <= 0) return;
+    const int64_t look_words = (n + kTile - 1) / kTile * kRadix;
     for (int i = threadIdx.x; i < kNW * 4 * kRadix; i += kNT) (&s_hist[0][0][0])[i] = 0;
     __syncthreads();
     const int64_t stride = (int64_t)gridDim.x * kNT;
@@ -98,8 +101,8 @@ __global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a,
 template <int MODE>
 __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__ a, const uint32_t* __restrict__ keys_in,
                                                     const uint32_t* __restrict__ vals_in, uint32_t* __restrict__ keys_out,
-                                                    uint32_t* __restrict__ vals_out, int64_t n, int shift,
-                                                    const uint32_t* __restrict__ hist, uint32_t* counter,
+                                                    uint32_t* __restrict__ vals_out, int64_t n, const int64_t* n_dev,
+                                                    int shift, const uint32_t* __restrict__ hist, uint32_t* counter,
                                                     unsigned long long* look, unsigned long long* look_next,
                                                     int32_t* status) {
     __shared__ uint32_t s_whist[kNW][kRadix];
@@ -111,11 +114,18 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
     __shared__ int64_t s_tile;
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    if (n_dev != nullptr) {
+        // count known only on the device (<= the launch bound): the first
+        // ceil(n / kTile) CTAs claim one tile each, the others leave at once
+        n = min(n, *n_dev);
+        if ((int64_t)blockIdx.x * kTile >= n) return;
+    }
     if (tid == 0) s_tile = atomicAdd(counter, 1u);
     for (int i = tid; i < kNW * kRadix; i += kNT) (&s_whist[0][0])[i] = 0;
     __syncthreads();
     const int64_t tile = s_tile;
     const int64_t base = tile * kTile;
+    if (base >= n) return;  // the tiles of a smaller device-side count (uniform per CTA)
     look_next[tile * kRadix + tid] = 0ull;  // the pass after next reuses this region
 
     // global exclusive digit offsets for this pass
@@ -428,7 +438,7 @@ size_t sort_workspace_bytes(int64_t n) {
 }
 
 cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, const int64_t* n_dev) {
     const int64_t T = (n + kTile - 1) / kTile;
     char* p = (char*)ws;
     uint32_t* keys_alt = (uint32_t*)p;
@@ -450,17 +460,17 @@ cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* pe
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t want = (n + kNT * 8 - 1) / (kNT * 8);
     const int hblocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
-    LAPLEX_TIMED("radix_hist", stream, k_radix_hist<<<hblocks, kNT, 0, stream>>>(a, n, hist, look[0], T * kRadix, status));
+    LAPLEX_TIMED("radix_hist", stream, k_radix_hist<<<hblocks, kNT, 0, stream>>>(a, n, n_dev, hist, look[0], status));
     uint32_t* ka = (uint32_t*)a_sorted;
     // pass 0: a -> alt; pass 1: alt -> out; pass 2: out -> alt; pass 3: alt -> out
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<0><<<(unsigned)T, kNT, 0, stream>>>(a, nullptr, nullptr, keys_alt, vals_alt, n, 0, hist + 0 * kRadix,
-                                                     counters + 0, look[0], look[1], status));
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, 8, hist + 1 * kRadix,
-                                                     counters + 1, look[1], look[0], status));
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, ka, perm, keys_alt, vals_alt, n, 16, hist + 2 * kRadix,
-                                                     counters + 2, look[0], look[1], status));
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<2><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, 24, hist + 3 * kRadix,
-                                                     counters + 3, look[1], look[0], status));
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<0><<<(unsigned)T, kNT, 0, stream>>>(a, nullptr, nullptr, keys_alt, vals_alt, n, n_dev, 0,
+                                                     hist + 0 * kRadix, counters + 0, look[0], look[1], status));
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, n_dev, 8,
+                                                     hist + 1 * kRadix, counters + 1, look[1], look[0], status));
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, ka, perm, keys_alt, vals_alt, n, n_dev, 16,
+                                                     hist + 2 * kRadix, counters + 2, look[0], look[1], status));
+    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<2><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, n_dev, 24,
+                                                     hist + 3 * kRadix, counters + 3, look[1], look[0], status));
     return cudaGetLastError();
 }
 

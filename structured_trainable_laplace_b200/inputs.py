@@ -97,6 +97,17 @@ class Workload:
         return key in self.arrays
 
 
+def moved(a: np.ndarray, step: float, seed: int = 1) -> np.ndarray:
+    """The anchors after one training update: a + step * N(0, 1), rounded to fp32
+    (a stand-in for a gradient step on trainable anchors)."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 0x6d6f7665]))
+    out = np.empty_like(a, dtype=np.float32)
+    for s in range(0, a.size, _CHUNK):
+        e = min(a.size, s + _CHUNK)
+        out[s:e] = (a[s:e].astype(np.float64) + step * rng.standard_normal(e - s)).astype(np.float32)
+    return out
+
+
 def symmetric(n: int, B: int, seed: int = 0, spacing: float = 0.05, tie_frac: float = 0.0,
               with_g: bool = True, name: str = "symmetric") -> Workload:
     """a ~ U[0, spacing*n], x, g ~ N(0,1) [n][B]; optional copies to make ties."""

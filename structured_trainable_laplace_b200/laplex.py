@@ -50,6 +50,8 @@ def lib():
             "laplex_read_status": ([P, P, P], I),
             "laplex_sort_workspace_size": ([I64], SZ),
             "laplex_sort_anchors": ([P, I64, P, P, P, SZ, P, P], I),
+            "laplex_resort_workspace_size": ([I64], SZ),
+            "laplex_resort_anchors": ([P, I64, P, P, P, P, SZ, P, P, P], I),
             "laplex_workspace_size": ([I, I64, I64, I64], SZ),
             "laplex_saved_size": ([I, I64, I64, I64], SZ),
             "laplex_apply_sym": ([P, P, I64, P, I64, P, P, P, SZ, P, P], I),
@@ -75,6 +77,7 @@ def lib():
 def exported_symbols() -> list:
     """Names of the C entry points this binding calls."""
     return ["laplex_status_string", "laplex_read_status", "laplex_sort_workspace_size", "laplex_sort_anchors",
+            "laplex_resort_workspace_size", "laplex_resort_anchors",
             "laplex_workspace_size", "laplex_saved_size", "laplex_apply_sym", "laplex_apply_sym_noalloc",
             "laplex_apply_general",
             "laplex_apply_transpose", "laplex_apply_phased", "laplex_backward", "laplex_gram_apply",
@@ -178,6 +181,29 @@ def sort_anchors(a: torch.Tensor):
     ws = workspace(nb, d)
     _ok(lib().laplex_sort_anchors(_p(a), n, _p(a_sorted), _p(perm), _p(ws), ws.numel(),
                                   _p(status_word(d)), _stream(d)), "sort_anchors")
+    return a_sorted, perm
+
+
+RESORT_PATHS = {0: "sorted", 1: "repaired", 2: "full"}
+
+
+def resort_workspace_size(n: int) -> int:
+    return int(lib().laplex_resort_workspace_size(n))
+
+
+def resort_anchors(a: torch.Tensor, perm_prev: torch.Tensor, path: torch.Tensor = None):
+    """Warm-start re-sort: (a_sorted, perm), identical to sort_anchors(a), from the
+    permutation of an earlier sort.  `path` (optional int32 device tensor of one
+    element) receives 0 / 1 / 2 = already sorted / repaired / full sort."""
+    n = a.numel()
+    d = _dev(a)
+    if perm_prev.numel() != n:
+        raise ValueError("perm_prev must have as many entries as a")
+    a_sorted = torch.empty(n, dtype=torch.float32, device=a.device)
+    perm = torch.empty(n, dtype=torch.uint32, device=a.device)
+    ws = workspace(resort_workspace_size(n), d)
+    _ok(lib().laplex_resort_anchors(_p(a), n, _p(perm_prev), _p(a_sorted), _p(perm), _p(ws), ws.numel(),
+                                    _p(status_word(d)), _p(path), _stream(d)), "resort_anchors")
     return a_sorted, perm
 
 
