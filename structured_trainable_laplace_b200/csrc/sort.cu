@@ -4,7 +4,7 @@
 //
 // Keys are the order-preserving uint32 images of the anchors (-0 folded onto
 // +0), values the original indices.  Least-significant digit first, 4 passes of
-// 8 bits.  Each pass is one kernel over tiles of 4096 keys claimed in order from
+// 8 bits.  Each pass is one kernel over tiles of 3840 keys claimed in order from
 // an atomic counter: the tile ranks its keys stably inside each warp (the lanes
 // sharing a digit found by ballots over its bits), publishes its per-digit counts, looks back over the tiles
 // before it for their per-digit prefixes (bounded waits), and scatters through
@@ -18,7 +18,7 @@ namespace laplex {
 namespace {
 
 constexpr int kNT = 256;
-constexpr int kItems = 16;
+constexpr int kItems = 15;  // 3840-key tiles: with the values loaded late, four CTAs per SM
 constexpr int kTile = kNT * kItems;
 constexpr int kNW = kNT / 32;
 constexpr int kRadix = 256;
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a,
 // MODE 1: keys/values from the previous pass.  MODE 2: like 1, and the keys
 // leave as fp32 anchors (last pass).
 template <int MODE>
-__global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__ a, const uint32_t* __restrict__ keys_in,
+__global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__ a, const uint32_t* __restrict__ keys_in,
                                                     const uint32_t* __restrict__ vals_in, uint32_t* __restrict__ keys_out,
                                                     uint32_t* __restrict__ vals_out, int64_t n, const int64_t* n_dev,
                                                     int shift, const uint32_t* __restrict__ hist, uint32_t* counter,
@@ -132,22 +132,20 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
     uint32_t gtot;
     const uint32_t gexcl = block_excl_scan_256(__ldg(hist + tid), s_scan, &gtot);
 
-    uint32_t key[kItems], val[kItems], rank[kItems];
+    // keys now; the values are loaded only when they are placed (fewer live
+    // registers: four CTAs per SM)
+    uint32_t key[kItems], rank[kItems];
     const int64_t wbase = base + (int64_t)w * 32 * kItems;
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
         const int64_t idx = wbase + i * 32 + lane;
         if (idx < n) {
-            if (MODE == 0) {
+            if (MODE == 0)
                 key[i] = float_to_key(__ldg(a + idx));
-                val[i] = (uint32_t)idx;
-            } else {
+            else
                 key[i] = __ldg(keys_in + idx);
-                val[i] = __ldg(vals_in + idx);
-            }
         } else {
             key[i] = 0xffffffffu;
-            val[i] = 0u;
         }
     }
     // stable rank inside the warp, items in (i, lane) order = index order.  The
@@ -208,7 +206,7 @@ __global__ void __launch_bounds__(kNT, 3) k_radix_pass(const float* __restrict__
             const uint32_t d = (key[i] >> shift) & 0xffu;
             const uint32_t p = s_start[d] + s_whist[w][d] + rank[i];
             s_keys[p] = key[i];
-            s_vals[p] = val[i];
+            s_vals[p] = (MODE == 0) ? (uint32_t)idx : __ldg(vals_in + idx);
         }
     }
     // decoupled lookback over earlier tiles for digit tid
