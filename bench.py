@@ -54,7 +54,7 @@ def make_workload(name: str, rank: int, n: int | None = None):
     gen = {
         "sym2p24": lambda s: inputs.sym_2p24_b16(s, n=n or (1 << 24)),
         "small": lambda s: inputs.sym_small_ties(s),
-        "sym1e9": lambda s: inputs.sym_extreme(s),
+        "sym1e9": lambda s: inputs.sym_extreme(s, n=n or 10 ** 9),
         "phased_head": lambda s: inputs.phased_head_2p22(s, n=n or (1 << 22)),
         "gram_image": lambda s: inputs.gram_image(s, n=n or 3 * 1024 * 1024),
         "gram_image_full": lambda s: _full_gram(inputs.gram_image(s, n=n or 3 * 1024 * 1024)),
@@ -120,6 +120,11 @@ def kernel_bytes_per_launch(kernel: str, w) -> float | None:
             "sym_bwd": (8 + 4 * B + 4 * B + 4 * B + 4) * n,  # s, perm, sorted x, sorted g -> gx rows, ga
             "radix_pass": (12 * n + 3 * 16 * n) / 4.0,       # pass 0 reads a; passes 1-3 read+write key,value
             "radix_hist": 4 * n,
+            "sort_small": 12 * n,                            # a in; a_sorted, perm out (n <= 8192)
+            # one channel past 2^24 rows: outputs placed through destination buckets
+            # (3 vectors per step: y, gx, ga; 2 split launches and 1 placement each)
+            "unpermute_split": 16 * n,                       # (destination, value) in and out
+            "unpermute_place": 12 * n,                       # pairs in, the output window out
         }
         return table.get(kernel)
     if w.op == "phased_transpose":
@@ -379,6 +384,28 @@ def main():
     st.sort()
     ms_infer = timed(infer_step, args.steps)
 
+    # the same train step captured once as a CUDA graph and replayed: every call of
+    # the step is stream-ordered and never synchronises, so all its launches go in
+    # the graph and the host's per-launch cost leaves the timed region (one GPU:
+    # a graph holding NCCL calls is not built here)
+    graph = None
+    if world == 1:
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            for _ in range(3):
+                train_step()  # workspaces at their full size before the capture
+        stream.wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            train_step()
+        ms_graph = timed(g.replay, args.steps)
+        L.check()
+        graph = {"value": round(elements(w) / (ms_graph * 1e-3), 1), "ms_per_step": round(ms_graph, 4),
+                 "what": "the train step (sort, forward, backward) replayed as one CUDA graph"}
+        del g
+        st.sort()
+
     # the same train steps with every kernel bracketed by CUDA events
     L.profile_enable(True)
     ms_prof = timed(train_step, args.steps)
@@ -503,6 +530,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
         "roofline": roof,
         "train_warm_start": warm,
+        "train_graph": graph,
         "kernels": {kname: {"launches_per_step": v[0] / args.steps, "ms_per_step": round(v[1] / args.steps, 5)}
                     for kname, v in sorted(prof.items(), key=lambda kv: -kv[1][1])},
         "profiled_ms_per_step": round(ms_prof, 4),

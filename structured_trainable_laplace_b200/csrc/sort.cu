@@ -258,6 +258,54 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     }
 }
 
+// ---------------------------------------------------------- small n
+//
+// Up to kSmallMax anchors: one CTA sorts the composites (key << 32 | index) with a
+// bitonic network in shared memory (padded with ~0 to a power of two).  The
+// composites are distinct and ordered as the stable sort orders the anchors, so
+// the result equals the radix sort's; one launch instead of five.
+
+constexpr int kSmallMax = 8192;
+constexpr int kSmallNT = 1024;
+
+__global__ void __launch_bounds__(kSmallNT) k_sort_small(const float* __restrict__ a, int n, int m,
+                                                         float* __restrict__ a_sorted, uint32_t* __restrict__ perm,
+                                                         int32_t* status) {
+    extern __shared__ unsigned long long s_c[];  // m = the power of two >= n
+    bool bad = false;
+    for (int i = threadIdx.x; i < m; i += kSmallNT) {
+        unsigned long long c = ~0ull;
+        if (i < n) {
+            const float f = __ldg(a + i);
+            bad |= is_nonfinite(f);
+            c = ((unsigned long long)float_to_key(f) << 32) | (unsigned)i;
+        }
+        s_c[i] = c;
+    }
+    if (bad) raise_status(status, kStatusNonFinite);
+    __syncthreads();
+    // pair q of a stage with distance j: lo = (q / j) * 2j + q % j, hi = lo + j;
+    // ascending where bit k of lo is clear
+    for (int k = 2; k <= m; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int q = threadIdx.x; q < (m >> 1); q += kSmallNT) {
+                const int lo = ((q & ~(j - 1)) << 1) | (q & (j - 1)), hi = lo + j;
+                const unsigned long long x = s_c[lo], y = s_c[hi];
+                if ((x > y) == ((lo & k) == 0)) {
+                    s_c[lo] = y;
+                    s_c[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = threadIdx.x; i < n; i += kSmallNT) {
+        const unsigned long long c = s_c[i];
+        a_sorted[i] = key_to_float((uint32_t)(c >> 32));
+        perm[i] = (uint32_t)c;
+    }
+}
+
 // ---------------------------------------------------------- unpermute
 //
 // out[perm[r]] = v[r] for vectors whose rows are single floats and too large for
@@ -437,6 +485,21 @@ size_t sort_workspace_bytes(int64_t n) {
 
 cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
                         cudaStream_t stream, const int64_t* n_dev) {
+    if (n_dev == nullptr && n <= kSmallMax) {
+        int m = 1;
+        while (m < n) m <<= 1;
+        static bool ready = false;
+        if (!ready) {
+            const cudaError_t e = cudaFuncSetAttribute(k_sort_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)(sizeof(unsigned long long) * kSmallMax));
+            if (e != cudaSuccess) return e;
+            ready = true;
+        }
+        LAPLEX_TIMED("sort_small", stream,
+                     k_sort_small<<<1, kSmallNT, sizeof(unsigned long long) * m, stream>>>(a, (int)n, m, a_sorted,
+                                                                                             perm, status));
+        return cudaGetLastError();
+    }
     const int64_t T = (n + kTile - 1) / kTile;
     char* p = (char*)ws;
     uint32_t* keys_alt = (uint32_t*)p;

@@ -46,6 +46,18 @@ def test_all_equal(L):
     check_sort(L, np.full(9000, 3.25, np.float32))
 
 
+# up to 8192 anchors one CTA sorts the (key, index) composites in shared memory
+@pytest.mark.parametrize("n", [5, 1000, 4096, 8191, 8192, 8193])
+def test_single_cta_range_and_its_boundary(L, n):
+    rng = np.random.default_rng(100 + n)
+    a = rng.integers(-20, 20, n).astype(np.float32) * 0.5
+    a[rng.random(n) < 0.1] = -0.0
+    a[rng.random(n) < 0.05] = 0.0
+    check_sort(L, a)
+    check_sort(L, np.full(n, -7.5, np.float32))
+    check_sort(L, np.linspace(1, -1, n).astype(np.float32))
+
+
 def test_full_size_sort_of_the_2p24_workload(L):
     check_sort(L, inputs.sym_2p24_b16(0)["a"])
 
