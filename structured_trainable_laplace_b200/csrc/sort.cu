@@ -260,49 +260,35 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
 
 // ---------------------------------------------------------- small n
 //
-// Up to kSmallMax anchors: one CTA sorts the composites (key << 32 | index) with a
-// bitonic network in shared memory (padded with ~0 to a power of two).  The
-// composites are distinct and ordered as the stable sort orders the anchors, so
-// the result equals the radix sort's; one launch instead of five.
+// Up to kSmallMax anchors: rank by counting.  The composites c_i = (key_i << 32 | i)
+// are distinct and ordered as the stable sort orders the anchors, so the position
+// of anchor i is the number of composites below c_i.  Each CTA holds all n
+// composites in shared memory and ranks kRankPer of them (four threads per
+// anchor, each counting over every fourth composite: consecutive words, no bank
+// conflicts), then writes those anchors to their positions.  One launch of
+// ceil(n / kRankPer) CTAs instead of five; the result equals the radix sort's.
 
 constexpr int kSmallMax = 8192;
-constexpr int kSmallNT = 1024;
+constexpr int kRankPer = 64;
+constexpr int kRankNT = 4 * kRankPer;
 
-__global__ void __launch_bounds__(kSmallNT) k_sort_small(const float* __restrict__ a, int n, int m,
-                                                         float* __restrict__ a_sorted, uint32_t* __restrict__ perm,
-                                                         int32_t* status) {
-    extern __shared__ unsigned long long s_c[];  // m = the power of two >= n
-    bool bad = false;
-    for (int i = threadIdx.x; i < m; i += kSmallNT) {
-        unsigned long long c = ~0ull;
-        if (i < n) {
-            const float f = __ldg(a + i);
-            bad |= is_nonfinite(f);
-            c = ((unsigned long long)float_to_key(f) << 32) | (unsigned)i;
-        }
-        s_c[i] = c;
-    }
-    if (bad) raise_status(status, kStatusNonFinite);
+__global__ void __launch_bounds__(kRankNT) k_sort_small(const float* __restrict__ a, int n,
+                                                        float* __restrict__ a_sorted, uint32_t* __restrict__ perm,
+                                                        int32_t* status) {
+    extern __shared__ unsigned long long s_c[];  // n composites
+    for (int i = threadIdx.x; i < n; i += kRankNT)
+        s_c[i] = ((unsigned long long)float_to_key(__ldg(a + i)) << 32) | (unsigned)i;
     __syncthreads();
-    // pair q of a stage with distance j: lo = (q / j) * 2j + q % j, hi = lo + j;
-    // ascending where bit k of lo is clear
-    for (int k = 2; k <= m; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int q = threadIdx.x; q < (m >> 1); q += kSmallNT) {
-                const int lo = ((q & ~(j - 1)) << 1) | (q & (j - 1)), hi = lo + j;
-                const unsigned long long x = s_c[lo], y = s_c[hi];
-                if ((x > y) == ((lo & k) == 0)) {
-                    s_c[lo] = y;
-                    s_c[hi] = x;
-                }
-            }
-            __syncthreads();
-        }
-    }
-    for (int i = threadIdx.x; i < n; i += kSmallNT) {
-        const unsigned long long c = s_c[i];
-        a_sorted[i] = key_to_float((uint32_t)(c >> 32));
-        perm[i] = (uint32_t)c;
+    const int el = blockIdx.x * kRankPer + (threadIdx.x >> 2), part = threadIdx.x & 3;
+    const unsigned long long mine = el < n ? s_c[el] : 0ull;
+    int below = 0;
+    for (int q = part; q < n; q += 4) below += s_c[q] < mine;
+    below += __shfl_xor_sync(0xffffffffu, below, 1);
+    below += __shfl_xor_sync(0xffffffffu, below, 2);
+    if (part == 0 && el < n) {
+        if (is_nonfinite(__ldg(a + el))) raise_status(status, kStatusNonFinite);
+        a_sorted[below] = key_to_float((uint32_t)(mine >> 32));
+        perm[below] = (uint32_t)mine;
     }
 }
 
@@ -486,8 +472,6 @@ size_t sort_workspace_bytes(int64_t n) {
 cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
                         cudaStream_t stream, const int64_t* n_dev) {
     if (n_dev == nullptr && n <= kSmallMax) {
-        int m = 1;
-        while (m < n) m <<= 1;
         static bool ready = false;
         if (!ready) {
             const cudaError_t e = cudaFuncSetAttribute(k_sort_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -496,8 +480,8 @@ cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* pe
             ready = true;
         }
         LAPLEX_TIMED("sort_small", stream,
-                     k_sort_small<<<1, kSmallNT, sizeof(unsigned long long) * m, stream>>>(a, (int)n, m, a_sorted,
-                                                                                             perm, status));
+                     k_sort_small<<<(unsigned)((n + kRankPer - 1) / kRankPer), kRankNT,
+                                    sizeof(unsigned long long) * n, stream>>>(a, (int)n, a_sorted, perm, status));
         return cudaGetLastError();
     }
     const int64_t T = (n + kTile - 1) / kTile;
