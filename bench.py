@@ -225,20 +225,32 @@ def summarize_clocks(path: str, gpu_index: int) -> dict:
             "samples": len(sm)}
 
 
-def source_hash() -> str:
+# the source file that defines each timed kernel (its launches are named by these prefixes)
+KERNEL_SOURCE = (("sym_", "sym.cu"), ("radix_", "sort.cu"), ("sort_small", "sort.cu"), ("unpermute_", "sort.cu"),
+                 ("resort_", "resort.cu"), ("large_", "rect.cu"), ("side_", "rect.cu"), ("finish", "rect.cu"),
+                 ("gram_", "rect.cu"))
+
+
+def source_hash(kernel: str) -> str:
+    """Hash of the kernel's own .cu file and every shared header it can include."""
+    csrc = os.path.join(ROOT, "structured_trainable_laplace_b200", "csrc")
+    own = next((f for pre, f in KERNEL_SOURCE if kernel.startswith(pre)), None)
+    files = sorted(glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.h")) +
+                   glob.glob(os.path.join(ROOT, "include", "*.h")))
+    files += [os.path.join(csrc, own)] if own else sorted(glob.glob(os.path.join(csrc, "*.cu")))
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "structured_trainable_laplace_b200", "csrc", "*"))):
+    for p in files:
         h.update(open(p, "rb").read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel sources (a line `traffic <kernel> <workload> <bytes> <source hash>`)."""
+    current sources of that kernel (a line `traffic <kernel> <workload> <bytes> <hash>`)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    cur = source_hash()
+    cur = source_hash(kernel)
     for line in open(path):
         f = line.split()
         if len(f) == 5 and f[0] == "traffic" and f[1] == kernel and f[2] == workload and f[4] == cur:

@@ -374,14 +374,30 @@ __global__ void k_bucket_cursors(uint32_t* cursor, int64_t count, int shift) {
 __global__ void __launch_bounds__(kNT) k_place_window(const uint32_t* __restrict__ p, const float* __restrict__ v,
                                                       int64_t n, int shift, float* __restrict__ out) {
     extern __shared__ float s_win[];
+    constexpr int U = 8;  // pairs in flight per thread
     const int64_t w0 = (int64_t)blockIdx.x << shift;
     const int cnt = (int)min((int64_t)1 << shift, n - w0);
-    for (int i = threadIdx.x; i < cnt; i += kNT) {
-        const int64_t d = (int64_t)__ldcs(p + w0 + i) - w0;
-        if (d >= 0 && d < cnt) s_win[d] = __ldcs(v + w0 + i);
+    for (int i0 = threadIdx.x; i0 < cnt; i0 += kNT * U) {
+        uint32_t pp[U];
+        float vv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * kNT;
+            pp[u] = i < cnt ? __ldcs(p + w0 + i) : 0xffffffffu;
+            vv[u] = i < cnt ? __ldcs(v + w0 + i) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t d = (int64_t)pp[u] - w0;
+            if (i0 + u * kNT < cnt && d >= 0 && d < cnt) s_win[d] = vv[u];
+        }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < cnt; i += kNT) __stcs(out + w0 + i, s_win[i]);
+    // windows start at multiples of 2^shift >= 512 floats: 16-byte aligned
+    float4* o4 = reinterpret_cast<float4*>(out + w0);
+    const float4* w4 = reinterpret_cast<const float4*>(s_win);
+    for (int i = threadIdx.x; i < cnt / 4; i += kNT) __stcs(o4 + i, w4[i]);
+    for (int i = (cnt / 4) * 4 + threadIdx.x; i < cnt; i += kNT) __stcs(out + w0 + i, s_win[i]);
 }
 
 // out[p[i]] = v[i], i in order, for windows too large for shared memory.

@@ -820,6 +820,9 @@ struct Rows1 {
     int64_t row0;
 };
 
+// WITH_PERM false: the permutation entries are not needed (outputs in sorted
+// order) and are not read.
+template <bool WITH_PERM = true>
 __device__ __forceinline__ void load_rows1(const float* __restrict__ s, const uint32_t* __restrict__ perm, int64_t n,
                                            int64_t row0, Rows1& r) {
     r.row0 = row0;
@@ -828,17 +831,21 @@ __device__ __forceinline__ void load_rows1(const float* __restrict__ s, const ui
 #pragma unroll
         for (int q = 0; q < k1E / 4; ++q) {
             const float4 av = __ldg(reinterpret_cast<const float4*>(s + row0) + q);
-            const uint4 pv = __ldg(reinterpret_cast<const uint4*>(perm + row0) + q);
             r.a[4 * q] = av.x, r.a[4 * q + 1] = av.y, r.a[4 * q + 2] = av.z, r.a[4 * q + 3] = av.w;
-            r.p[4 * q] = min(pv.x, last), r.p[4 * q + 1] = min(pv.y, last);
-            r.p[4 * q + 2] = min(pv.z, last), r.p[4 * q + 3] = min(pv.w, last);
+            if (WITH_PERM) {
+                const uint4 pv = __ldg(reinterpret_cast<const uint4*>(perm + row0) + q);
+                r.p[4 * q] = min(pv.x, last), r.p[4 * q + 1] = min(pv.y, last);
+                r.p[4 * q + 2] = min(pv.z, last), r.p[4 * q + 3] = min(pv.w, last);
+            } else {
+                r.p[4 * q] = r.p[4 * q + 1] = r.p[4 * q + 2] = r.p[4 * q + 3] = 0u;
+            }
         }
     } else {
 #pragma unroll
         for (int e = 0; e < k1E; ++e) {
             const bool in = row0 + e < n;
             r.a[e] = in ? __ldg(s + row0 + e) : kHighAnchor;
-            r.p[e] = in ? min(__ldg(perm + row0 + e), last) : 0u;
+            r.p[e] = (in && WITH_PERM) ? min(__ldg(perm + row0 + e), last) : 0u;
         }
     }
     r.ap = (row0 == 0) ? kLowAnchor : (row0 - 1 < n ? __ldg(s + row0 - 1) : kHighAnchor);
@@ -1000,11 +1007,12 @@ __device__ __forceinline__ void put_rows1(float* __restrict__ dst, const float (
 
 // Sweep for one channel: NV = 1 forward (xs -> y), NV = 2 backward (xs, gs -> gx,
 // ga), from the sorted copies, RS and the range carries (as k_sym_sweep).
-template <int NV>
+// SORTED: the outputs are written in sorted order (for launch_unpermute) and the
+// permutation is not read.
+template <int NV, bool SORTED>
 __global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a, const float* __restrict__ xs,
                                                        const float* __restrict__ gs, RangeState sx, RangeState sg,
-                                                       float* __restrict__ out, float* __restrict__ ga,
-                                                       int sorted_out) {
+                                                       float* __restrict__ out, float* __restrict__ ga) {
     __shared__ Cross1<NV> cx;
     __shared__ double2 s_runL[NV];
     const CtaTiles cw = cta_tiles(a);
@@ -1019,7 +1027,7 @@ __global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a,
         const int64_t lo = t * (int64_t)k1R, J = t / a.tpr;
         const bool more = (t + 1 < min(a.T, (J + 1) * a.tpr)), hasRin = (J + 1 < a.P);
         Rows1 r;
-        load_rows1(a.s, a.perm, a.n, lo + threadIdx.x * k1E, r);
+        load_rows1<!SORTED>(a.s, a.perm, a.n, lo + threadIdx.x * k1E, r);
         float xv[NV][k1E];
 #pragma unroll
         for (int vv = 0; vv < NV; ++vv) {
@@ -1128,7 +1136,7 @@ __global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a,
                 pl = fmaf(fabsf(d[e]), pl, xv[0][e]);
                 yv[e] += pl;
             }
-            put_rows1(out, yv, r, a.n, sorted_out);
+            put_rows1(out, yv, r, a.n, SORTED);
         } else {
             LP ax = inR[0], ag = inR[NV - 1];
             float gxr[k1E], gap[k1E];
@@ -1150,8 +1158,8 @@ __global__ void __launch_bounds__(k1NT, NV == 1 ? 3 : 2) k_sym1_sweep(SymScan a,
                 gxr[e] += ag.P;
                 gap[e] = fmaf(-ge, ax.L, fmaf(-xe, ag.L, gap[e]));
             }
-            if (out != nullptr) put_rows1(out, gxr, r, a.n, sorted_out);
-            if (ga != nullptr) put_rows1(ga, gap, r, a.n, sorted_out);
+            if (out != nullptr) put_rows1(out, gxr, r, a.n, SORTED);
+            if (ga != nullptr) put_rows1(ga, gap, r, a.n, SORTED);
         }
         if (threadIdx.x == 0) {
             const float fl = (lo + k1R <= a.n) ? __ldg(a.s + lo + k1R - 1) : kHighAnchor;
@@ -1302,15 +1310,19 @@ cudaError_t launch_sym_sweep_fwd(const SymPlan& p, const float* s, const uint32_
                                  const float* xs, const RangeState& sx, float* y, cudaStream_t st,
                                  void* ws = nullptr) {
     if constexpr (C == 1) {
-        static int occ_cache = 0;
-        const int occ = prepare(k_sym1_sweep<1>, k1NT, 0, occ_cache);
+        static int occ_cache[2] = {0, 0};
+        const bool bucketed = p.bucketed && ws != nullptr;
+        const int occ = bucketed ? prepare(k_sym1_sweep<1, true>, k1NT, 0, occ_cache[1])
+                                 : prepare(k_sym1_sweep<1, false>, k1NT, 0, occ_cache[0]);
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
-        const bool bucketed = p.bucketed && ws != nullptr;
-        float* ys = bucketed ? unperm_outputs(p, ws) : y;
-        LAPLEX_TIMED("sym_fwd", st,
-                     k_sym1_sweep<1><<<grid, k1NT, 0, st>>>(a, xs, nullptr, sx, sx, ys, nullptr, bucketed ? 1 : 0));
-        if (bucketed) return launch_unpermute(perm, ys, n, y, unperm_scratch(p, ws, n), st);
+        if (bucketed) {
+            float* ys = unperm_outputs(p, ws);
+            LAPLEX_TIMED("sym_fwd", st,
+                         k_sym1_sweep<1, true><<<grid, k1NT, 0, st>>>(a, xs, nullptr, sx, sx, ys, nullptr));
+            return launch_unpermute(perm, ys, n, y, unperm_scratch(p, ws, n), st);
+        }
+        LAPLEX_TIMED("sym_fwd", st, k_sym1_sweep<1, false><<<grid, k1NT, 0, st>>>(a, xs, nullptr, sx, sx, y, nullptr));
     } else {
         using SM = SweepSmem<C, 1, kAheadFwd>;
         static int occ_cache = 0;
@@ -1371,14 +1383,17 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
     e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, gs, st);
     if (e != cudaSuccess) return e;
     if constexpr (C == 1) {
-        static int occ_cache = 0;
-        const int occ = prepare(k_sym1_sweep<2>, k1NT, 0, occ_cache);
+        static int occ_cache[2] = {0, 0};
+        const int occ = p.bucketed ? prepare(k_sym1_sweep<2, true>, k1NT, 0, occ_cache[1])
+                                   : prepare(k_sym1_sweep<2, false>, k1NT, 0, occ_cache[0]);
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
         float* gxs = p.bucketed && gx ? unperm_outputs(p, ws) : gx;
         float* gas = p.bucketed && ga ? unperm_outputs(p, ws) + align_up((size_t)n, 64) : ga;
-        LAPLEX_TIMED("sym_bwd", st,
-                     k_sym1_sweep<2><<<grid, k1NT, 0, st>>>(a, xs, gs, sx, sg, gxs, gas, p.bucketed ? 1 : 0));
+        if (p.bucketed)
+            LAPLEX_TIMED("sym_bwd", st, k_sym1_sweep<2, true><<<grid, k1NT, 0, st>>>(a, xs, gs, sx, sg, gxs, gas));
+        else
+            LAPLEX_TIMED("sym_bwd", st, k_sym1_sweep<2, false><<<grid, k1NT, 0, st>>>(a, xs, gs, sx, sg, gxs, gas));
         if (p.bucketed) {
             void* scratch = unperm_scratch(p, ws, n);
             if (gx) LAPLEX_TRY_SYM(launch_unpermute(perm, gxs, n, gx, scratch, st));
