@@ -13,6 +13,23 @@ namespace laplex {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// A value cached once per device (kernel attributes and occupancies belong to a
+// device, and one process may drive several).  Devices past kMaxDevices get no
+// cache: here() returns a fresh zero each time, so the setup simply reruns.
+struct PerDevice {
+    static constexpr int kMaxDevices = 64;
+    int v[kMaxDevices] = {};
+    int& here() {
+        int d = 0;
+        if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) {
+            static thread_local int none;
+            none = 0;
+            return none;
+        }
+        return v[d];
+    }
+};
+
 // profile.cu: optional CUDA-event bracket around each kernel launch.
 bool profiling();
 void* profile_begin(const char* name, cudaStream_t stream);

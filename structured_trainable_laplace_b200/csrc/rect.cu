@@ -915,17 +915,19 @@ template <int VEC, bool PHASED, int MODE>
 cudaError_t launch_large(LargePass A, int chunks, const char* name, cudaStream_t st) {
     const bool wide = A.lpr >= kLargeBatch<VEC, PHASED, MODE>;
     const size_t smem = large_smem_bytes<VEC, PHASED, MODE>(wide);
-    static int occ[2] = {0, 0};
-    if (occ[wide] == 0) {
+    static PerDevice occ_dev[2];
+    int& occ_w = occ_dev[wide].here();
+    if (occ_w == 0) {
         int o = 1;
         cudaFuncSetAttribute(k_large<VEC, PHASED, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)large_smem_bytes<VEC, PHASED, MODE>(true));
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large<VEC, PHASED, MODE>, 256, smem) != cudaSuccess)
             o = 1;
-        occ[wide] = std::max(o, 1);
+        occ_w = std::max(o, 1);
     }
+    const int occ_here = occ_w;
     const int64_t groups_per_block = 8 * (32 / A.lpr);
-    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ[wide] / chunks);
+    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ_here / chunks);
     const int64_t need = (A.m + groups_per_block * kLargeMinRows - 1) / (groups_per_block * kLargeMinRows);
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
     A.rows_per_group = (A.m + blocks * groups_per_block - 1) / (blocks * groups_per_block);

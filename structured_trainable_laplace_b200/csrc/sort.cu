@@ -313,7 +313,7 @@ constexpr int kPlaceMaxWindow = 1 << 14;  // floats of a window placed in shared
 // second pass's tiles lie inside one first-pass bucket).  Per-bucket counts
 // (shared atomics), a block scan into per-bucket starts, one global cursor claim
 // per bucket, then runs of equal buckets leave as contiguous stores.
-__global__ void __launch_bounds__(kNT) k_bucket_split(const uint32_t* __restrict__ p_in, const float* __restrict__ v_in,
+__global__ void __launch_bounds__(kNT, 4) k_bucket_split(const uint32_t* __restrict__ p_in, const float* __restrict__ v_in,
                                                       int64_t n, int shift, uint32_t* cursor, uint32_t* __restrict__ p_out,
                                                       float* __restrict__ v_out) {
     __shared__ uint32_t s_cnt[kRadix], s_start[kRadix], s_base[kRadix], s_scan[kNW];
@@ -326,12 +326,30 @@ __global__ void __launch_bounds__(kNT) k_bucket_split(const uint32_t* __restrict
     const uint32_t last = (uint32_t)(n - 1);
     uint32_t pv[kSplitItems], rk[kSplitItems];
     float vv[kSplitItems];
+    // item i of thread tid: position base + (i / 4) * 4 * kNT + 4 * tid + i % 4 (the
+    // order inside a bucket is free), loaded 16 bytes at a time in full tiles
+    const bool full = base + kSplitTile <= n;
+#pragma unroll
+    for (int q = 0; q < kSplitItems / 4; ++q) {
+        const int64_t idx0 = base + (int64_t)q * 4 * kNT + 4 * tid;
+        if (full) {
+            const uint4 p4 = __ldcs(reinterpret_cast<const uint4*>(p_in + idx0));
+            const float4 v4 = __ldcs(reinterpret_cast<const float4*>(v_in + idx0));
+            pv[4 * q] = p4.x, pv[4 * q + 1] = p4.y, pv[4 * q + 2] = p4.z, pv[4 * q + 3] = p4.w;
+            vv[4 * q] = v4.x, vv[4 * q + 1] = v4.y, vv[4 * q + 2] = v4.z, vv[4 * q + 3] = v4.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                pv[4 * q + u] = idx0 + u < n ? __ldcs(p_in + idx0 + u) : 0u;
+                vv[4 * q + u] = idx0 + u < n ? __ldcs(v_in + idx0 + u) : 0.f;
+            }
+        }
+    }
 #pragma unroll
     for (int i = 0; i < kSplitItems; ++i) {
-        const int64_t idx = base + i * kNT + tid;
+        const int64_t idx = base + (int64_t)(i / 4) * 4 * kNT + 4 * tid + (i % 4);
         if (idx < n) {
-            pv[i] = min(__ldcs(p_in + idx), last);
-            vv[i] = __ldcs(v_in + idx);
+            pv[i] = min(pv[i], last);
             rk[i] = atomicAdd(&s_cnt[(pv[i] >> shift) & 0xffu], 1u);
         }
     }
@@ -344,7 +362,7 @@ __global__ void __launch_bounds__(kNT) k_bucket_split(const uint32_t* __restrict
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < kSplitItems; ++i) {
-        const int64_t idx = base + i * kNT + tid;
+        const int64_t idx = base + (int64_t)(i / 4) * 4 * kNT + 4 * tid + (i % 4);
         if (idx < n) {
             const uint32_t q = s_start[(pv[i] >> shift) & 0xffu] + rk[i];
             s_p[q] = pv[i];
@@ -460,12 +478,12 @@ cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* o
     LAPLEX_TIMED("unpermute_split", stream,
                  k_bucket_split<<<(unsigned)tiles, kNT, 0, stream>>>(p1, v1, n, s2, cursor, p2, v2));
     if ((1ll << s2) <= kPlaceMaxWindow) {
-        static bool ready = false;
-        if (!ready) {
+        static PerDevice ready;
+        if (!ready.here()) {
             const cudaError_t e = cudaFuncSetAttribute(k_place_window, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        (int)(sizeof(float) * kPlaceMaxWindow));
             if (e != cudaSuccess) return e;
-            ready = true;
+            ready.here() = 1;
         }
         LAPLEX_TIMED("unpermute_place", stream,
                      k_place_window<<<(unsigned)nb2, kNT, sizeof(float) << s2, stream>>>(p2, v2, n, s2, out));
@@ -488,12 +506,12 @@ size_t sort_workspace_bytes(int64_t n) {
 cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
                         cudaStream_t stream, const int64_t* n_dev) {
     if (n_dev == nullptr && n <= kSmallMax) {
-        static bool ready = false;
-        if (!ready) {
+        static PerDevice ready;
+        if (!ready.here()) {
             const cudaError_t e = cudaFuncSetAttribute(k_sort_small, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        (int)(sizeof(unsigned long long) * kSmallMax));
             if (e != cudaSuccess) return e;
-            ready = true;
+            ready.here() = 1;
         }
         LAPLEX_TIMED("sort_small", stream,
                      k_sort_small<<<(unsigned)((n + kRankPer - 1) / kRankPer), kRankNT,

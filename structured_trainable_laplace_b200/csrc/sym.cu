@@ -1240,7 +1240,7 @@ int device_sms() {
 }
 
 // Opt a kernel into its dynamic shared memory and return its resident CTAs per SM
-// (cached: one device type per process).
+// (cached per device).
 template <class F>
 int prepare(F* f, int threads, size_t smem, int& cached) {
     if (cached > 0) return cached;
@@ -1272,15 +1272,15 @@ template <int C>
 cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms,
                          const float* v, RangeState st, float* vs, cudaStream_t stream) {
     if constexpr (C == 1) {
-        static int occ_cache = 0;
-        const int occ = prepare(k_sym1_agg, k1NT, 0, occ_cache);
+        static PerDevice occ_cache;
+        const int occ = prepare(k_sym1_agg, k1NT, 0, occ_cache.here());
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
         LAPLEX_TIMED("sym_agg", stream, k_sym1_agg<<<grid, k1NT, 0, stream>>>(a, v, st, vs));
     } else {
         using SM = AggSmem<C, kAheadAgg>;
-        static int occ_cache = 0;
-        const int occ = prepare(k_sym_agg<C, kAheadAgg>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+        static PerDevice occ_cache;
+        const int occ = prepare(k_sym_agg<C, kAheadAgg>, SymGeo<C>::NT, sizeof(SM), occ_cache.here());
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
         LAPLEX_TIMED("sym_agg", stream,
@@ -1288,11 +1288,11 @@ cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm,
     }
     const SymScan a = scan_args(p, s, perm, n, B, sms, 1);
     const size_t dsm = sizeof(double) * 2 * (size_t)p.P;
-    static int carry_ready = 0;
-    if (!carry_ready) {
+    static PerDevice carry_ready;
+    if (!carry_ready.here()) {
         cudaFuncSetAttribute(k_sym_carry<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)(sizeof(double) * 2 * kMaxRanges));
-        carry_ready = 1;
+        carry_ready.here() = 1;
     }
     LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, kCarryThreads, dsm, stream>>>(a, st));
     return cudaGetLastError();
@@ -1310,10 +1310,10 @@ cudaError_t launch_sym_sweep_fwd(const SymPlan& p, const float* s, const uint32_
                                  const float* xs, const RangeState& sx, float* y, cudaStream_t st,
                                  void* ws = nullptr) {
     if constexpr (C == 1) {
-        static int occ_cache[2] = {0, 0};
+        static PerDevice occ_cache[2];
         const bool bucketed = p.bucketed && ws != nullptr;
-        const int occ = bucketed ? prepare(k_sym1_sweep<1, true>, k1NT, 0, occ_cache[1])
-                                 : prepare(k_sym1_sweep<1, false>, k1NT, 0, occ_cache[0]);
+        const int occ = bucketed ? prepare(k_sym1_sweep<1, true>, k1NT, 0, occ_cache[1].here())
+                                 : prepare(k_sym1_sweep<1, false>, k1NT, 0, occ_cache[0].here());
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
         if (bucketed) {
@@ -1325,8 +1325,8 @@ cudaError_t launch_sym_sweep_fwd(const SymPlan& p, const float* s, const uint32_
         LAPLEX_TIMED("sym_fwd", st, k_sym1_sweep<1, false><<<grid, k1NT, 0, st>>>(a, xs, nullptr, sx, sx, y, nullptr));
     } else {
         using SM = SweepSmem<C, 1, kAheadFwd>;
-        static int occ_cache = 0;
-        const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+        static PerDevice occ_cache;
+        const int occ = prepare(k_sym_sweep<C, 1, kAheadFwd>, SymGeo<C>::NT, sizeof(SM), occ_cache.here());
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
         LAPLEX_TIMED("sym_fwd", st,
@@ -1383,9 +1383,9 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
     e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, gs, st);
     if (e != cudaSuccess) return e;
     if constexpr (C == 1) {
-        static int occ_cache[2] = {0, 0};
-        const int occ = p.bucketed ? prepare(k_sym1_sweep<2, true>, k1NT, 0, occ_cache[1])
-                                   : prepare(k_sym1_sweep<2, false>, k1NT, 0, occ_cache[0]);
+        static PerDevice occ_cache[2];
+        const int occ = p.bucketed ? prepare(k_sym1_sweep<2, true>, k1NT, 0, occ_cache[1].here())
+                                   : prepare(k_sym1_sweep<2, false>, k1NT, 0, occ_cache[0].here());
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
         float* gxs = p.bucketed && gx ? unperm_outputs(p, ws) : gx;
@@ -1401,8 +1401,8 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
         }
     } else {
         using SM = SweepSmem<C, 2, kAheadBwd>;
-        static int occ_cache = 0;
-        const int occ = prepare(k_sym_sweep<C, 2, kAheadBwd>, SymGeo<C>::NT, sizeof(SM), occ_cache);
+        static PerDevice occ_cache;
+        const int occ = prepare(k_sym_sweep<C, 2, kAheadBwd>, SymGeo<C>::NT, sizeof(SM), occ_cache.here());
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), (unsigned)p.G);
         LAPLEX_TIMED("sym_bwd", st,

@@ -95,11 +95,13 @@ def _dev(t: torch.Tensor) -> int:
 
 
 def workspace(nbytes: int, device: int) -> torch.Tensor:
-    """A grow-only scratch buffer per device (stream-ordered reuse)."""
-    buf = _ws.get(device)
+    """A grow-only scratch buffer per (device, current stream): the calls of one
+    stream reuse it in stream order, calls on different streams never share it."""
+    key = (device, torch.cuda.current_stream(device).cuda_stream)
+    buf = _ws.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=f"cuda:{device}")
-        _ws[device] = buf
+        _ws[key] = buf
     return buf
 
 

@@ -1,7 +1,8 @@
-"""Every entry point is stream-ordered and never synchronises, so a whole training
-step (sort, forward, backward) can be captured once as a CUDA graph and replayed
-on new inputs copied into the captured input buffers.  The replays must match the
-fp64 oracle on those new inputs like the eager calls do."""
+"""Stream use of the binding.  Every entry point is stream-ordered and never
+synchronises, so a whole training step (sort, forward, backward) can be captured
+once as a CUDA graph and replayed on new inputs copied into the captured input
+buffers; the replays must match the fp64 oracle on those new inputs like the eager
+calls do.  Calls on two streams at once use separate scratch and must each match."""
 import numpy as np
 import pytest
 
@@ -92,3 +93,31 @@ def test_phased_head_train_step_replays(L):
     for key in ("gx", "ga", "gb", "gphi", "gpsi"):
         assert_close(host(gr[key]).reshape(np.shape(ref[key])), ref[key], tw[key], key)
     del g
+
+
+def test_two_streams_run_concurrently(L):
+    # each stream gets its own scratch: interleaved calls on two streams must each
+    # match the oracle
+    import torch
+    ws = [inputs.symmetric(200_003, 4, seed=51), inputs.symmetric(150_001, 8, seed=52)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    dv = [{k: dev(v) for k, v in w.arrays.items()} for w in ws]
+    torch.cuda.synchronize()
+    outs = [None, None]
+    for rep in range(3):
+        for i in (0, 1):
+            with torch.cuda.stream(streams[i]):
+                s, p = L.sort_anchors(dv[i]["a"])
+                y = L.apply_sym(s, p, dv[i]["x"])
+                gr = L.backward("sym", s, p, dv[i]["x"], dv[i]["g"], need=("gx", "ga"))
+                outs[i] = (y, gr["gx"], gr["ga"])
+    torch.cuda.synchronize()
+    L.check()
+    for i, w in enumerate(ws):
+        a, x, g = w["a"], w["x"], w["g"]
+        y, gx, ga = outs[i]
+        assert_close(host(y), oracle.sym_apply(a, x), oracle.sym_apply(a, x, twin=True), f"y{i}")
+        gx_ref, ga_ref = oracle.sym_backward(a, x, g)
+        gx_tw, ga_tw = oracle.sym_backward(a, x, g, twin=True)
+        assert_close(host(gx), gx_ref, gx_tw, f"gx{i}")
+        assert_close(host(ga), ga_ref, ga_tw, f"ga{i}")
