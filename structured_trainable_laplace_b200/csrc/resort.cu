@@ -170,30 +170,49 @@ __global__ void __launch_bounds__(kNT) k_resort_gather(const float* __restrict__
     __shared__ uint64_t s_max[kNT / 32], s_min[kNT / 32];
     const int64_t base = (int64_t)blockIdx.x * kTile;
     const uint32_t last = (uint32_t)(n - 1);
+    // item i of thread t: position base + (i / 4) * 4 * kNT + 4 t + i % 4, moved 16
+    // bytes at a time in full tiles (the tile's max and min do not depend on order)
+    const bool full = base + kTile <= n;
+    auto pos = [&](int i) { return base + (int64_t)(i / 4) * 4 * kNT + 4 * threadIdx.x + (i % 4); };
     uint32_t idx[kItems];
     float f[kItems];
 #pragma unroll
-    for (int i = 0; i < kItems; ++i) {
-        const int64_t r = base + i * kNT + threadIdx.x;
-        idx[i] = r < n ? min(__ldcs(perm_prev + r), last) : 0u;
+    for (int q = 0; q < kItems / 4; ++q) {
+        if (full) {
+            const uint4 p4 = __ldcs(reinterpret_cast<const uint4*>(perm_prev + pos(4 * q)));
+            idx[4 * q] = p4.x, idx[4 * q + 1] = p4.y, idx[4 * q + 2] = p4.z, idx[4 * q + 3] = p4.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) idx[4 * q + u] = pos(4 * q + u) < n ? __ldcs(perm_prev + pos(4 * q + u)) : 0u;
+        }
     }
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
-        const int64_t r = base + i * kNT + threadIdx.x;
-        f[i] = r < n ? __ldg(a + idx[i]) : 0.f;
+        idx[i] = min(idx[i], last);
+        f[i] = pos(i) < n ? __ldg(a + idx[i]) : 0.f;
     }
     uint64_t mx = 0, mn = ~0ull;
     bool bad = false;
+    uint32_t k[kItems];
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
-        const int64_t r = base + i * kNT + threadIdx.x;
-        if (r < n) {
+        k[i] = float_to_key(f[i]);
+        if (pos(i) < n) {
             bad |= is_nonfinite(f[i]);
-            const uint32_t k = float_to_key(f[i]);
-            __stcs(w.keys + r, k);
-            const uint64_t c = comp(k, idx[i]);
+            const uint64_t c = comp(k[i], idx[i]);
             mx = max(mx, c);
             mn = min(mn, c);
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < kItems / 4; ++q) {
+        if (full) {
+            __stcs(reinterpret_cast<uint4*>(w.keys + pos(4 * q)),
+                   make_uint4(k[4 * q], k[4 * q + 1], k[4 * q + 2], k[4 * q + 3]));
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (pos(4 * q + u) < n) w.keys[pos(4 * q + u)] = k[4 * q + u];
         }
     }
     if (bad) raise_status(status, kStatusNonFinite);
