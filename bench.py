@@ -396,26 +396,32 @@ def main():
     st.sort()
     ms_infer = timed(infer_step, args.steps)
 
+    peak_mem = torch.cuda.max_memory_allocated(device) / 1e9  # the device-resident step
+
     # the same train step captured once as a CUDA graph and replayed: every call of
     # the step is stream-ordered and never synchronises, so all its launches go in
     # the graph and the host's per-launch cost leaves the timed region (one GPU:
     # a graph holding NCCL calls is not built here)
     graph = None
     if world == 1:
-        side = torch.cuda.Stream(device)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
+        # warm-up and capture on one stream, whose scratch (one more workspace) is
+        # released afterwards
+        cap = torch.cuda.Stream(device)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
             for _ in range(3):
-                train_step()  # workspaces at their full size before the capture
-        stream.wait_stream(side)
+                train_step()  # the capture stream's workspace at its full size
+        stream.wait_stream(cap)
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
+        with torch.cuda.graph(g, stream=cap):
             train_step()
         ms_graph = timed(g.replay, args.steps)
         L.check()
         graph = {"value": round(elements(w) / (ms_graph * 1e-3), 1), "ms_per_step": round(ms_graph, 4),
                  "what": "the train step (sort, forward, backward) replayed as one CUDA graph"}
         del g
+        L.release_workspace(cap)
+        torch.cuda.synchronize(device)
         st.sort()
 
     # the same train steps with every kernel bracketed by CUDA events
@@ -424,8 +430,6 @@ def main():
     prof = L.profile_report()
     L.profile_enable(False)
     L.check()
-
-    peak_mem = torch.cuda.max_memory_allocated(device) / 1e9  # the device-resident step
 
     # training with a warm-start re-sort: the anchors alternate between two sets
     # one update apart (a and a + WARM_MOVE * N(0, 1)); each step re-sorts from the
@@ -461,6 +465,8 @@ def main():
                 "paths_seen": sorted({L.RESORT_PATHS[q] for q in paths})}
         warm["full_sort_ms"] = round(timed(lambda: L.sort_anchors(anchors[0]), args.steps), 4)
         st.sort()
+
+    torch.cuda.reset_peak_memory_stats(device)  # the end-to-end leg's own peak below
 
     # end to end through host buffers: every step copies its inputs from pinned host
     # memory to the device, runs, and copies its results back.  The steps are

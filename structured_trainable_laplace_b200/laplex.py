@@ -105,6 +105,14 @@ def workspace(nbytes: int, device: int) -> torch.Tensor:
     return buf
 
 
+def release_workspace(stream=None, device: int | None = None) -> None:
+    """Drop the cached scratch of `stream` (default: the current stream), e.g. after
+    a side stream or a graph-capture stream is no longer used."""
+    device = torch.cuda.current_device() if device is None else device
+    stream = torch.cuda.current_stream(device) if stream is None else stream
+    _ws.pop((device, stream.cuda_stream), None)
+
+
 def status_word(device: int) -> torch.Tensor:
     st = _status.get(device)
     if st is None:
