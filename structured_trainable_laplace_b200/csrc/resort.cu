@@ -41,11 +41,6 @@ constexpr int64_t kMaxDisplacedDen = 2;
 
 __device__ __forceinline__ uint64_t comp(uint32_t key, uint32_t idx) { return ((uint64_t)key << 32) | idx; }
 
-__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
-    const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
-    const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
-    return ((uint64_t)hi << 32) | lo;
-}
 __device__ __forceinline__ uint64_t shfl_up_u64(uint64_t v, int d) {
     const uint32_t lo = __shfl_up_sync(0xffffffffu, (uint32_t)v, d);
     const uint32_t hi = __shfl_up_sync(0xffffffffu, (uint32_t)(v >> 32), d);
