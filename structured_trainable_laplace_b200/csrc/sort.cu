@@ -263,14 +263,15 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
 // Up to kSmallMax anchors: rank by counting.  The composites c_i = (key_i << 32 | i)
 // are distinct and ordered as the stable sort orders the anchors, so the position
 // of anchor i is the number of composites below c_i.  Each CTA holds all n
-// composites in shared memory and ranks kRankPer of them (four threads per
-// anchor, each counting over every fourth composite: consecutive words, no bank
-// conflicts), then writes those anchors to their positions.  One launch of
+// composites in shared memory and ranks kRankPer of them (kRankParts threads per
+// anchor, each counting over every kRankParts-th composite: consecutive words, no
+// bank conflicts), then writes those anchors to their positions.  One launch of
 // ceil(n / kRankPer) CTAs instead of five; the result equals the radix sort's.
 
 constexpr int kSmallMax = 8192;
-constexpr int kRankPer = 64;
-constexpr int kRankNT = 4 * kRankPer;
+constexpr int kRankParts = 8;
+constexpr int kRankPer = 32;
+constexpr int kRankNT = kRankParts * kRankPer;
 
 __global__ void __launch_bounds__(kRankNT) k_sort_small(const float* __restrict__ a, int n,
                                                         float* __restrict__ a_sorted, uint32_t* __restrict__ perm,
@@ -279,12 +280,12 @@ __global__ void __launch_bounds__(kRankNT) k_sort_small(const float* __restrict_
     for (int i = threadIdx.x; i < n; i += kRankNT)
         s_c[i] = ((unsigned long long)float_to_key(__ldg(a + i)) << 32) | (unsigned)i;
     __syncthreads();
-    const int el = blockIdx.x * kRankPer + (threadIdx.x >> 2), part = threadIdx.x & 3;
+    const int el = blockIdx.x * kRankPer + threadIdx.x / kRankParts, part = threadIdx.x % kRankParts;
     const unsigned long long mine = el < n ? s_c[el] : 0ull;
     int below = 0;
-    for (int q = part; q < n; q += 4) below += s_c[q] < mine;
-    below += __shfl_xor_sync(0xffffffffu, below, 1);
-    below += __shfl_xor_sync(0xffffffffu, below, 2);
+    for (int q = part; q < n; q += kRankParts) below += s_c[q] < mine;
+#pragma unroll
+    for (int d = 1; d < kRankParts; d <<= 1) below += __shfl_xor_sync(0xffffffffu, below, d);
     if (part == 0 && el < n) {
         if (is_nonfinite(__ldg(a + el))) raise_status(status, kStatusNonFinite);
         a_sorted[below] = key_to_float((uint32_t)(mine >> 32));
