@@ -51,6 +51,9 @@ def test_status_strings(L):
 def test_size_queries(L):
     from structured_trainable_laplace_b200 import laplex
     assert laplex.sort_workspace_size(1 << 24) >= 8 * (1 << 24)
+    # the re-sort's workspace also holds the full sort's (its fallback)
+    assert laplex.resort_workspace_size(1 << 24) >= laplex.sort_workspace_size(1 << 24)
+    assert laplex.resort_workspace_size(0) == 0
     assert laplex.workspace_size("sym", 1 << 24, 1, 16) > 0
     assert laplex.saved_size("sym", 1 << 24, 1, 16) > 0
     assert laplex.workspace_size("phased_transpose", 1 << 22, 1024, 128) > 0
@@ -90,3 +93,13 @@ def test_bad_arguments_are_rejected_before_launch(L):
     assert L.laplex_apply_sym_noalloc(fake, fake, 4097, fake, 257, P(1 << 24), None, None) == 3
     # sort: n too large
     assert L.laplex_sort_anchors(fake, 1 << 33, fake, fake, ws, 1 << 30, None, None) == 1
+    # warm-start re-sort: NULL previous permutation, small workspace, misaligned
+    # output, output overlapping perm_prev
+    big = 1 << 30
+    assert L.laplex_resort_anchors(fake, 8, None, fake, fake, ws, big, None, None, None) == 1
+    assert L.laplex_resort_anchors(P(1 << 20), 8, P(1 << 22), P(1 << 23), P(1 << 24), P(1 << 25), 64, None, None,
+                                   None) == 3
+    assert L.laplex_resort_anchors(P(1 << 20), 8, P(1 << 22), P((1 << 23) + 4), P(1 << 24), P(1 << 25), big, None,
+                                   None, None) == 2
+    assert L.laplex_resort_anchors(P(1 << 20), 8, P(1 << 22), P(1 << 22), P(1 << 24), P(1 << 25), big, None, None,
+                                   None) == 1
