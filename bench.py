@@ -2,7 +2,8 @@
 """Throughput of the LAPLEX hot path on B200: one JSON line on rank 0.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload sym2p24|small|phased_head|gram_image|sym1e9]
+                    [--workload sym2p24|small|phased_head|gram_image|gram_image_full|sym1e9]
+                    [--n N]  (large-side size override, for profiling captures of a smaller case)
 
 A step is one training pass of the operator on one batch: sort the anchors,
 forward, backward (all gradients), and for N > 1 GPUs the all-reduce of the

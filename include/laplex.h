@@ -104,7 +104,9 @@ size_t laplex_sort_workspace_size(int64_t n);
  *   perm      [n] uint32 out: a_sorted[r] == a[perm[r]]; equal anchors keep
  *             ascending original index, so perm is unique (stable sort).
  * A least-significant-digit radix sort of an order-preserving uint32 key
- * (4 passes of 8 bits).  NaN or infinite anchors set LAPLEX_ERR_NONFINITE. */
+ * (4 passes of 8 bits); up to 8192 anchors, one launch that ranks each anchor by
+ * counting the (key, index) pairs below its own.  Both give the same unique order.
+ * NaN or infinite anchors set LAPLEX_ERR_NONFINITE. */
 laplex_status laplex_sort_anchors(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws,
                                   size_t ws_bytes, int32_t* d_status, laplex_stream_t stream);
 
