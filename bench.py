@@ -232,8 +232,34 @@ KERNEL_SOURCE = (("sym_", "sym.cu"), ("radix_", "sort.cu"), ("sort_small", "sort
                  ("gram_", "rect.cu"))
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source with comments removed and whitespace collapsed (string
+    literals kept), so that editing a comment leaves the hash unchanged."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash(kernel: str) -> str:
-    """Hash of the kernel's own .cu file and every shared header it can include."""
+    """Hash of the code (comments removed) of the kernel's own .cu file and every
+    shared header it can include."""
     csrc = os.path.join(ROOT, "structured_trainable_laplace_b200", "csrc")
     own = next((f for pre, f in KERNEL_SOURCE if kernel.startswith(pre)), None)
     files = sorted(glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.h")) +
@@ -241,7 +267,7 @@ def source_hash(kernel: str) -> str:
     files += [os.path.join(csrc, own)] if own else sorted(glob.glob(os.path.join(csrc, "*.cu")))
     h = hashlib.sha256()
     for p in files:
-        h.update(open(p, "rb").read())
+        h.update(_code_only(open(p, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -74,3 +74,10 @@ def test_clock_summary(bench, tmp_path):
     assert s["samples"] == 3 and s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
     assert s["reasons"] == ["sw_power_cap"]
     assert bench.summarize_clocks(str(tmp_path / "missing.csv"), 0)["samples"] == 0
+
+
+def test_comment_edits_leave_the_source_hash_alone(bench):
+    a = 'int a; // one\n/* two\n lines */ const char* s = "x // kept"; float f;'
+    b = 'int a;   // changed\n/* other */ const char* s = "x // kept";\nfloat f;'
+    assert bench._code_only(a) == bench._code_only(b) == 'int a; const char* s = "x // kept"; float f;'
+    assert bench._code_only('x = "a\\"b // in string"; y; // gone') == 'x = "a\\"b // in string"; y;'
