@@ -169,8 +169,14 @@ laplex_status laplex_apply_sym(const float* a_sorted, const uint32_t* perm, int6
  *     the next of 1, 2, 4, 8, 16, 32, or to a multiple of 32 above 32 (B = 16
  *     allows n up to 65536); larger problems return LAPLEX_ERR_WORKSPACE before
  *     anything is launched -- use laplex_apply_sym for them;
- *   - the first call on each device performs a one-time setup (it looks up the
- *     device address of the static array), so make it before any stream capture;
+ *   - the first call in each CUDA context performs a one-time setup (it looks up
+ *     the device address of the static array in that context), so make it before
+ *     any stream capture; a new context on the same device (after
+ *     cudaDeviceReset, or another context made current) gets its own setup on
+ *     its first call, since the array may then sit at another address;
+ *   - on a device with many more SMs than a B200 the per-SM scan state can
+ *     exceed the array at sizes below the limit: such calls also return
+ *     LAPLEX_ERR_WORKSPACE before anything is launched;
  *   - calls must not overlap on one device: two calls in flight at once (on two
  *     streams, or from two host threads) share the scratch and race;
  *   - nothing has to be zeroed beforehand. */

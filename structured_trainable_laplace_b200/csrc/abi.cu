@@ -182,6 +182,7 @@ laplex_status laplex_apply_sym_noalloc(const float* a_sorted, const uint32_t* pe
                                        int64_t B, float* y, int32_t* d_status, laplex_stream_t stream) {
     if (!size_ok(n) || !batch_ok(B) || !a_sorted || !perm || !x || !y) return LAPLEX_ERR_ARG;
     if (n > LAPLEX_NOALLOC_MAX_ELEMS / sym_padded_batch(B)) return LAPLEX_ERR_WORKSPACE;
+    if (!sym_noalloc_fits(n, B)) return LAPLEX_ERR_WORKSPACE;  // the plan on this device's SM count
     laplex_status s = check_ranges({{a_sorted, fbytes(n)}, {perm, fbytes(n)}, {x, fbytes(n * B)}},
                                    {{y, fbytes(n * B)}, {d_status, 4}});
     if (s != LAPLEX_OK) return s;

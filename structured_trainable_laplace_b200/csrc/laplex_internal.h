@@ -74,9 +74,11 @@ cudaError_t launch_sym_backward(const float* s, const uint32_t* perm, int64_t n,
                                 int64_t B, const void* saved, float* gx, float* ga, void* ws, int32_t* status,
                                 cudaStream_t stream);
 // The symmetric forward on the library's static scratch (laplex_apply_sym_noalloc):
-// B rounded up to whole channel groups, and the launcher.  The launcher returns
-// cudaErrorInvalidValue if the problem does not fit the scratch.
+// B rounded up to whole channel groups; whether the plan of (n, B) on the current
+// device fits the scratch (checked before any launch); the launcher, which returns
+// cudaErrorInvalidValue if the problem does not fit.
 int64_t sym_padded_batch(int64_t B);
+bool sym_noalloc_fits(int64_t n, int64_t B);
 cudaError_t launch_sym_forward_noalloc(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B,
                                        float* y, int32_t* status, cudaStream_t stream);
 

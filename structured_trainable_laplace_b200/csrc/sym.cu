@@ -34,6 +34,8 @@
 // are computed one tile ahead.  No kernel waits on another CTA.
 #include <mutex>
 
+#include <cuda.h>
+
 #include "laplex.h"
 #include "laplex_internal.h"
 #include "pipeline.cuh"
@@ -1453,7 +1455,9 @@ cudaError_t launch_sym_backward(const float* s, const uint32_t* perm, int64_t n,
 // Scratch of laplex_apply_sym_noalloc: part of the library's static device
 // memory (one copy per device, created with the module), so that entry point
 // takes no workspace and allocates nothing.  LAPLEX_NOALLOC_SCRATCH_BYTES covers
-// every problem with n * sym_padded_batch(B) <= LAPLEX_NOALLOC_MAX_ELEMS.
+// every problem with n * sym_padded_batch(B) <= LAPLEX_NOALLOC_MAX_ELEMS on a GPU
+// of up to about 300 SMs (the range arrays grow with the SM count);
+// sym_noalloc_fits checks the actual plan on the current device before any launch.
 // Nothing in it has to start at zero: every word the kernels read is written
 // earlier in the same call.  Calls whose work overlaps on one device (two
 // streams, or two host threads) share the array and corrupt each other.
@@ -1461,30 +1465,82 @@ static __device__ __align__(256) unsigned char g_sym_scratch[LAPLEX_NOALLOC_SCRA
 
 namespace {
 
+// The device address of g_sym_scratch belongs to the CUDA context that loaded the
+// module: a new context on the same device (after cudaDeviceReset, or another
+// context made current) loads the module again, possibly elsewhere.  The address
+// is therefore cached per device together with the unique id of the context it
+// was looked up in, and looked up again when the current context's id differs.
+// The context calls come from the driver through the runtime's entry-point query,
+// so the library needs no link to the driver library.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+struct ScratchCache {
+    unsigned long long ctx_id = 0;  // 0: nothing cached (context ids start at 1)
+    void* ptr = nullptr;
+};
+
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+ScratchCache g_scratch[kMaxDevices];
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
 
-// Device address of g_sym_scratch on the current device, looked up the first
-// time a device is used (the only setup step; later calls reuse it).
+cudaError_t current_context_id(unsigned long long* id) {
+    if (g_ctx_current == nullptr || g_ctx_id == nullptr) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = q1;
+        cudaError_t e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1);
+        if (e == cudaSuccess) e = cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2);
+        if (e != cudaSuccess) return e;
+        if (q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || !f1 || !f2)
+            return cudaErrorNotSupported;
+        g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        g_ctx_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+    if (g_ctx_id(ctx, id) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    return cudaSuccess;
+}
+
+// Device address of g_sym_scratch in the current context, looked up the first
+// time a context is used on a device (the only setup step; later calls in the same
+// context reuse it).
 cudaError_t sym_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    e = cudaFree(nullptr);  // makes the device's primary context current (allocates nothing)
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    unsigned long long id = 0;
+    e = current_context_id(&id);
+    if (e != cudaSuccess) return e;
+    ScratchCache& c = g_scratch[dev];
+    if (c.ptr == nullptr || c.ctx_id != id) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_sym_scratch);
         if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
+        c.ptr = p;
+        c.ctx_id = id;
     }
-    *out = g_scratch_ptr[dev];
+    *out = c.ptr;
     return cudaSuccess;
 }
 
-// The forward of sym_forward_t with its scratch carved from g_sym_scratch: range
-// arrays sized for this device's ranges only, no saved state.
+// Plan of the static-scratch forward: the plan of sym_forward_t with the range
+// arrays sized for this device's ranges only and no saved state; the bytes it
+// carves from g_sym_scratch.
+SymPlan plan_sym_static(int64_t n, int64_t B, int sms, size_t* state_bytes) {
+    SymPlan p = plan_sym(n, B, sms);
+    p.rng_elems = (size_t)p.G * p.P * p.C;
+    *state_bytes = align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
+    return p;
+}
+
 template <int C>
 cudaError_t sym_forward_static_t(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B, float* y,
                                  cudaStream_t st) {
@@ -1492,9 +1548,9 @@ cudaError_t sym_forward_static_t(const float* s, const uint32_t* perm, int64_t n
     cudaError_t e = sym_scratch(&scratch);
     if (e != cudaSuccess) return e;
     const int sms = device_sms();
-    SymPlan p = plan_sym(n, B, sms);
-    p.rng_elems = (size_t)p.G * p.P * p.C;
-    const size_t state = align_up(sizeof(double2) * (p.rs_elems + 4 * p.rng_elems), 256);
+    size_t state = 0;
+    const SymPlan p = plan_sym_static(n, B, sms, &state);
+    // checked before the call by sym_noalloc_fits; kept as a guard
     if (state + p.sorted_bytes > (size_t)LAPLEX_NOALLOC_SCRATCH_BYTES) return cudaErrorInvalidValue;
     const RangeState sx = carve(p, (double2*)scratch, true);
     float* xs = (float*)((char*)scratch + state);
@@ -1508,6 +1564,13 @@ cudaError_t sym_forward_static_t(const float* s, const uint32_t* perm, int64_t n
 int64_t sym_padded_batch(int64_t B) {
     const int64_t C = choose_channels(B);
     return (B + C - 1) / C * C;
+}
+
+bool sym_noalloc_fits(int64_t n, int64_t B) {
+    if (n > LAPLEX_NOALLOC_MAX_ELEMS / sym_padded_batch(B)) return false;
+    size_t state = 0;
+    const SymPlan p = plan_sym_static(n, B, device_sms(), &state);
+    return state + p.sorted_bytes <= (size_t)LAPLEX_NOALLOC_SCRATCH_BYTES;
 }
 
 cudaError_t launch_sym_forward_noalloc(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B,

@@ -240,7 +240,9 @@ def apply_sym_noalloc(a_sorted, perm, x):
     return back(y)
 
 
-def _rect(fn, op, a_sorted, perm_a, b_sorted, perm_b, x, out_rows, saved, extra_front=(), extra_mid=()):
+def _rect(op, a_sorted, b_sorted, x, out_rows):
+    """Rows of x, the output buffer, its reshaping back, and the workspace of a
+    rectangular op."""
     xr, sq = _rows(x)
     B = xr.shape[1]
     n, k = a_sorted.numel(), b_sorted.numel()
@@ -252,8 +254,7 @@ def _rect(fn, op, a_sorted, perm_a, b_sorted, perm_b, x, out_rows, saved, extra_
 
 def apply_general(a_sorted, perm_a, b_sorted, perm_b, x, saved=None):
     """y = E x with E_ij = exp(-|a_i - b_j|); x [k][B] -> y [n][B]."""
-    xr, y, back, ws, d, n, k, B = _rect(None, OP_GENERAL, a_sorted, perm_a, b_sorted, perm_b, x,
-                                        a_sorted.numel(), saved)
+    xr, y, back, ws, d, n, k, B = _rect(OP_GENERAL, a_sorted, b_sorted, x, a_sorted.numel())
     _ok(lib().laplex_apply_general(_p(a_sorted), _p(perm_a), n, _p(b_sorted), _p(perm_b), k, _p(xr), B, _p(y),
                                    _p(saved), _p(ws), ws.numel(), _p(status_word(d)), _stream(d)), "apply_general")
     return back(y)
@@ -261,8 +262,7 @@ def apply_general(a_sorted, perm_a, b_sorted, perm_b, x, saved=None):
 
 def apply_transpose(a_sorted, perm_a, b_sorted, perm_b, x, saved=None):
     """z = E^T x; x [n][B] -> z [k][B]."""
-    xr, z, back, ws, d, n, k, B = _rect(None, OP_TRANSPOSE, a_sorted, perm_a, b_sorted, perm_b, x,
-                                        b_sorted.numel(), saved)
+    xr, z, back, ws, d, n, k, B = _rect(OP_TRANSPOSE, a_sorted, b_sorted, x, b_sorted.numel())
     _ok(lib().laplex_apply_transpose(_p(a_sorted), _p(perm_a), n, _p(b_sorted), _p(perm_b), k, _p(xr), B, _p(z),
                                      _p(saved), _p(ws), ws.numel(), _p(status_word(d)), _stream(d)),
         "apply_transpose")
@@ -273,7 +273,7 @@ def apply_phased(a_sorted, perm_a, phi, b_sorted, perm_b, psi, x, transpose=Fals
     """Phased operator E_ij = exp(-|a_i - b_j|) cos(phi_i - psi_j); transpose selects E^T."""
     op = OP_PHASED_TRANSPOSE if transpose else OP_PHASED
     rows = b_sorted.numel() if transpose else a_sorted.numel()
-    xr, out, back, ws, d, n, k, B = _rect(None, op, a_sorted, perm_a, b_sorted, perm_b, x, rows, saved)
+    xr, out, back, ws, d, n, k, B = _rect(op, a_sorted, b_sorted, x, rows)
     _ok(lib().laplex_apply_phased(_p(a_sorted), _p(perm_a), n, _p(phi), _p(b_sorted), _p(perm_b), k, _p(psi),
                                   int(bool(transpose)), _p(xr), B, _p(out), _p(saved), _p(ws), ws.numel(),
                                   _p(status_word(d)), _stream(d)), "apply_phased")

@@ -74,3 +74,42 @@ def test_shard_columns_partition(B, world):
     cols = [dp.shard_columns(B, r, world) for r in range(world)]
     covered = np.concatenate([np.arange(B)[c] for c in cols])
     np.testing.assert_array_equal(covered, np.arange(B))
+
+
+class _FakeDist:
+    """Stands in for torch.distributed: a group of `world` ranks whose other ranks
+    all hold `other` times this rank's values; counts the collectives issued."""
+
+    def __init__(self, world, other):
+        self.world, self.other, self.calls = world, other, []
+
+    def is_initialized(self):
+        return True
+
+    def get_world_size(self, group=None):
+        return self.world
+
+    def all_reduce(self, t, group=None):
+        self.calls.append(t.numel())
+        t.mul_(1 + self.other * (self.world - 1))
+
+
+def test_param_grads_reduced_in_one_collective():
+    """Every shared-parameter gradient present goes through one flat all-reduce and
+    comes back in place with its own shape; vector gradients are left alone."""
+    rng = np.random.default_rng(0)
+    grads = {"gx": torch.from_numpy(rng.standard_normal((7, 3))), "ga": torch.from_numpy(rng.standard_normal(7)),
+             "gb": torch.from_numpy(rng.standard_normal(5)), "gphi": torch.from_numpy(rng.standard_normal(7)),
+             "gpsi": torch.from_numpy(rng.standard_normal(5))}
+    before = {k: v.clone() for k, v in grads.items()}
+    fake = _FakeDist(world=3, other=2.0)
+    out = dp.allreduce_param_grads(grads, dist=fake)
+    assert out is grads
+    assert fake.calls == [7 + 5 + 7 + 5]
+    for key in ("ga", "gb", "gphi", "gpsi"):
+        np.testing.assert_array_equal(grads[key].numpy(), 5.0 * before[key].numpy())
+    np.testing.assert_array_equal(grads["gx"].numpy(), before["gx"].numpy())
+    one = {"ga": torch.ones(4)}
+    fake1 = _FakeDist(world=2, other=1.0)
+    dp.allreduce_param_grads(one, dist=fake1)
+    assert fake1.calls == [4] and torch.equal(one["ga"], torch.full((4,), 2.0))
