@@ -34,10 +34,11 @@ _ERRORS = {1: "bad argument", 4: "non-finite anchor", 7: "out of memory"}
 
 
 def build(force: bool = False) -> str:
-    """Compile the C oracle into oracle/liblaplex_oracle.so (gcc, -O2)."""
+    """Compile the C oracle into oracle/liblaplex_oracle.so (gcc, -O2, OpenMP for the
+    optional threading of the sampled evaluation)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -60,7 +61,7 @@ def _load():
         lib.oracle_rect_backward.argtypes = [P, I64, P, I64, P, P, P, P, I64, I, P, P, P, P, P, I]
         lib.oracle_gram_apply.argtypes = [P, I64, P, I64, P, P, I64, P, P, I]
         lib.oracle_gram_backward_D.argtypes = [P, I64, P, I64, P, P, I64, P, I]
-        lib.oracle_sym_sampled.argtypes = [P, I64, P, P, I64, P, I64, D, P, P, P, P, P]
+        lib.oracle_sym_sampled.argtypes = [P, I64, P, P, I64, P, I64, D, P, P, P, P, P, I]
         for f in ("oracle_sort", "oracle_sym_apply", "oracle_sym_backward", "oracle_rect_apply",
                   "oracle_rect_backward", "oracle_gram_apply", "oracle_gram_backward_D", "oracle_sym_sampled"):
             getattr(lib, f).restype = ctypes.c_int
@@ -198,9 +199,10 @@ def gram_backward(a, b, D, v, g, twin=False):
     }
 
 
-def sym_sampled(a, x, samples, g=None, window=100.0):
+def sym_sampled(a, x, samples, g=None, window=100.0, threads=1):
     """Windowed direct evaluation of the symmetric operator at sample indices.
-    Returns dict y, y_twin [m][B], dropped [B] (and ga, ga_twin [m] if g given)."""
+    Returns dict y, y_twin [m][B], dropped [B] (and ga, ga_twin [m] if g given).
+    threads > 1 evaluates the samples on that many host threads."""
     a, x = _f32(a), _rows(x)
     g = None if g is None else _rows(g)
     samples = np.ascontiguousarray(samples, dtype=np.int64)
@@ -212,7 +214,7 @@ def sym_sampled(a, x, samples, g=None, window=100.0):
     ga = np.empty(m, np.float64) if g is not None else None
     gat = np.empty(m, np.float64) if g is not None else None
     _check(_load().oracle_sym_sampled(_ptr(a), n, _ptr(x), _ptr(g), B, _ptr(samples), m, float(window), _ptr(y),
-                                      _ptr(yt), _ptr(ga), _ptr(gat), _ptr(drop)), "sym_sampled")
+                                      _ptr(yt), _ptr(ga), _ptr(gat), _ptr(drop), int(threads)), "sym_sampled")
     out = {"y": y, "y_twin": yt, "dropped": drop}
     if g is not None:
         out["ga"] = ga

@@ -534,10 +534,11 @@ int oracle_gram_backward_D(const float* a, int64_t n, const float* b, int64_t k,
  * Anchors are first binned by floor(a / window) (a counting sort, O(n)); each
  * sample then visits the bins within reach.  The dropped mass is at most
  * exp(-window) * sum_j |x_j|, returned in *dropped_bound (per channel maximum).
- * Outputs: y [m][B], ga [m] (NULL to skip), twins likewise. */
+ * Outputs: y [m][B], ga [m] (NULL to skip), twins likewise.  threads > 1 shares
+ * the samples out over that many host threads (when built with OpenMP). */
 int oracle_sym_sampled(const float* a, int64_t n, const float* x, const float* g, int64_t B, const int64_t* samples,
                        int64_t m, double window, double* y, double* y_twin, double* ga, double* ga_twin,
-                       double* dropped_bound) {
+                       double* dropped_bound, int threads) {
     if (n < 1 || B < 1 || m < 0 || !a || !x || !samples || !(window > 0)) return OR_ERR_ARG;
     double amin = INFINITY, amax = -INFINITY;
     for (int64_t i = 0; i < n; ++i) {
@@ -573,33 +574,29 @@ int oracle_sym_sampled(const float* a, int64_t n, const float* x, const float* g
             for (int64_t c = 0; c < B; ++c) dropped_bound[c] += fabs((double)x[i * B + c]);
         for (int64_t c = 0; c < B; ++c) dropped_bound[c] *= exp(-window);
     }
-    double* tmp = dalloc(8 * B);
-    if (!tmp) {
-        free(start);
-        free(order);
-        return OR_ERR_NOMEM;
-    }
     for (int64_t s = 0; s < m; ++s) {
-        int64_t i = samples[s];
-        if (i < 0 || i >= n) {
-            free(tmp);
+        if (samples[s] < 0 || samples[s] >= n) {
             free(start);
             free(order);
             return OR_ERR_ARG;
         }
+    }
+    int failed = 0;
+    /* the samples are independent: with threads > 1 they are shared out over host
+     * threads, each with its own accumulators; the arithmetic is the same */
+#pragma omp parallel for num_threads(threads > 1 ? threads : 1) schedule(dynamic, 64) reduction(| : failed)
+    for (int64_t s = 0; s < m; ++s) {
+        const int64_t i = samples[s];
+        double* tmp = dalloc(10 * B);
+        if (!tmp) {
+            failed = 1;
+            continue;
+        }
         double ai = a[i];
         int64_t bi = (int64_t)floor((ai - amin) / window);
         double *Lx = tmp, *Rx = tmp + B, *Tx = tmp + 2 * B, *Lg = tmp + 3 * B, *Rg = tmp + 4 * B;
-        double *aLx = tmp + 5 * B, *aRx = tmp + 6 * B, *aT = tmp + 7 * B;
-        for (int64_t c = 0; c < 8 * B; ++c) tmp[c] = 0.0;
+        double *aLx = tmp + 5 * B, *aRx = tmp + 6 * B, *aT = tmp + 7 * B, *aLg = tmp + 8 * B, *aRg = tmp + 9 * B;
         double ga_acc = 0, gat_acc = 0;
-        double *aLg = NULL, *aRg = NULL;
-        double* extra = NULL;
-        if (g) {
-            extra = dalloc(2 * B);
-            aLg = extra;
-            aRg = extra + B;
-        }
         /* the window spans bins bi-1..bi+1; two more absorb rounding in the bin index */
         for (int64_t t = bi - 2; t <= bi + 2; ++t) {
             if (t < 0 || t >= nb) continue;
@@ -634,10 +631,9 @@ int oracle_sym_sampled(const float* a, int64_t n, const float* x, const float* g
         }
         if (g && ga) ga[s] = ga_acc;
         if (g && ga_twin) ga_twin[s] = gat_acc;
-        free(extra);
+        free(tmp);
     }
-    free(tmp);
     free(start);
     free(order);
-    return OR_OK;
+    return failed ? OR_ERR_NOMEM : OR_OK;
 }

@@ -62,6 +62,14 @@ def test_full_size_sort_of_the_2p24_workload(L):
     check_sort(L, inputs.sym_2p24_b16(0)["a"])
 
 
+def test_bit_exact_past_2p24():
+    """2^25 + 4097 anchors of the 10^9 workload's recipe (a ~ U[0, 0.05 n], fp32
+    ulp 2 at the top: runs of ties), bit for bit against the oracle's stable sort:
+    past 2^24 the radix passes run 8739 tiles and the lookback reaches further."""
+    L = laplex_or_fail()
+    check_sort(L, inputs.sym_extreme(4, n=(1 << 25) + 4097)["a"])
+
+
 def test_nonfinite_anchor_sets_the_status_word(L):
     a = np.linspace(0, 1, 5000).astype(np.float32)
     a[1234] = np.nan
