@@ -109,39 +109,81 @@ def compulsory_bytes(w) -> int:
     raise ValueError(w.op)
 
 
-# Algorithmic bytes per element row of each kernel (sorted anchor 4 + permutation 4
-# + the row values it must read or write), used for the roofline of the kernel
-# that dominates the step.  Units per launch: the rows that launch walks.
-def kernel_bytes_per_launch(kernel: str, w) -> float | None:
+# Algorithmic bytes of each kernel per training step, two ways:
+#   method  the bytes of the method's own data the kernel must move (sorted anchors,
+#           permutation, the input and output vectors and gradients), each counted
+#           where the path reads or writes it -- the unit of the roofline fraction;
+#   design  the bytes the kernel moves in this design, including its intermediates
+#           (the sorted tile-major copies of the symmetric path, the radix passes'
+#           key and value arrays, the bucketed single-channel outputs).
+# Per step, so that kernels launched several times per step (the aggregate pass on
+# x and on g, the radix passes of both sorts of a rectangular operator) are summed
+# over their launches.
+def _sort_bytes(m: int):
+    """(method, design) per step of the radix kernels sorting m anchors (up to 8192
+    the counting sort runs instead)."""
+    if m <= 8192:
+        return {"sort_small": (12 * m, 12 * m)}
+    # hist reads a; pass 0 reads a and writes key+value, passes 1-3 read and write
+    # key+value (the last writes a_sorted and perm)
+    return {"radix_hist": (4 * m, 4 * m), "radix_pass": (8 * m, (12 + 3 * 16) * m)}
+
+
+def _merge(*tables):
+    out = {}
+    for t in tables:
+        for key, (m, d) in t.items():
+            pm, pd = out.get(key, (0, 0))
+            out[key] = (pm + m, pd + d)
+    return out
+
+
+def kernel_bytes_per_step(kernel: str, w):
+    """(method bytes, design bytes) that `kernel` moves per training step, or None."""
     n, B, k = w.n, w.B, w.k
     if w.op == "sym":
+        bucketed = B == 1 and n > (1 << 24)
         table = {
-            "sym_agg": (8 + 4 * B + 4 * B) * n,              # s, perm, x rows gathered -> sorted copy of x
-            "sym_fwd": (8 + 4 * B + 4 * B) * n,              # s, perm, sorted copy of x -> y rows scattered
-            "sym_bwd": (8 + 4 * B + 4 * B + 4 * B + 4) * n,  # s, perm, sorted x, sorted g -> gx rows, ga
-            "radix_pass": (12 * n + 3 * 16 * n) / 4.0,       # pass 0 reads a; passes 1-3 read+write key,value
-            "radix_hist": 4 * n,
-            "sort_small": 12 * n,                            # a in; a_sorted, perm out (n <= 8192)
-            # one channel past 2^24 rows: outputs placed through destination buckets
-            # (3 vectors per step: y, gx, ga; 2 split launches and 1 placement each)
-            "unpermute_split": 16 * n,                       # (destination, value) in and out
-            "unpermute_place": 12 * n,                       # pairs in, the output window out
+            # x (forward) and g (backward) gathered through the permutation; the
+            # design also writes their sorted copies
+            "sym_agg": (2 * (8 + 4 * B) * n, 2 * (8 + 8 * B) * n),
         }
+        if bucketed:
+            # the sweeps write sorted-order outputs; the permutation is read and the
+            # outputs y, gx, ga written in original order by the bucketed unpermute
+            table.update({
+                "sym_fwd": (4 * n, (4 + 8 * B) * n),
+                "sym_bwd": (4 * n, (4 + 12 * B + 4) * n),
+                "unpermute_split": (3 * 4 * n, 3 * 2 * 16 * n),
+                "unpermute_place": (3 * 4 * n, 3 * 12 * n),
+            })
+        else:
+            table.update({
+                "sym_fwd": ((8 + 4 * B) * n, (8 + 8 * B) * n),               # + the sorted copy of x read
+                "sym_bwd": ((8 + 4 * B + 4) * n, (8 + 12 * B + 4) * n),      # + sorted x and g read
+            })
+        table = _merge(table, _sort_bytes(n))
         return table.get(kernel)
     if w.op == "phased_transpose":
-        table = {
-            "large_accum": (12 + 4 * B) * n,                 # s, perm, phi, x rows
-            "large_expand_grad": (12 + 4 * B + 4 * B + 8) * n,  # + gx rows, ga, gphi
-            "radix_pass": (12 * n + 3 * 16 * n) / 4.0,
-        }
+        table = _merge({
+            "large_accum": ((12 + 4 * B) * n, (12 + 4 * B) * n),              # s, perm, phi, x rows
+            "large_expand_grad": ((12 + 8 * B + 8) * n, (12 + 8 * B + 8) * n),  # + gx rows, ga, gphi
+        }, _sort_bytes(n), _sort_bytes(k))
         return table.get(kernel)
-    if w.op in ("gram", "gram_full"):
-        table = {
-            "large_accum": (8 + 8 * B) * n,                  # paired pass: s, perm, v and g rows
-            "large_expand": (8 + 4 * B) * n,
-            "large_accum_grad": (8 + 4 * B + 4) * n,         # s, perm, upstream rows, ga
-            "radix_pass": (12 * n + 3 * 16 * n) / 4.0,
-        }
+    if w.op == "gram":
+        table = _merge({
+            "large_accum": ((8 + 8 * B) * n, (8 + 8 * B) * n),    # paired pass: s, perm, v and g rows
+            "large_expand": ((8 + 4 * B) * n, (8 + 4 * B) * n),   # y rows
+        }, _sort_bytes(n), _sort_bytes(k))
+        return table.get(kernel)
+    if w.op == "gram_full":
+        table = _merge({
+            # A^T v (B channels, the apply) and the paired A^T v, A^T g (backward)
+            "large_accum": ((8 + 4 * B + 8 + 8 * B) * n, (8 + 4 * B + 8 + 8 * B) * n),
+            "large_expand": (2 * (8 + 4 * B) * n, 2 * (8 + 4 * B) * n),  # y and gv rows
+            # the two accumulating anchor-gradient passes: upstream rows, ga (read back by the second)
+            "large_accum_grad": ((2 * (8 + 4 * B + 4) + 4) * n, (2 * (8 + 4 * B + 4) + 4) * n),
+        }, _sort_bytes(n), _sort_bytes(k))
         return table.get(kernel)
     return None
 
@@ -151,10 +193,11 @@ def kernel_bytes_per_launch(kernel: str, w) -> float | None:
 class Step:
     """Device buffers and one training step of the workload through the binding."""
 
-    def __init__(self, L, w, device, torch):
+    def __init__(self, L, w, device, torch, tensors=None):
         self.L, self.w, self.torch = L, w, torch
         self.dev = device
-        self.t = {key: torch.from_numpy(np.ascontiguousarray(v)).to(device) for key, v in w.arrays.items()}
+        self.t = tensors if tensors is not None else \
+            {key: torch.from_numpy(np.ascontiguousarray(v)).to(device) for key, v in w.arrays.items()}
         self.saved = None
         if w.op == "sym":
             self.saved = L.saved_buffer("sym", w.n, 1, w.B, device)
@@ -295,37 +338,52 @@ def measured_peak():
 
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_sample(w, budget_s: float):
-    """Run the fp64 oracle (sort + forward + backward) on a prefix-sized draw of the
-    same workload, growing the sample until it takes about budget_s.  Returns
-    (elements/s, description)."""
+def oracle_inputs(w, n_s: int):
+    """A draw of n_s rows of the workload's recipe for the oracle (seed 123)."""
+    if w.op == "sym":
+        return inputs.symmetric(n_s, w.B, seed=123, spacing=0.05)
+    if w.op == "phased_transpose":
+        return inputs.phased_head(n_s, w.k, w.B, seed=123)
+    return inputs.gram(n_s, max(1, int(round(w.k * n_s / w.n))), w.B, seed=123)
+
+
+def oracle_pass(w, ws):
+    """One step of the fp64 oracle (sort + forward + backward, as the GPU step) on
+    the draw ws.  Returns (elements, seconds)."""
     import oracle
+    t0 = time.perf_counter()
+    if w.op == "sym":
+        oracle.sym_apply(ws["a"], ws["x"])
+        oracle.sym_backward(ws["a"], ws["x"], ws["g"])
+    elif w.op == "phased_transpose":
+        oracle.rect_apply(ws["a"], ws["b"], ws["x"], ws["phi"], ws["psi"], transpose=True)
+        oracle.rect_backward(ws["a"], ws["b"], ws["x"], ws["h"], ws["phi"], ws["psi"], transpose=True)
+    else:
+        oracle.gram_apply(ws["a"], ws["b"], ws["D"], ws["v"])
+        if w.op == "gram_full":
+            oracle.gram_backward(ws["a"], ws["b"], ws["D"], ws["v"], ws["g"])
+        else:
+            oracle.gram_backward_D(ws["a"], ws["b"], ws["v"], ws["g"])
+    return ws.n * w.B, time.perf_counter() - t0
+
+
+def oracle_sample_size(w, budget_s: float) -> int:
+    """Rows of the oracle sample that take about budget_s (grown from 2^14, at most
+    the workload's own n)."""
     n_s = 1 << 14
     while True:
-        t0 = time.perf_counter()
-        if w.op == "sym":
-            ws = inputs.symmetric(n_s, w.B, seed=123, spacing=0.05)
-            oracle.sym_apply(ws["a"], ws["x"])
-            oracle.sym_backward(ws["a"], ws["x"], ws["g"])
-            units = n_s * w.B
-        elif w.op == "phased_transpose":
-            ws = inputs.phased_head(n_s, w.k, w.B, seed=123)
-            oracle.rect_apply(ws["a"], ws["b"], ws["x"], ws["phi"], ws["psi"], transpose=True)
-            oracle.rect_backward(ws["a"], ws["b"], ws["x"], ws["h"], ws["phi"], ws["psi"], transpose=True)
-            units = n_s * w.B
-        else:
-            k_s = max(1, int(round(w.k * n_s / w.n)))
-            ws = inputs.gram(n_s, k_s, w.B, seed=123)
-            oracle.gram_apply(ws["a"], ws["b"], ws["D"], ws["v"])
-            if w.op == "gram_full":
-                oracle.gram_backward(ws["a"], ws["b"], ws["D"], ws["v"], ws["g"])
-            else:
-                oracle.gram_backward_D(ws["a"], ws["b"], ws["v"], ws["g"])
-            units = n_s * w.B
-        dt = time.perf_counter() - t0
-        if dt >= budget_s or n_s >= w.n:
-            return units / dt, f"{w.op} n={n_s} (same recipe, seed 123), sort+fwd+bwd in fp64, {dt:.2f} s"
+        _, dt = oracle_pass(w, oracle_inputs(w, n_s))
+        if dt >= 0.5 * budget_s or n_s >= w.n:
+            return n_s
         n_s = min(w.n, n_s * max(2, int(budget_s / max(dt, 1e-3))))
+
+
+def oracle_sample(w, budget_s: float):
+    """The oracle's throughput on a bounded sample of about budget_s.  Returns
+    (elements/s, description)."""
+    n_s = oracle_sample_size(w, budget_s)
+    units, dt = oracle_pass(w, oracle_inputs(w, n_s))
+    return units / dt, f"{w.op} n={n_s} B={w.B} (same recipe, seed 123), sort+fwd+bwd in fp64, {dt:.2f} s timed"
 
 
 def cpu_model() -> str:
@@ -336,6 +394,114 @@ def cpu_model() -> str:
     except OSError:
         pass
     return "unknown"
+
+
+# ------------------------------------------------------------------ measurement
+
+# the other workloads measured inside the default run (nested under "configs")
+NESTED = ("small", "phased_head", "gram_image", "gram_image_full", "sym1e9")
+
+
+def config_of(w, args_workload: str, world: int) -> dict:
+    """The line's config (the reference arm prints the same one)."""
+    return {"workload": args_workload, "op": w.op, "n": w.n, "k": w.k, "B": w.B, "mode": "train (re-sort)",
+            "l2": "per-step inputs > 126 MB L2, no flush" if w.n * w.B * 4 > (126 << 20)
+            else "inputs fit in the 126 MB L2 (latency-bound size), no flush",
+            "parallelism": f"dp{world}" if world > 1 else "1 GPU"}
+
+
+def roofline_of(prof: dict, w, steps: int, workload: str, peak_gbs: float, peak_kind: str):
+    """Roofline of the kernel with the largest share of the step: the method's bytes
+    (and the design's) per launch over its average CUDA-event launch time."""
+    if not prof:
+        return None
+    name, (cnt, tot_ms) = max(prof.items(), key=lambda kv: kv[1][1])
+    per_step = kernel_bytes_per_step(name, w)
+    if per_step is None:
+        return {"kernel": name, "bound": "hbm", "achieved": None, "peak": peak_gbs, "unit": "GB/s", "frac": None,
+                "traffic": None, "note": "no byte count for this kernel"}
+    launches_per_step = cnt / steps
+    avg_ms = tot_ms / cnt
+    m_pl, d_pl = per_step[0] / launches_per_step, per_step[1] / launches_per_step
+    ach = m_pl / (avg_ms * 1e-3) / 1e9
+    dach = d_pl / (avg_ms * 1e-3) / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": peak_gbs, "unit": "GB/s",
+            "frac": round(ach / peak_gbs, 4), "traffic": recorded_traffic(name, workload),
+            "algorithmic_bytes_per_launch": int(m_pl), "bytes": "the method's own data (sorted anchors, "
+            "permutation, input and output vectors and gradients) per launch",
+            "design_bytes_per_launch": int(d_pl), "design_achieved": round(dach, 1),
+            "design_frac": round(dach / peak_gbs, 4), "avg_launch_ms": round(avg_ms, 5),
+            "launches_per_step": launches_per_step, "peak_source": peak_kind}
+
+
+def measure_workload(L, st, w, workload: str, device, torch, steps: int, warmup: int, timed, peak):
+    """Train (re-sort) and cached-sort timings, the per-kernel profile and the
+    dominant kernel's roofline of one workload; peak device memory of its step."""
+    from structured_trainable_laplace_b200 import dp
+
+    def train_step():
+        st.sort()
+        return dp.allreduce_param_grads(st.compute())
+
+    for _ in range(warmup):
+        train_step()
+    L.check()
+    ms_train = timed(train_step, steps)
+    L.check()
+    st.sort()
+    ms_infer = timed(lambda: dp.allreduce_param_grads(st.compute()), steps)
+    L.profile_enable(True)
+    ms_prof = timed(train_step, steps)
+    prof = L.profile_report()
+    L.profile_enable(False)
+    L.check()
+    comp = compulsory_bytes(w)
+    return {
+        "ms_per_step": round(ms_train, 4), "value": round(elements(w) / (ms_train * 1e-3), 1),
+        "infer": {"ms_per_step": round(ms_infer, 4), "value": round(elements(w) / (ms_infer * 1e-3), 1)},
+        "hbm": {"compulsory_bytes_per_step": comp, "achieved_gbs": round(comp / (ms_train * 1e-3) / 1e9, 1),
+                "frac_of_measured": round(comp / (ms_train * 1e-3) / 1e9 / peak[0], 4),
+                "frac_of_8tbs": round(comp / (ms_train * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4)},
+        "roofline": roofline_of(prof, w, steps, workload, peak[0], peak[1]),
+        "kernels": {k: {"launches_per_step": v[0] / steps, "ms_per_step": round(v[1] / steps, 5)}
+                    for k, v in sorted(prof.items(), key=lambda kv: -kv[1][1])},
+        "profiled_ms_per_step": round(ms_prof, 4),
+        "gpu_launches": int(sum(v[0] for v in prof.values())),
+    }, train_step
+
+
+def nested_config(L, name: str, device, torch, timed, peak, steps: int) -> dict:
+    """One of the other workloads, measured inside the default run: the same
+    train / cached-sort / per-kernel measurement as the headline, with the peak
+    device memory of its step (the inputs, outputs, sorted anchors, saved state and
+    workspace).  The n = 10^9 inputs are drawn on the device (torch's seeded
+    generator, the same distributions as the host recipe); the others come from the
+    host recipe.  No end-to-end leg: the headline carries it."""
+    gc = __import__("gc")
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    torch.cuda.reset_peak_memory_stats(device)
+    base = torch.cuda.memory_allocated(device)
+    if name == "sym1e9":
+        w, tensors = inputs.device_symmetric(10 ** 9, 1, device, seed=0, name="sym_n1000000000_b1")
+        st = Step(L, w, device, torch, tensors)
+        how = "drawn on the device (torch generator, seed 0): a ~ U[0, 0.05 n], x, g ~ N(0, 1)"
+    else:
+        w = make_workload(name, 0)
+        st = Step(L, w, device, torch)
+        how = "host recipe (structured_trainable_laplace_b200.inputs, seed 0)"
+    res, _ = measure_workload(L, st, w, name, device, torch, steps, 3, timed, peak)
+    res["peak_mem_gb"] = round((torch.cuda.max_memory_allocated(device) - base) / 1e9, 2)
+    res["hbm_gb"] = 180
+    res["config"] = config_of(w, name, 1)
+    res["inputs"] = how
+    res["steps"] = steps
+    del st
+    gc.collect()
+    L.release_workspace()
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------ main
@@ -350,6 +516,8 @@ def main():
                     choices=["sym2p24", "small", "phased_head", "gram_image", "gram_image_full", "sym1e9"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle CPU time")
     ap.add_argument("--n", type=int, default=None, help="large-side anchors (profiling captures of a smaller case)")
+    ap.add_argument("--configs", default="auto", choices=["auto", "none"],
+                    help="auto: the default single-GPU run also measures the other workloads (nested)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -379,9 +547,6 @@ def main():
         st.sort()
         return dp.allreduce_param_grads(st.compute())
 
-    def infer_step():
-        return dp.allreduce_param_grads(st.compute())
-
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
@@ -403,6 +568,7 @@ def main():
             ms = float(tt.item())
         return ms
 
+    peak = measured_peak()
     for _ in range(args.warmup):
         train_step()
     L.check()
@@ -419,10 +585,8 @@ def main():
     clocks = summarize_clocks(clk_path, local)
     L.check()
 
-    # inference mode: cached sort
-    st.sort()
-    ms_infer = timed(infer_step, args.steps)
-
+    # cached sort, per-kernel profile and roofline (the same train steps again)
+    head, _ = measure_workload(L, st, w, args.workload, device, torch, args.steps, 1, timed, peak)
     peak_mem = torch.cuda.max_memory_allocated(device) / 1e9  # the device-resident step
 
     # the same train step captured once as a CUDA graph and replayed: every call of
@@ -451,19 +615,11 @@ def main():
         torch.cuda.synchronize(device)
         st.sort()
 
-    # the same train steps with every kernel bracketed by CUDA events
-    L.profile_enable(True)
-    ms_prof = timed(train_step, args.steps)
-    prof = L.profile_report()
-    L.profile_enable(False)
-    L.check()
-
     # training with a warm-start re-sort: the anchors alternate between two sets
     # one update apart (a and a + WARM_MOVE * N(0, 1)); each step re-sorts from the
     # previous step's permutation, then runs the same forward + backward
     warm = None
     if w.op == "sym" and w.n <= WARM_MAX_N:
-        from structured_trainable_laplace_b200 import inputs
         anchors = [st.t["a"], torch.from_numpy(inputs.moved(w.arrays["a"], WARM_MOVE, seed=1)).to(device)]
         path = torch.zeros(1, dtype=torch.int32, device=device)
         paths = []
@@ -491,6 +647,7 @@ def main():
                 "move": f"anchors alternate between a and a + {WARM_MOVE} * N(0, 1) (mean spacing 0.05)",
                 "paths_seen": sorted({L.RESORT_PATHS[q] for q in paths})}
         warm["full_sort_ms"] = round(timed(lambda: L.sort_anchors(anchors[0]), args.steps), 4)
+        del anchors
         st.sort()
 
     torch.cuda.reset_peak_memory_stats(device)  # the end-to-end leg's own peak below
@@ -503,6 +660,7 @@ def main():
     host_in = {key: torch.from_numpy(np.ascontiguousarray(v)).pin_memory() for key, v in w.arrays.items()}
     outs = train_step()
     host_out = {key: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for key, v in outs.items()}
+    del outs
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
     s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
@@ -542,52 +700,51 @@ def main():
 
     units = elements(w) * world
     value = units / (ms_train * 1e-3)
-    peak_gbs, peak_kind = measured_peak()
     comp = compulsory_bytes(w)
-
-    # dominant kernel of the step and its roofline
-    dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
-    roof = None
-    launches_total = sum(v[0] for v in prof.values()) if prof else 0
-    if dom is not None:
-        name, (cnt, tot_ms) = dom
-        avg_ms = tot_ms / cnt
-        bpl = kernel_bytes_per_launch(name, w)
-        if bpl is not None:
-            achieved = bpl / (avg_ms * 1e-3) / 1e9
-            traffic = recorded_traffic(name, args.workload)
-            roof = {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak_gbs,
-                    "unit": "GB/s", "frac": round(achieved / peak_gbs, 4), "traffic": traffic,
-                    "algorithmic_bytes_per_launch": bpl, "avg_launch_ms": round(avg_ms, 5),
-                    "peak_source": peak_kind}
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_train, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; anchors shared, vectors per rank)",
-        "config": {"workload": args.workload, "op": w.op, "n": w.n, "k": w.k, "B": w.B, "mode": "train (re-sort)",
-                   "l2": "per-step inputs > 126 MB L2, no flush", "parallelism": f"dp{world}" if world > 1 else "1 GPU"},
-        "infer": {"value": round(units / (ms_infer * 1e-3), 1), "ms_per_step": round(ms_infer, 4)},
+        "config": config_of(w, args.workload, world),
+        "infer": {"value": round(units / (head["infer"]["ms_per_step"] * 1e-3), 1),
+                  "ms_per_step": head["infer"]["ms_per_step"]},
         "hbm": {"compulsory_bytes_per_step": comp, "achieved_gbs": round(comp / (ms_train * 1e-3) / 1e9, 1),
-                "frac_of_measured": round(comp / (ms_train * 1e-3) / 1e9 / peak_gbs, 4),
+                "frac_of_measured": round(comp / (ms_train * 1e-3) / 1e9 / peak[0], 4),
                 "frac_of_8tbs": round(comp / (ms_train * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 4)},
-        "e2e": {"value": round(units / (ms_e2e * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "schedule": "copies of step k+1 and k-1 overlap step k",
-                "d2h_bytes_per_step": d2h, "ms_per_step": round(ms_e2e, 4)},
-        "roofline": roof,
+        "e2e": {"value": round(units / (ms_e2e * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "schedule": "copies of step k+1 and k-1 overlap step k", "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(ms_e2e, 4)},
+        "roofline": head["roofline"],
         "train_warm_start": warm,
         "train_graph": graph,
-        "kernels": {kname: {"launches_per_step": v[0] / args.steps, "ms_per_step": round(v[1] / args.steps, 5)}
-                    for kname, v in sorted(prof.items(), key=lambda kv: -kv[1][1])},
-        "profiled_ms_per_step": round(ms_prof, 4),
-        "gpu_launches": int(launches_total),
+        "kernels": head["kernels"],
+        "profiled_ms_per_step": head["profiled_ms_per_step"],
+        "gpu_launches": head["gpu_launches"],
         "clocks": clocks,
         "peak_mem_gb": round(peak_mem, 2),
         "peak_mem_e2e_gb": round(peak_mem_e2e, 2),
     }
+    del bufs, host_in, host_out, st
+    L.release_workspace()
     if rank == 0 and world == 1:
         v, desc = oracle_sample(w, args.cpu_budget)
         result["cpu_baseline"] = {"value": round(v, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                                   "cpu": cpu_model()}
+    if world == 1 and args.configs == "auto" and args.workload == "sym2p24" and args.n is None:
+        result["configs"] = {}
+        for name in NESTED:
+            try:
+                result["configs"][name] = nested_config(L, name, device, torch, timed, peak,
+                                                        steps=5 if name == "sym1e9" else 20)
+            except Exception as e:  # recorded in the line, not fatal to the headline
+                result["configs"][name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+                L.release_workspace()
+                torch.cuda.empty_cache()
+        result["configs_note"] = ("the other workloads, measured in this run after the headline: train "
+                                  "(re-sort) and cached-sort steps, per-kernel CUDA-event profile, the dominant "
+                                  "kernel's roofline, peak device memory of the step against 180 GB; no "
+                                  "end-to-end leg for these (the headline carries it)")
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -595,24 +752,33 @@ def main():
 
 
 def reference_arm(args, world, rank):
-    """The fp64 oracle, as it stands, on the host cores; rank 0 only."""
+    """The fp64 oracle, as it stands, on the host cores; rank 0 only.  Each step is
+    one oracle pass (sort + forward + backward) over a fixed bounded sample of the
+    workload, sized once so that the warm-up and timed steps together take about
+    two minutes; ms_per_step is the measured time of one such step."""
     if rank != 0:
         return
     w = make_workload(args.workload, 0, args.n)
-    per_step = []
-    desc = ""
+    per_step_s = min(args.cpu_budget, 120.0 / max(1, args.steps + args.warmup))
+    n_s = oracle_sample_size(w, per_step_s)
+    ws = oracle_inputs(w, n_s)
     for _ in range(args.warmup):
-        oracle_sample(w, min(2.0, args.cpu_budget / 4))
+        oracle_pass(w, ws)
+    units, secs = 0, 0.0
     for _ in range(args.steps):
-        v, desc = oracle_sample(w, min(4.0, args.cpu_budget / 2))
-        per_step.append(v)
-    v = float(np.median(per_step))
-    units = elements(w)
+        u, dt = oracle_pass(w, ws)
+        units += u
+        secs += dt
+    v = units / secs
+    ms = secs / args.steps * 1e3
+    desc = (f"{w.op} n={n_s} B={w.B} per step (a bounded sample of the n={w.n} workload, same recipe, seed 123); "
+            f"{args.steps} timed steps took {secs:.2f} s of fp64 sort+fwd+bwd")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(v, 1), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(units / v * 1e3, 2),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "op": w.op, "n": w.n, "k": w.k, "B": w.B},
+        "config": config_of(w, args.workload, world),
+        "sample": {"n": n_s, "B": w.B, "elements_per_step": n_s * w.B, "timed_s": round(secs, 3)},
         "cpu_baseline": {"value": round(v, 1), "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
                          "cpu": cpu_model()},
         "e2e": {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -168,6 +168,24 @@ def rectangular(n: int, k: int, B: int, seed: int = 0, span_a: float = 100.0, sp
     return Workload(name, op, n, B, k, arrays)
 
 
+def device_symmetric(n: int, B: int, device, seed: int = 0, spacing: float = 0.05, name: str = "symmetric"):
+    """The symmetric recipe (a ~ U[0, spacing*n], x, g ~ N(0,1) [n][B]) drawn
+    directly on a CUDA device with torch's seeded generator, for sizes whose host
+    draw and upload would take longer than the measurement (n = 10^9).  Same
+    distributions as ``symmetric`` (not the same numbers).  Returns (Workload
+    without host arrays, dict of device tensors a, x, g)."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    a = torch.empty(n, dtype=torch.float32, device=device)
+    a.uniform_(0.0, spacing * n, generator=gen)
+    x = torch.empty((n, B), dtype=torch.float32, device=device)
+    x.normal_(generator=gen)
+    g = torch.empty((n, B), dtype=torch.float32, device=device)
+    g.normal_(generator=gen)
+    return Workload(name, "sym", n, B, 0, {}), {"a": a, "x": x, "g": g}
+
+
 # The five named workloads.  Sizes and distributions are the ones stated for each.
 def sym_small_ties(seed: int = 0) -> Workload:
     """n=4096, a ~ U[0, 0.05n] with 5% overwritten by copies of other anchors, B=1."""

@@ -31,13 +31,51 @@ def test_compulsory_bytes_of_the_symmetric_step(bench):
     assert bench.compulsory_bytes(wl("sym", n, B)) == expect == 5905580032
 
 
-def test_kernel_bytes_per_launch(bench):
-    w = wl("sym", 1 << 24, 16)
-    assert bench.kernel_bytes_per_launch("sym_agg", w) == (8 + 64 + 64) * (1 << 24)
-    assert bench.kernel_bytes_per_launch("sym_bwd", w) == (8 + 64 * 3 + 4) * (1 << 24)
-    assert bench.kernel_bytes_per_launch("no_such_kernel", w) is None
+def test_kernel_bytes_per_step(bench):
+    n, B = 1 << 24, 16
+    w = wl("sym", n, B)
+    # the aggregate pass runs on x and on g: the method's bytes are the sorted
+    # anchors, the permutation and the gathered rows; the design adds the sorted copy
+    assert bench.kernel_bytes_per_step("sym_agg", w) == (2 * (8 + 64) * n, 2 * (8 + 128) * n)
+    assert bench.kernel_bytes_per_step("sym_bwd", w) == ((8 + 64 + 4) * n, (8 + 64 * 3 + 4) * n)
+    assert bench.kernel_bytes_per_step("radix_pass", w) == (8 * n, 60 * n)
+    assert bench.kernel_bytes_per_step("no_such_kernel", w) is None
+    # summed over the kernels, the method's bytes are the compulsory bytes less the
+    # backward's second read of x (it reads the forward's saved sorted copy) plus
+    # the second reads of the sorted anchors and permutation by the sweeps
+    names = ("sym_agg", "sym_fwd", "sym_bwd", "radix_pass", "radix_hist")
+    total = sum(bench.kernel_bytes_per_step(k, w)[0] for k in names)
+    assert total == bench.compulsory_bytes(w) - 4 * B * n + 16 * n == 304 * n
     g = wl("gram", 3 << 20, 8, 65536)
-    assert bench.kernel_bytes_per_launch("large_accum", g) == (8 + 64) * (3 << 20)  # paired v and g rows
+    assert bench.kernel_bytes_per_step("large_accum", g) == ((8 + 64) * (3 << 20),) * 2  # paired v and g rows
+    # both sorts of the Gram operator are radix sorts (k > 8192): the step's radix
+    # bytes cover both
+    assert bench.kernel_bytes_per_step("radix_pass", g) == (8 * ((3 << 20) + 65536), 60 * ((3 << 20) + 65536))
+    h = wl("phased_transpose", 1 << 22, 128, 1024)
+    assert bench.kernel_bytes_per_step("sort_small", h) == (12 * 1024, 12 * 1024)  # k <= 8192: counting sort
+    one = wl("sym", 10 ** 9, 1)
+    assert bench.kernel_bytes_per_step("unpermute_place", one) == (12 * 10 ** 9, 36 * 10 ** 9)
+
+
+def test_roofline_of_the_dominant_kernel(bench):
+    n, B = 1 << 24, 16
+    w = wl("sym", n, B)
+    steps = 10
+    prof = {"sym_agg": (2 * steps, 2 * steps * 0.6), "sym_bwd": (steps, steps * 1.0), "radix_pass": (40, 5.0)}
+    r = bench.roofline_of(prof, w, steps, "sym2p24", 6549.1, "measured")
+    assert r["kernel"] == "sym_agg" and r["launches_per_step"] == 2
+    assert r["algorithmic_bytes_per_launch"] == (8 + 64) * n
+    assert r["design_bytes_per_launch"] == (8 + 128) * n
+    assert abs(r["achieved"] - (8 + 64) * n / 0.6e-3 / 1e9) < 0.1
+    assert abs(r["frac"] - r["achieved"] / 6549.1) < 1e-4 and r["design_frac"] > r["frac"]
+    assert bench.roofline_of({}, w, steps, "sym2p24", 6549.1, "measured") is None
+
+
+def test_reference_arm_config_matches(bench):
+    w = wl("sym", 1 << 24, 16)
+    c = bench.config_of(w, "sym2p24", 1)
+    assert c == bench.config_of(w, "sym2p24", 1) and c["workload"] == "sym2p24" and c["B"] == 16
+    assert "no flush" in c["l2"]
 
 
 def test_traffic_records_follow_the_kernel_sources(bench, tmp_path, monkeypatch):
