@@ -64,6 +64,16 @@ cudaError_t launch_resort(const float* a, int64_t n, const uint32_t* perm_prev, 
 // overwritten (it holds the regrouped values of the last split).
 size_t unpermute_workspace_bytes(int64_t n);
 cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* out, void* ws, cudaStream_t stream);
+// The same placement out[dest[i]] = v[i] with v left alone: v2 (n floats) holds the
+// second split's values.  v == nullptr places the positions themselves (v[i] = i,
+// uint32 bits in the float slots).
+cudaError_t launch_place(const uint32_t* dest, const float* v, int64_t n, float* out, void* ws, float* v2,
+                         cudaStream_t stream);
+// inv[perm[r]] = r: the inverse permutation, by the same placement (v2: n floats
+// of scratch).  With it a gather v[perm[r]] into sorted order becomes the placement
+// out[inv[i]] = v[i], which reads v in order.
+cudaError_t launch_inverse_perm(const uint32_t* perm, int64_t n, uint32_t* inv, void* ws, float* v2,
+                                cudaStream_t stream);
 
 // sym.cu
 size_t sym_workspace_bytes(int64_t n, int64_t B);

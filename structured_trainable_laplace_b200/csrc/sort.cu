@@ -314,6 +314,9 @@ constexpr int kPlaceMaxWindow = 1 << 14;  // floats of a window placed in shared
 // second pass's tiles lie inside one first-pass bucket).  Per-bucket counts
 // (shared atomics), a block scan into per-bucket starts, one global cursor claim
 // per bucket, then runs of equal buckets leave as contiguous stores.
+// IOTA: the values are the pairs' own positions (their uint32 bits in a float
+// slot), not read from v_in: out[p[i]] = i builds the inverse permutation.
+template <bool IOTA>
 __global__ void __launch_bounds__(kNT, 4) k_bucket_split(const uint32_t* __restrict__ p_in, const float* __restrict__ v_in,
                                                       int64_t n, int shift, uint32_t* cursor, uint32_t* __restrict__ p_out,
                                                       float* __restrict__ v_out) {
@@ -335,15 +338,21 @@ __global__ void __launch_bounds__(kNT, 4) k_bucket_split(const uint32_t* __restr
         const int64_t idx0 = base + (int64_t)q * 4 * kNT + 4 * tid;
         if (full) {
             const uint4 p4 = __ldcs(reinterpret_cast<const uint4*>(p_in + idx0));
-            const float4 v4 = __ldcs(reinterpret_cast<const float4*>(v_in + idx0));
             pv[4 * q] = p4.x, pv[4 * q + 1] = p4.y, pv[4 * q + 2] = p4.z, pv[4 * q + 3] = p4.w;
-            vv[4 * q] = v4.x, vv[4 * q + 1] = v4.y, vv[4 * q + 2] = v4.z, vv[4 * q + 3] = v4.w;
+            if (!IOTA) {
+                const float4 v4 = __ldcs(reinterpret_cast<const float4*>(v_in + idx0));
+                vv[4 * q] = v4.x, vv[4 * q + 1] = v4.y, vv[4 * q + 2] = v4.z, vv[4 * q + 3] = v4.w;
+            }
         } else {
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 pv[4 * q + u] = idx0 + u < n ? __ldcs(p_in + idx0 + u) : 0u;
-                vv[4 * q + u] = idx0 + u < n ? __ldcs(v_in + idx0 + u) : 0.f;
+                if (!IOTA) vv[4 * q + u] = idx0 + u < n ? __ldcs(v_in + idx0 + u) : 0.f;
             }
+        }
+        if (IOTA) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) vv[4 * q + u] = __uint_as_float((uint32_t)(idx0 + u));
         }
     }
 #pragma unroll
@@ -419,7 +428,8 @@ __global__ void __launch_bounds__(kNT) k_place_window(const uint32_t* __restrict
     for (int i = (cnt / 4) * 4 + threadIdx.x; i < cnt; i += kNT) __stcs(out + w0 + i, s_win[i]);
 }
 
-// out[p[i]] = v[i], i in order, for windows too large for shared memory.
+// out[p[i]] = v[i] (v null: the position i itself, as uint32 bits), i in order,
+// for windows too large for shared memory.
 __global__ void __launch_bounds__(kNT) k_scatter_pairs(const uint32_t* __restrict__ p, const float* __restrict__ v,
                                                        int64_t n, float* __restrict__ out) {
     const int64_t stride = (int64_t)gridDim.x * kNT * 4;
@@ -429,7 +439,7 @@ __global__ void __launch_bounds__(kNT) k_scatter_pairs(const uint32_t* __restric
             const int64_t i = i0 + u * kNT;
             if (i < n) {
                 const uint32_t d = __ldcs(p + i);
-                if ((int64_t)d < n) out[d] = __ldcs(v + i);
+                if ((int64_t)d < n) out[d] = v != nullptr ? __ldcs(v + i) : __uint_as_float((uint32_t)i);
             }
         }
     }
@@ -442,6 +452,16 @@ size_t unpermute_workspace_bytes(int64_t n) {
 }
 
 cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* out, void* ws, cudaStream_t stream) {
+    return launch_place(perm, v, n, out, ws, v, stream);
+}
+
+cudaError_t launch_inverse_perm(const uint32_t* perm, int64_t n, uint32_t* inv, void* ws, float* v2,
+                                cudaStream_t stream) {
+    return launch_place(perm, nullptr, n, reinterpret_cast<float*>(inv), ws, v2, stream);
+}
+
+cudaError_t launch_place(const uint32_t* perm, const float* v, int64_t n, float* out, void* ws, float* v2,
+                         cudaStream_t stream) {
     if (n <= 0) return cudaSuccess;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -466,18 +486,22 @@ cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* o
     uint32_t* p2 = (uint32_t*)q;
     q += align_up((size_t)n * 4, 256);
     uint32_t* cursor = (uint32_t*)q;  // 65536 entries
-    float* v2 = v;                    // v is read only by the first split
+    // v2 (the second split's values) may be v itself: v is read only by the first split
     const int64_t tiles = (n + kSplitTile - 1) / kSplitTile;
     const int64_t nb1 = ((n - 1) >> s1) + 1, nb2 = ((n - 1) >> s2) + 1;  // buckets of each level
     LAPLEX_TIMED("unpermute_split", stream, k_bucket_cursors<<<1, kRadix, 0, stream>>>(cursor, nb1, s1));
-    LAPLEX_TIMED("unpermute_split", stream,
-                 k_bucket_split<<<(unsigned)tiles, kNT, 0, stream>>>(perm, v, n, s1, cursor, p1, v1));
+    if (v == nullptr)
+        LAPLEX_TIMED("unpermute_split", stream,
+                     k_bucket_split<true><<<(unsigned)tiles, kNT, 0, stream>>>(perm, nullptr, n, s1, cursor, p1, v1));
+    else
+        LAPLEX_TIMED("unpermute_split", stream,
+                     k_bucket_split<false><<<(unsigned)tiles, kNT, 0, stream>>>(perm, v, n, s1, cursor, p1, v1));
     // bucket q of the first level fills [q << s1, (q + 1) << s1) and 2^s1 is a
     // multiple of the tile, so every second-level tile lies inside one of them
     LAPLEX_TIMED("unpermute_split", stream,
                  k_bucket_cursors<<<(unsigned)((nb2 + kNT - 1) / kNT), kNT, 0, stream>>>(cursor, nb2, s2));
     LAPLEX_TIMED("unpermute_split", stream,
-                 k_bucket_split<<<(unsigned)tiles, kNT, 0, stream>>>(p1, v1, n, s2, cursor, p2, v2));
+                 k_bucket_split<false><<<(unsigned)tiles, kNT, 0, stream>>>(p1, v1, n, s2, cursor, p2, v2));
     if ((1ll << s2) <= kPlaceMaxWindow) {
         static PerDevice ready;
         if (!ready.here()) {

@@ -68,3 +68,27 @@ def test_two_splits_and_windows_permute(n):
     ref = np.empty(n, np.float32)
     ref[perm] = v
     np.testing.assert_array_equal(out, ref)
+
+
+@pytest.mark.parametrize("n", [(1 << 20) + 4097, 3 << 19])
+def test_inverse_permutation_turns_the_gather_into_a_placement(n):
+    """The gather xs[r] = x[perm[r]] of the single-channel path past 2^24 rows: the
+    placement with positions as values builds inv (inv[perm[r]] = r), and the
+    placement out[inv[i]] = x[i], which reads x in order, equals the gather."""
+    rng = np.random.default_rng(n + 1)
+    perm = rng.permutation(n).astype(np.uint32)
+    x = rng.standard_normal(n).astype(np.float32)
+    bits = int(np.ceil(np.log2(n)))
+    s2 = max(bits - 16, 0)
+    s1 = s2 + 8
+    tile = min(TILE, 1 << s1)
+
+    def placed(dest, vals):
+        p1, v1 = split(dest, vals, s1, tile)
+        p2, v2 = split(p1, v1, s2, tile)
+        return place(p2, v2, s2)
+
+    iota = np.arange(n, dtype=np.uint32).view(np.float32)  # positions as uint32 bits
+    inv = placed(perm, iota).view(np.uint32)
+    np.testing.assert_array_equal(inv[perm], np.arange(n, dtype=np.uint32))
+    np.testing.assert_array_equal(placed(inv, x), x[perm])
