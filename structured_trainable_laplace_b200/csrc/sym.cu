@@ -928,6 +928,9 @@ __device__ __forceinline__ void cross_warps1(Cross1<NV>& cx) {
 
 // Aggregate pass for one channel: walks its base ranges' tiles right to left,
 // writes the sorted copy, RS and the range aggregates (as k_sym_agg).
+// SORTED_IN: the sorted copy vs already holds the values in sorted order (placed
+// there through the inverse permutation); it is read, the permutation is not.
+template <bool SORTED_IN>
 __global__ void __launch_bounds__(k1NT, 3) k_sym1_agg(SymScan a, const float* __restrict__ v, RangeState st,
                                                      float* __restrict__ vs) {
     __shared__ Cross1<1> cx;
@@ -938,11 +941,23 @@ __global__ void __launch_bounds__(k1NT, 3) k_sym1_agg(SymScan a, const float* __
     for (int64_t t = w.te - 1; t >= w.tb; --t) {
         const int64_t lo = t * (int64_t)k1R, J = t / a.tpr;
         Rows1 r;
-        load_rows1(a.s, a.perm, a.n, lo + threadIdx.x * k1E, r);
+        load_rows1<!SORTED_IN>(a.s, a.perm, a.n, lo + threadIdx.x * k1E, r);
         float x[k1E];
+        if (SORTED_IN) {
+            if (r.row0 + k1E <= a.n) {
+                const float4* src = reinterpret_cast<const float4*>(vs + r.row0);
 #pragma unroll
-        for (int e = 0; e < k1E; ++e) x[e] = (r.row0 + e < a.n) ? __ldg(v + r.p[e]) : 0.f;
-        {
+                for (int q = 0; q < k1E / 4; ++q) {
+                    const float4 f = __ldcs(src + q);
+                    x[4 * q] = f.x, x[4 * q + 1] = f.y, x[4 * q + 2] = f.z, x[4 * q + 3] = f.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < k1E; ++e) x[e] = (r.row0 + e < a.n) ? __ldcs(vs + r.row0 + e) : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < k1E; ++e) x[e] = (r.row0 + e < a.n) ? __ldg(v + r.p[e]) : 0.f;
             float4* dst = reinterpret_cast<float4*>(vs + r.row0);
 #pragma unroll
             for (int q = 0; q < k1E / 4; ++q) __stcs(dst + q, make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]));
@@ -1187,8 +1202,10 @@ struct SymPlan {
     size_t state_bytes;          // RS, Lin, Rin, Lagg, Ragg of one vector
     size_t saved_state_bytes;    // RS, Lin, Rin of one vector
     size_t sorted_bytes;         // sorted copy of one vector (G * T * R * C floats)
-    bool bucketed;               // one channel past the L2: outputs leave through launch_unpermute
+    bool bucketed;               // one channel past the L2: outputs leave through launch_unpermute and the
+                                 // inputs enter through the inverse permutation (launch_place)
     size_t unperm_bytes;         // two sorted-order outputs + the unpermute scratch
+    size_t inv_bytes;            // the inverse permutation (bucketed only)
     size_t total;
 };
 
@@ -1213,7 +1230,8 @@ SymPlan plan_sym(int64_t n, int64_t B, int sms) {
     // than the L2 are written in sorted order and regrouped by destination instead
     p.bucketed = (p.C == 1 && n > kUnpermuteMinRows);
     p.unperm_bytes = p.bucketed ? 2 * align_up(sizeof(float) * (size_t)n, 256) + unpermute_workspace_bytes(n) : 0;
-    p.total += p.unperm_bytes;
+    p.inv_bytes = p.bucketed ? align_up(sizeof(uint32_t) * (size_t)n, 256) : 0;
+    p.total += p.unperm_bytes + p.inv_bytes;  // the inverse permutation here when there is no saved buffer
     return p;
 }
 
@@ -1222,6 +1240,15 @@ SymPlan plan_sym(int64_t n, int64_t B, int sms) {
 float* unperm_outputs(const SymPlan& p, void* ws) { return (float*)((char*)ws + 2 * (p.state_bytes + p.sorted_bytes)); }
 void* unperm_scratch(const SymPlan& p, void* ws, int64_t n) {
     return (char*)unperm_outputs(p, ws) + 2 * align_up(sizeof(float) * (size_t)n, 256);
+}
+// The second sorted-order output slot, free while the inputs are placed: the
+// placement's second-split values.
+float* place_scratch(const SymPlan& p, void* ws, int64_t n) { return unperm_outputs(p, ws) + align_up((size_t)n, 64); }
+// The inverse permutation: after the saved state and sorted copy of the saved
+// buffer, or at the end of the workspace.
+uint32_t* inv_slot(const SymPlan& p, void* ws, void* saved, int64_t n) {
+    if (saved != nullptr) return (uint32_t*)((char*)saved + p.saved_state_bytes + p.sorted_bytes);
+    return (uint32_t*)((char*)unperm_scratch(p, ws, n) + unpermute_workspace_bytes(n));
 }
 
 RangeState carve(const SymPlan& p, double2* base, bool with_aggs) {
@@ -1270,15 +1297,21 @@ SymScan scan_args(const SymPlan& p, const float* s, const uint32_t* perm, int64_
 }
 
 // Pass A + pass B for one vector.
+// sorted_in (one channel): vs already holds v in sorted order (launch_place); the
+// pass reads it instead of gathering v through the permutation.
 template <int C>
 cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm, int64_t n, int64_t B, int sms,
-                         const float* v, RangeState st, float* vs, cudaStream_t stream) {
+                         const float* v, RangeState st, float* vs, cudaStream_t stream, bool sorted_in = false) {
     if constexpr (C == 1) {
-        static PerDevice occ_cache;
-        const int occ = prepare(k_sym1_agg, k1NT, 0, occ_cache.here());
+        static PerDevice occ_cache[2];
+        const int occ = sorted_in ? prepare(k_sym1_agg<true>, k1NT, 0, occ_cache[1].here())
+                                  : prepare(k_sym1_agg<false>, k1NT, 0, occ_cache[0].here());
         const SymScan a = scan_args(p, s, perm, n, B, sms, occ);
         const dim3 grid((unsigned)((p.P + a.m - 1) / a.m), 1u);
-        LAPLEX_TIMED("sym_agg", stream, k_sym1_agg<<<grid, k1NT, 0, stream>>>(a, v, st, vs));
+        if (sorted_in)
+            LAPLEX_TIMED("sym_agg", stream, k_sym1_agg<true><<<grid, k1NT, 0, stream>>>(a, v, st, vs));
+        else
+            LAPLEX_TIMED("sym_agg", stream, k_sym1_agg<false><<<grid, k1NT, 0, stream>>>(a, v, st, vs));
     } else {
         using SM = AggSmem<C, kAheadAgg>;
         static PerDevice occ_cache;
@@ -1338,6 +1371,19 @@ cudaError_t launch_sym_sweep_fwd(const SymPlan& p, const float* s, const uint32_
     return cudaGetLastError();
 }
 
+// One channel past 2^24 rows: v enters the sorted copy vs through the inverse
+// permutation, vs[inv[i]] = v[i] (a bucketed placement that reads v in order,
+// instead of one random 4-byte gather per row); the rows of the last tile past n
+// are zeroed, as the gathering pass would have written them.
+cudaError_t place_sorted1(const SymPlan& p, const uint32_t* inv, int64_t n, const float* v, float* vs, void* ws,
+                          cudaStream_t st) {
+    cudaError_t e = launch_place(inv, v, n, vs, unperm_scratch(p, ws, n), place_scratch(p, ws, n), st);
+    if (e != cudaSuccess) return e;
+    const int64_t padded = p.T * p.R;
+    if (padded > n) e = cudaMemsetAsync(vs + n, 0, sizeof(float) * (size_t)(padded - n), st);
+    return e;
+}
+
 template <int C>
 cudaError_t sym_forward_t(const float* s, const uint32_t* perm, int64_t n, const float* x, int64_t B, float* y,
                           void* saved, void* ws, cudaStream_t st) {
@@ -1352,7 +1398,17 @@ cudaError_t sym_forward_t(const float* s, const uint32_t* perm, int64_t n, const
         sx.Rin = sv.Rin;
         xs = (float*)((char*)saved + p.saved_state_bytes);
     }
-    cudaError_t e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
+    cudaError_t e;
+    if (C == 1 && p.bucketed) {
+        // the inverse permutation (kept with the saved state for the backward), then
+        // x placed into sorted order
+        uint32_t* inv = inv_slot(p, ws, saved, n);
+        e = launch_inverse_perm(perm, n, inv, unperm_scratch(p, ws, n), place_scratch(p, ws, n), st);
+        if (e == cudaSuccess) e = place_sorted1(p, inv, n, x, xs, ws, st);
+        if (e == cudaSuccess) e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st, true);
+    } else {
+        e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
+    }
     if (e != cudaSuccess) return e;
     return launch_sym_sweep_fwd<C>(p, s, perm, n, B, sms, xs, sx, y, st, ws);
 }
@@ -1378,12 +1434,27 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
         e = cudaMemsetAsync(ga, 0, sizeof(float) * n, st);
         if (e != cudaSuccess) return e;
     }
-    if (saved == nullptr) {
-        e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
+    if (C == 1 && p.bucketed) {
+        // the forward's inverse permutation (saved), or a new one; x (without a saved
+        // buffer) and g placed into sorted order
+        uint32_t* inv = inv_slot(p, ws, const_cast<void*>(saved), n);
+        if (saved == nullptr) {
+            e = launch_inverse_perm(perm, n, inv, unperm_scratch(p, ws, n), place_scratch(p, ws, n), st);
+            if (e == cudaSuccess) e = place_sorted1(p, inv, n, x, xs, ws, st);
+            if (e == cudaSuccess) e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st, true);
+            if (e != cudaSuccess) return e;
+        }
+        e = place_sorted1(p, inv, n, g, gs, ws, st);
+        if (e == cudaSuccess) e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, gs, st, true);
+        if (e != cudaSuccess) return e;
+    } else {
+        if (saved == nullptr) {
+            e = sym_ranges_t<C>(p, s, perm, n, B, sms, x, sx, xs, st);
+            if (e != cudaSuccess) return e;
+        }
+        e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, gs, st);
         if (e != cudaSuccess) return e;
     }
-    e = sym_ranges_t<C>(p, s, perm, n, B, sms, g, sg, gs, st);
-    if (e != cudaSuccess) return e;
     if constexpr (C == 1) {
         static PerDevice occ_cache[2];
         const int occ = p.bucketed ? prepare(k_sym1_sweep<2, true>, k1NT, 0, occ_cache[1].here())
@@ -1420,7 +1491,7 @@ size_t sym_workspace_bytes(int64_t n, int64_t B) { return plan_sym(n, B, 1).tota
 
 size_t sym_saved_bytes(int64_t n, int64_t B) {
     const SymPlan p = plan_sym(n, B, 1);
-    return p.saved_state_bytes + p.sorted_bytes;
+    return p.saved_state_bytes + p.sorted_bytes + p.inv_bytes;
 }
 
 #define LAPLEX_SYM_DISPATCH(C_, CALL) \
