@@ -154,9 +154,11 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     // the AND over the digit's 8 bits of the ballot of lanes agreeing on that bit
     // (plus the ballot of valid lanes, so that rows past n group apart).  rank[]
     // holds the mask until the rank replaces it.
+    // rows of this warp's slice below n (32-bit from here on: a slice holds 32 * kItems)
+    const int wn = (int)max((int64_t)0, min((int64_t)(32 * kItems), n - wbase));
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
-        const bool valid = wbase + i * 32 + lane < n;
+        const bool valid = i * 32 + lane < wn;
         const uint32_t d = (key[i] >> shift) & 0xffu;
         const uint32_t vb = __ballot_sync(0xffffffffu, valid);
         uint32_t peers = valid ? vb : ~vb;
@@ -170,7 +172,7 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     }
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
-        const bool valid = wbase + i * 32 + lane < n;
+        const bool valid = i * 32 + lane < wn;
         const uint32_t d = (key[i] >> shift) & 0xffu, peers = rank[i];
         uint32_t before = 0;
         if (valid) {
@@ -201,8 +203,8 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     // place keys in shared memory in (digit, rank) order
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
-        const int64_t idx = wbase + i * 32 + lane;
-        if (idx < n) {
+        if (i * 32 + lane < wn) {
+            const int64_t idx = wbase + i * 32 + lane;
             const uint32_t d = (key[i] >> shift) & 0xffu;
             const uint32_t p = s_start[d] + s_whist[w][d] + rank[i];
             s_keys[p] = key[i];
