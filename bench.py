@@ -206,9 +206,24 @@ class Step:
         self.sorted = None
 
     def sort(self):
-        L, t = self.L, self.t
+        """Sort the anchor sets.  The two sets of a rectangular operator are
+        independent: b is sorted on a side stream while a is sorted on the current
+        one (stream-ordered calls, joined by an event before the products), so the
+        small, launch-latency-bound sort of b overlaps the large sort of a."""
+        L, t, torch = self.L, self.t, self.torch
+        if "b" not in t:
+            self.sorted = (L.sort_anchors(t["a"]), None)
+            return
+        cur = torch.cuda.current_stream(self.dev)
+        if getattr(self, "side", None) is None:
+            self.side = torch.cuda.Stream(self.dev)
+        self.side.wait_stream(cur)
+        with torch.cuda.stream(self.side):
+            sb = L.sort_anchors(t["b"])
         sa = L.sort_anchors(t["a"])
-        sb = L.sort_anchors(t["b"]) if "b" in t else None
+        cur.wait_stream(self.side)
+        for x in sb:
+            x.record_stream(cur)
         self.sorted = (sa, sb)
 
     def compute(self):
