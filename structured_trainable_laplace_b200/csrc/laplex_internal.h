@@ -111,9 +111,12 @@ cudaError_t launch_rect_forward(Side O, Side I, const float* x, int64_t B, float
 //   gx [n_in][B], gO/gI anchor gradients, gtO/gtI phase gradients (each nullable).
 // accumulate: add the anchor and phase gradients into gO, gI, gtO, gtI instead of
 // writing them (gx is always written).
+// g2 (nullable): paired rows -- channels [0, B/2) of each output-side row come from g
+// and [B/2, B) from g2 (both [m_O][B/2]), so that two products with the same anchors
+// share one backward (output side larger than the input side, unphased, no gx).
 cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g, int64_t B, const void* saved,
                                  float* gx, float* gO, float* gI, float* gtO, float* gtI, void* ws, int32_t* status,
-                                 cudaStream_t stream, bool accumulate = false);
+                                 cudaStream_t stream, bool accumulate = false, const float* g2 = nullptr);
 
 // The bounded lookback against a predecessor that never publishes (failure-
 // detection self-check): ws holds the chain, zeroed here.

@@ -1084,8 +1084,10 @@ cudaError_t launch_rect_forward(Side O, Side I, const float* x, int64_t B, float
 
 cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g, int64_t B, const void* saved,
                                  float* gx, float* gO, float* gI, float* gtO, float* gtI, void* ws, int32_t* status,
-                                 cudaStream_t st, bool accumulate) {
+                                 cudaStream_t st, bool accumulate, const float* g2) {
     const bool phased = O.theta != nullptr;
+    // paired rows: only the pass over a larger output side takes them
+    if (g2 != nullptr && (O.m <= I.m || phased || (B % 2) != 0 || gx != nullptr)) return cudaErrorInvalidValue;
     const RectPlan p = plan_rect(O.m, I.m, B, phased, ws);
     const int64_t sz = p.ms * (int64_t)p.Cb;
     if (!phased) gtO = gtI = nullptr;
@@ -1162,6 +1164,10 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
     if (mode != 0) {
         LargePass A = large_args(O, I, p, B);
         A.rows = g;
+        if (g2 != nullptr) {  // channels [0, B/2) of a row from g, [B/2, B) from g2
+            A.rows2 = g2;
+            A.Bs = (int)(B / 2);
+        }
         A.Pst = Pst;
         A.Sst = Pst ? Pst + sz : nullptr;
         A.g_anchor = gO;
@@ -1204,9 +1210,12 @@ cudaError_t launch_check_wait_bound(void* ws, int32_t* status, cudaStream_t st) 
 // The middle of the Gram backward, one warp per small-side row j: x1 = D_j w_j,
 // x2 = D_j u_j (the inputs of the general products A (D w) and A (D u)) and
 // gD_j = <u_j, w_j>.  w and u are rows of ld floats.
+// xp (nullable): [k][2B], D_j w_j followed by D_j u_j (the input of the paired
+// backward, which takes both general products at once).
 __global__ void __launch_bounds__(256) k_gram_mid2(const float* __restrict__ D, const float* __restrict__ w,
                                                    const float* __restrict__ u, int ld, float* __restrict__ x1,
-                                                   float* __restrict__ x2, float* __restrict__ gD, int64_t k, int B) {
+                                                   float* __restrict__ x2, float* __restrict__ xp,
+                                                   float* __restrict__ gD, int64_t k, int B) {
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= k) return;
     const int lane = threadIdx.x & 31;
@@ -1216,6 +1225,10 @@ __global__ void __launch_bounds__(256) k_gram_mid2(const float* __restrict__ D, 
         const float wv = __ldg(w + r * ld + c), uv = __ldg(u + r * ld + c);
         x1[r * B + c] = d * wv;
         x2[r * B + c] = d * uv;
+        if (xp != nullptr) {
+            xp[r * 2 * B + c] = d * wv;
+            xp[r * 2 * B + B + c] = d * uv;
+        }
         acc = fmaf(uv, wv, acc);
     }
     if (gD != nullptr) {
@@ -1282,10 +1295,12 @@ cudaError_t launch_gram_backward(Side A, Side Bs, const float* D, const float* v
     float* wpair = p2.rows3;           // [k][2B] (paired) or w | u ([k][B] each)
     float* x1 = p2.rows3 + 2 * kb;     // [k][B]  D w
     float* x2 = p2.rows3 + 3 * kb;     // [k][B]  D u
+    float* xp = p2.rows3 + 4 * kb;     // [k][2B] D w | D u (paired backward)
+    const bool paired = A.m > Bs.m;
     const float* w;
     const float* u;
     int ld;
-    if (A.m > Bs.m) {  // A^T v and A^T g in one paired reduce pass
+    if (paired) {  // A^T v and A^T g in one paired reduce pass
         const RectPlan pp = plan_rect(Bs.m, A.m, 2 * B, false, ws);
         const int64_t sz = pp.ms * (int64_t)pp.Cb;
         LAPLEX_TRY(reduce_parts(pp, Bs, A, v, 2 * B, pp.bufA, pp.bufA + sz, pp.bufA + 2 * sz, status, st, g));
@@ -1309,11 +1324,19 @@ cudaError_t launch_gram_backward(Side A, Side Bs, const float* D, const float* v
         u = wpair + kb;
         ld = (int)B;
     }
+    const bool need_ab = ga != nullptr || gb != nullptr;
     LAPLEX_TIMED("gram_mid", st,
-                 k_gram_mid2<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, w, u, ld, x1, x2, gD, Bs.m, (int)B));
+                 k_gram_mid2<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, w, u, ld, x1, x2,
+                                                                        (paired && need_ab) ? xp : nullptr, gD, Bs.m,
+                                                                        (int)B));
     LAPLEX_TRY(cudaGetLastError());
     if (gv != nullptr) LAPLEX_TRY(launch_rect_forward(A, Bs, x2, B, gv, nullptr, ws, status, st));  // gv = A (D u)
-    if (ga != nullptr || gb != nullptr) {
+    if (need_ab && paired) {
+        // both general products in one backward over 2B channels: inputs D w | D u at
+        // b, rows g | v at a (ga sums over all 2B channels, and so does gb)
+        LAPLEX_TRY(launch_rect_backward(A, Bs, xp, g, 2 * B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status,
+                                        st, false, v));
+    } else if (need_ab) {
         LAPLEX_TRY(launch_rect_backward(A, Bs, x1, g, B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
                                         false));
         LAPLEX_TRY(launch_rect_backward(A, Bs, x2, v, B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
