@@ -67,8 +67,16 @@ cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* o
 // The same placement out[dest[i]] = v[i] with v left alone: v2 (n floats) holds the
 // second split's values.  v == nullptr places the positions themselves (v[i] = i,
 // uint32 bits in the float slots).
+// vb, outb (both or neither): a second value per destination placed along with v
+// (outb[dest[i]] = vb[i]); v1b, v2b: n floats each for its split levels (v2b may be
+// vb itself).
 cudaError_t launch_place(const uint32_t* dest, const float* v, int64_t n, float* out, void* ws, float* v2,
-                         cudaStream_t stream);
+                         cudaStream_t stream, const float* vb = nullptr, float* outb = nullptr, float* v1b = nullptr,
+                         float* v2b = nullptr);
+// launch_unpermute of two vectors through the same permutation at once (va and vb
+// are overwritten; v1b: n floats of scratch).
+cudaError_t launch_unpermute2(const uint32_t* perm, float* va, float* vb, int64_t n, float* outa, float* outb,
+                              float* v1b, void* ws, cudaStream_t stream);
 // inv[perm[r]] = r: the inverse permutation, by the same placement (v2: n floats
 // of scratch).  With it a gather v[perm[r]] into sorted order becomes the placement
 // out[inv[i]] = v[i], which reads v in order.

@@ -318,13 +318,17 @@ constexpr int kPlaceMaxWindow = 1 << 14;  // floats of a window placed in shared
 // per bucket, then runs of equal buckets leave as contiguous stores.
 // IOTA: the values are the pairs' own positions (their uint32 bits in a float
 // slot), not read from v_in: out[p[i]] = i builds the inverse permutation.
-template <bool IOTA>
+// TWO: a second value per destination travels along (vb_in -> vb_out), read when
+// the tile is placed in shared memory (dynamic shared memory: kSplitTile floats).
+template <bool IOTA, bool TWO>
 __global__ void __launch_bounds__(kNT, 4) k_bucket_split(const uint32_t* __restrict__ p_in, const float* __restrict__ v_in,
                                                       int64_t n, int shift, uint32_t* cursor, uint32_t* __restrict__ p_out,
-                                                      float* __restrict__ v_out) {
+                                                      float* __restrict__ v_out, const float* __restrict__ vb_in,
+                                                      float* __restrict__ vb_out) {
     __shared__ uint32_t s_cnt[kRadix], s_start[kRadix], s_base[kRadix], s_scan[kNW];
     __shared__ uint32_t s_p[kSplitTile];
     __shared__ float s_v[kSplitTile];
+    extern __shared__ float s_vb[];  // TWO only
     const int tid = threadIdx.x;
     const int64_t base = (int64_t)blockIdx.x * kSplitTile;
     s_cnt[tid] = 0;
@@ -379,6 +383,7 @@ __global__ void __launch_bounds__(kNT, 4) k_bucket_split(const uint32_t* __restr
             const uint32_t q = s_start[(pv[i] >> shift) & 0xffu] + rk[i];
             s_p[q] = pv[i];
             s_v[q] = vv[i];
+            if (TWO) s_vb[q] = __ldcs(vb_in + idx);
         }
     }
     __syncthreads();
@@ -389,6 +394,7 @@ __global__ void __launch_bounds__(kNT, 4) k_bucket_split(const uint32_t* __restr
         if (dst < n) {  // always, for a permutation; a bad perm never writes out of range
             p_out[dst] = p;
             v_out[dst] = s_v[q];
+            if (TWO) vb_out[dst] = s_vb[q];
         }
     }
 }
@@ -400,26 +406,34 @@ __global__ void k_bucket_cursors(uint32_t* cursor, int64_t count, int shift) {
 
 // One CTA per window of W = 1 << shift destinations: its pairs (contiguous after
 // the splits) go to a shared-memory copy of the window, which then leaves with
-// contiguous stores.
+// contiguous stores.  TWO: a second value per destination (vb -> outb), placed in a
+// second window copy (dynamic shared memory 2 W floats).
+template <bool TWO>
 __global__ void __launch_bounds__(kNT) k_place_window(const uint32_t* __restrict__ p, const float* __restrict__ v,
-                                                      int64_t n, int shift, float* __restrict__ out) {
+                                                      int64_t n, int shift, float* __restrict__ out,
+                                                      const float* __restrict__ vb, float* __restrict__ outb) {
     extern __shared__ float s_win[];
+    float* s_win2 = s_win + ((size_t)1 << shift);
     constexpr int U = 8;  // pairs in flight per thread
     const int64_t w0 = (int64_t)blockIdx.x << shift;
     const int cnt = (int)min((int64_t)1 << shift, n - w0);
     for (int i0 = threadIdx.x; i0 < cnt; i0 += kNT * U) {
         uint32_t pp[U];
-        float vv[U];
+        float vv[U], wb[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int i = i0 + u * kNT;
             pp[u] = i < cnt ? __ldcs(p + w0 + i) : 0xffffffffu;
             vv[u] = i < cnt ? __ldcs(v + w0 + i) : 0.f;
+            if (TWO) wb[u] = i < cnt ? __ldcs(vb + w0 + i) : 0.f;
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t d = (int64_t)pp[u] - w0;
-            if (i0 + u * kNT < cnt && d >= 0 && d < cnt) s_win[d] = vv[u];
+            if (i0 + u * kNT < cnt && d >= 0 && d < cnt) {
+                s_win[d] = vv[u];
+                if (TWO) s_win2[d] = wb[u];
+            }
         }
     }
     __syncthreads();
@@ -428,12 +442,20 @@ __global__ void __launch_bounds__(kNT) k_place_window(const uint32_t* __restrict
     const float4* w4 = reinterpret_cast<const float4*>(s_win);
     for (int i = threadIdx.x; i < cnt / 4; i += kNT) __stcs(o4 + i, w4[i]);
     for (int i = (cnt / 4) * 4 + threadIdx.x; i < cnt; i += kNT) __stcs(out + w0 + i, s_win[i]);
+    if (TWO) {
+        float4* ob4 = reinterpret_cast<float4*>(outb + w0);
+        const float4* wb4 = reinterpret_cast<const float4*>(s_win2);
+        for (int i = threadIdx.x; i < cnt / 4; i += kNT) __stcs(ob4 + i, wb4[i]);
+        for (int i = (cnt / 4) * 4 + threadIdx.x; i < cnt; i += kNT) __stcs(outb + w0 + i, s_win2[i]);
+    }
 }
 
 // out[p[i]] = v[i] (v null: the position i itself, as uint32 bits), i in order,
 // for windows too large for shared memory.
 __global__ void __launch_bounds__(kNT) k_scatter_pairs(const uint32_t* __restrict__ p, const float* __restrict__ v,
-                                                       int64_t n, float* __restrict__ out) {
+                                                       int64_t n, float* __restrict__ out,
+                                                       const float* __restrict__ vb = nullptr,
+                                                       float* __restrict__ outb = nullptr) {
     const int64_t stride = (int64_t)gridDim.x * kNT * 4;
     for (int64_t i0 = (int64_t)blockIdx.x * kNT * 4 + threadIdx.x; i0 < n; i0 += stride) {
 #pragma unroll
@@ -441,7 +463,10 @@ __global__ void __launch_bounds__(kNT) k_scatter_pairs(const uint32_t* __restric
             const int64_t i = i0 + u * kNT;
             if (i < n) {
                 const uint32_t d = __ldcs(p + i);
-                if ((int64_t)d < n) out[d] = v != nullptr ? __ldcs(v + i) : __uint_as_float((uint32_t)i);
+                if ((int64_t)d < n) {
+                    out[d] = v != nullptr ? __ldcs(v + i) : __uint_as_float((uint32_t)i);
+                    if (vb != nullptr) outb[d] = __ldcs(vb + i);
+                }
             }
         }
     }
@@ -457,14 +482,21 @@ cudaError_t launch_unpermute(const uint32_t* perm, float* v, int64_t n, float* o
     return launch_place(perm, v, n, out, ws, v, stream);
 }
 
+cudaError_t launch_unpermute2(const uint32_t* perm, float* va, float* vb, int64_t n, float* outa, float* outb,
+                              float* v1b, void* ws, cudaStream_t stream) {
+    return launch_place(perm, va, n, outa, ws, va, stream, vb, outb, v1b, vb);
+}
+
 cudaError_t launch_inverse_perm(const uint32_t* perm, int64_t n, uint32_t* inv, void* ws, float* v2,
                                 cudaStream_t stream) {
     return launch_place(perm, nullptr, n, reinterpret_cast<float*>(inv), ws, v2, stream);
 }
 
 cudaError_t launch_place(const uint32_t* perm, const float* v, int64_t n, float* out, void* ws, float* v2,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, const float* vb, float* outb, float* v1b, float* v2b) {
     if (n <= 0) return cudaSuccess;
+    const bool two = vb != nullptr;
+    if (two && (v == nullptr || outb == nullptr || v1b == nullptr || v2b == nullptr)) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -477,7 +509,7 @@ cudaError_t launch_place(const uint32_t* perm, const float* v, int64_t n, float*
     const int s2 = bits > 16 ? bits - 16 : 0, s1 = s2 + 8;
     if (s1 < 12) {  // second-level tiles would straddle first-level buckets: one plain scatter
         LAPLEX_TIMED("unpermute_place", stream,
-                     k_scatter_pairs<<<scatter_grid(n), kNT, 0, stream>>>(perm, v, n, out));
+                     k_scatter_pairs<<<scatter_grid(n), kNT, 0, stream>>>(perm, v, n, out, vb, outb));
         return cudaGetLastError();
     }
     char* q = (char*)ws;
@@ -491,31 +523,57 @@ cudaError_t launch_place(const uint32_t* perm, const float* v, int64_t n, float*
     // v2 (the second split's values) may be v itself: v is read only by the first split
     const int64_t tiles = (n + kSplitTile - 1) / kSplitTile;
     const int64_t nb1 = ((n - 1) >> s1) + 1, nb2 = ((n - 1) >> s2) + 1;  // buckets of each level
+    static PerDevice ready;
+    if (!ready.here()) {
+        cudaError_t e = cudaFuncSetAttribute(k_place_window<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(sizeof(float) * kPlaceMaxWindow));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_place_window<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(2 * sizeof(float) * kPlaceMaxWindow));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_bucket_split<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(sizeof(float) * kSplitTile));
+        if (e != cudaSuccess) return e;
+        ready.here() = 1;
+    }
+    const size_t sb = two ? sizeof(float) * kSplitTile : 0;
     LAPLEX_TIMED("unpermute_split", stream, k_bucket_cursors<<<1, kRadix, 0, stream>>>(cursor, nb1, s1));
     if (v == nullptr)
         LAPLEX_TIMED("unpermute_split", stream,
-                     k_bucket_split<true><<<(unsigned)tiles, kNT, 0, stream>>>(perm, nullptr, n, s1, cursor, p1, v1));
+                     k_bucket_split<true, false><<<(unsigned)tiles, kNT, 0, stream>>>(perm, nullptr, n, s1, cursor, p1,
+                                                                                     v1, nullptr, nullptr));
+    else if (two)
+        LAPLEX_TIMED("unpermute_split", stream,
+                     k_bucket_split<false, true><<<(unsigned)tiles, kNT, sb, stream>>>(perm, v, n, s1, cursor, p1, v1,
+                                                                                      vb, v1b));
     else
         LAPLEX_TIMED("unpermute_split", stream,
-                     k_bucket_split<false><<<(unsigned)tiles, kNT, 0, stream>>>(perm, v, n, s1, cursor, p1, v1));
+                     k_bucket_split<false, false><<<(unsigned)tiles, kNT, 0, stream>>>(perm, v, n, s1, cursor, p1, v1,
+                                                                                      nullptr, nullptr));
     // bucket q of the first level fills [q << s1, (q + 1) << s1) and 2^s1 is a
     // multiple of the tile, so every second-level tile lies inside one of them
     LAPLEX_TIMED("unpermute_split", stream,
                  k_bucket_cursors<<<(unsigned)((nb2 + kNT - 1) / kNT), kNT, 0, stream>>>(cursor, nb2, s2));
-    LAPLEX_TIMED("unpermute_split", stream,
-                 k_bucket_split<false><<<(unsigned)tiles, kNT, 0, stream>>>(p1, v1, n, s2, cursor, p2, v2));
+    if (two)
+        LAPLEX_TIMED("unpermute_split", stream,
+                     k_bucket_split<false, true><<<(unsigned)tiles, kNT, sb, stream>>>(p1, v1, n, s2, cursor, p2, v2,
+                                                                                      v1b, v2b));
+    else
+        LAPLEX_TIMED("unpermute_split", stream,
+                     k_bucket_split<false, false><<<(unsigned)tiles, kNT, 0, stream>>>(p1, v1, n, s2, cursor, p2, v2,
+                                                                                      nullptr, nullptr));
     if ((1ll << s2) <= kPlaceMaxWindow) {
-        static PerDevice ready;
-        if (!ready.here()) {
-            const cudaError_t e = cudaFuncSetAttribute(k_place_window, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       (int)(sizeof(float) * kPlaceMaxWindow));
-            if (e != cudaSuccess) return e;
-            ready.here() = 1;
-        }
-        LAPLEX_TIMED("unpermute_place", stream,
-                     k_place_window<<<(unsigned)nb2, kNT, sizeof(float) << s2, stream>>>(p2, v2, n, s2, out));
+        if (two)
+            LAPLEX_TIMED("unpermute_place", stream,
+                         k_place_window<true><<<(unsigned)nb2, kNT, 2 * (sizeof(float) << s2), stream>>>(
+                             p2, v2, n, s2, out, v2b, outb));
+        else
+            LAPLEX_TIMED("unpermute_place", stream,
+                         k_place_window<false><<<(unsigned)nb2, kNT, sizeof(float) << s2, stream>>>(p2, v2, n, s2, out,
+                                                                                                   nullptr, nullptr));
     } else {
-        LAPLEX_TIMED("unpermute_place", stream, k_scatter_pairs<<<scatter_grid(n), kNT, 0, stream>>>(p2, v2, n, out));
+        LAPLEX_TIMED("unpermute_place", stream,
+                     k_scatter_pairs<<<scatter_grid(n), kNT, 0, stream>>>(p2, v2, n, out, two ? v2b : nullptr, outb));
     }
     return cudaGetLastError();
 }

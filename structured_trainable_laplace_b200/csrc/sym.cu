@@ -1469,8 +1469,12 @@ cudaError_t sym_backward_t(const float* s, const uint32_t* perm, int64_t n, cons
             LAPLEX_TIMED("sym_bwd", st, k_sym1_sweep<2, false><<<grid, k1NT, 0, st>>>(a, xs, gs, sx, sg, gxs, gas));
         if (p.bucketed) {
             void* scratch = unperm_scratch(p, ws, n);
-            if (gx) LAPLEX_TRY_SYM(launch_unpermute(perm, gxs, n, gx, scratch, st));
-            if (ga) LAPLEX_TRY_SYM(launch_unpermute(perm, gas, n, ga, scratch, st));
+            if (gx && ga)  // both through one placement (the sorted copy of g is free by now)
+                LAPLEX_TRY_SYM(launch_unpermute2(perm, gxs, gas, n, gx, ga, gs, scratch, st));
+            else if (gx)
+                LAPLEX_TRY_SYM(launch_unpermute(perm, gxs, n, gx, scratch, st));
+            else if (ga)
+                LAPLEX_TRY_SYM(launch_unpermute(perm, gas, n, ga, scratch, st));
         }
     } else {
         using SM = SweepSmem<C, 2, kAheadBwd>;
