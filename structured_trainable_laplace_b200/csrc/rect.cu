@@ -708,6 +708,169 @@ __global__ void __launch_bounds__(256, 2) k_large(LargePass A) {
     if (ACCUM) flush(cur);
 }
 
+// The interval-sum pass (accumulate only) for full 32-lane groups, 16-byte
+// slices: one warp per contiguous run of sorted rows, lane l owning channels
+// c0 .. c0+3 of every row (as k_large with lpr = 32, VEC = 4, MODE = kLmAccum, and the
+// same interval sums, tie sums, fp32-then-fp64 partials and owner-or-atomic
+// flushes).  Per batch of 32 rows, lane l computes the scalars of row rb + l (its
+// permutation entry, its bins among the small-side anchors, and the four weights
+// e_R w_p, e_L w_p of its phase weights w_p and decays to the neighbouring
+// small-side anchors) into a per-warp slot in shared memory; the warp then walks
+// the batch reading each row's scalars with two broadcast loads and its 512-byte
+// row with one coalesced load per lane, issued four rows ahead of their use.
+struct AccumSlot {
+    float4 w;  // (e_R w_0, e_R w_1, e_L w_0, e_L w_1), or (w_0, w_1, 0, 0) for a row tied with the small side
+    uint4 ib;  // permutation entry, bin m (anchors < q), bin mp (anchors <= q), unused
+};
+
+template <bool PHASED>
+__global__ void __launch_bounds__(256, 3) k_large_accum_w(LargePass A) {
+    constexpr int NP = PHASED ? 2 : 1, VEC = 4, ND = 2 * NP * VEC, PF = 4;
+    extern __shared__ __align__(16) unsigned char accum_smem[];
+    double(*s_dacc)[256] = reinterpret_cast<double(*)[256]>(accum_smem);
+    AccumSlot* slots = reinterpret_cast<AccumSlot*>(accum_smem + sizeof(double) * ND * 256);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    AccumSlot* ws = slots + warp * 32;
+    const int64_t gid = (int64_t)blockIdx.x * 8 + warp;
+    const int c0 = (blockIdx.y * 32 + lane) * VEC;
+    const bool cval = c0 < A.B;
+    const int64_t r0 = gid * A.rows_per_group;
+    const int64_t r1 = min(A.m, r0 + A.rows_per_group);
+    if (r0 >= r1) return;  // the whole warp leaves together; no block barrier follows
+    const int64_t ms = A.ms;
+    const int B = A.B, Cb = A.Cb;
+    // this lane's slice of a row: channels [0, Bs) from rows, [Bs, B) from rows2
+    const float* src = (A.rows2 != nullptr && c0 >= A.Bs) ? A.rows2 + (c0 - A.Bs) : A.rows + c0;
+    const int64_t stride = A.Bs;
+
+#pragma unroll
+    for (int i = 0; i < ND; ++i) s_dacc[i][threadIdx.x] = 0.0;
+    int64_t m_run = lower_bound_f(A.sp, ms, __ldg(A.s + r0));
+    int64_t mp_run = upper_bound_f(A.sp, ms, __ldg(A.s + r0));
+    const int64_t m_first = m_run;
+    const int64_t m_last = lower_bound_f(A.sp, ms, __ldg(A.s + r1 - 1));
+    int64_t cur = m_run;
+    float fu[NP][VEC], fv[NP][VEC];
+#pragma unroll
+    for (int q = 0; q < NP; ++q)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) fu[q][v] = fv[q][v] = 0.f;
+    int cnt = 0;
+    auto fold = [&]() {
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                s_dacc[q * VEC + v][threadIdx.x] += (double)fu[q][v];
+                s_dacc[NP * VEC + q * VEC + v][threadIdx.x] += (double)fv[q][v];
+                fu[q][v] = fv[q][v] = 0.f;
+            }
+        cnt = 0;
+    };
+    auto flush = [&](int64_t bin) {
+        fold();
+        if (!cval) return;
+        const bool owner = bin > m_first && bin < m_last;  // no other warp touches this bin
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                const int ch = q * B + c0 + v;
+                double& du = s_dacc[q * VEC + v][threadIdx.x];
+                double& dv = s_dacc[NP * VEC + q * VEC + v][threadIdx.x];
+                if (bin < ms) {
+                    double* dst = A.U + bin * Cb + ch;
+                    if (owner)
+                        *dst = du;
+                    else if (du != 0.0)
+                        atomicAdd(dst, du);
+                }
+                if (bin >= 1) {
+                    double* dst = A.V + (bin - 1) * Cb + ch;
+                    if (owner)
+                        *dst = dv;
+                    else if (dv != 0.0)
+                        atomicAdd(dst, dv);
+                }
+                du = 0.0;
+                dv = 0.0;
+            }
+    };
+
+    for (int64_t rb = r0; rb < r1; rb += 32) {
+        const int nb = (int)min((int64_t)32, r1 - rb);
+        __syncwarp();  // the previous batch's slots have been read
+        if (lane < nb) {
+            const int64_t r = rb + lane;
+            const float q = __ldg(A.s + r);
+            AccumSlot sl;
+            const uint32_t pr = min(__ldg(A.perm + r), (uint32_t)(A.m - 1));
+            float w0 = 1.f, w1 = 0.f;
+            if (PHASED) sincosf(__ldg(A.theta + pr), &w1, &w0);
+            int64_t mm = m_run;
+            while (mm < ms && __ldg(A.sp + mm) < q) ++mm;
+            int64_t mmp = max(mp_run, mm);
+            while (mmp < ms && __ldg(A.sp + mmp) <= q) ++mmp;
+            const float eL = (mm > 0) ? expf(__ldg(A.sp + mm - 1) - q) : 0.f;
+            const float eR = (mmp < ms) ? expf(q - __ldg(A.sp + mmp)) : 0.f;
+            sl.w = (mmp > mm) ? make_float4(w0, w1, 0.f, 0.f) : make_float4(eR * w0, eR * w1, eL * w0, eL * w1);
+            sl.ib = make_uint4(pr, (uint32_t)mm, (uint32_t)mmp, 0u);
+            ws[lane] = sl;
+        }
+        __syncwarp();
+        {
+            const uint4 last = ws[nb - 1].ib;  // where the next batch's searches start
+            m_run = last.y;
+            mp_run = last.z;
+        }
+        for (int u0 = 0; u0 < nb; u0 += PF) {
+            float4 h[PF];
+#pragma unroll
+            for (int i = 0; i < PF; ++i) {
+                h[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (u0 + i < nb && cval) h[i] = __ldg(reinterpret_cast<const float4*>(src + (int64_t)ws[u0 + i].ib.x * stride));
+            }
+#pragma unroll
+            for (int i = 0; i < PF; ++i) {
+                if (u0 + i >= nb) break;
+                const float4 w = ws[u0 + i].w;
+                const uint4 ib = ws[u0 + i].ib;
+                const int64_t mr = ib.y, mpr = ib.z;
+                if (mr != cur) {
+                    flush(cur);
+                    cur = mr;
+                }
+                const float hv[4] = {h[i].x, h[i].y, h[i].z, h[i].w};
+                if (mpr == mr) {
+                    // untied rows feed the interval sums u (weighted to the right
+                    // neighbour) and v (to the left one)
+                    const float wr[2] = {w.x, w.y}, wl[2] = {w.z, w.w};
+#pragma unroll
+                    for (int q = 0; q < NP; ++q)
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) {
+                            fu[q][v] = fmaf(wr[q], hv[v], fu[q][v]);
+                            fv[q][v] = fmaf(wl[q], hv[v], fv[q][v]);
+                        }
+                } else if (cval) {
+                    // a row tied with a run of small-side anchors enters that run only
+                    const float wt[2] = {w.x, w.y};
+#pragma unroll
+                    for (int q = 0; q < NP; ++q)
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) {
+                            const double val = (double)(wt[q] * hv[v]);
+                            atomicAdd(A.TL + mr * Cb + q * B + c0 + v, val);
+                            atomicAdd(A.TR + (mpr - 1) * Cb + q * B + c0 + v, val);
+                        }
+                }
+                if (++cnt == 16) fold();
+            }
+        }
+    }
+    flush(cur);
+}
+
 // ------------------------------------------------------------------ finish
 
 struct Finish {
@@ -950,6 +1113,28 @@ cudaError_t large_mode(LargePass A, int mode, int chunks, cudaStream_t st) {
     }
 }
 
+template <bool PHASED>
+cudaError_t launch_large_accum_w(LargePass A, int chunks, cudaStream_t st) {
+    constexpr int NP = PHASED ? 2 : 1;
+    const size_t smem = sizeof(double) * 2 * NP * 4 * 256 + sizeof(AccumSlot) * 256;
+    static PerDevice occ_dev;
+    int& occ = occ_dev.here();
+    if (occ == 0) {
+        int o = 1;
+        cudaFuncSetAttribute(k_large_accum_w<PHASED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large_accum_w<PHASED>, 256, smem) != cudaSuccess)
+            o = 1;
+        occ = std::max(o, 1);
+    }
+    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ / chunks);
+    const int64_t need = (A.m + 8 * kLargeMinRows - 1) / (8 * kLargeMinRows);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
+    A.rows_per_group = (A.m + blocks * 8 - 1) / (blocks * 8);
+    const dim3 grid((unsigned)blocks, (unsigned)chunks);
+    LAPLEX_TIMED("large_accum", st, k_large_accum_w<PHASED><<<grid, 256, smem, st>>>(A));
+    return cudaGetLastError();
+}
+
 cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
     const bool phased = A.theta != nullptr;
     if (A.Bs == 0) A.Bs = A.B;
@@ -963,6 +1148,8 @@ cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
         if (A.g_anchor) LAPLEX_TRY(cudaMemsetAsync(A.g_anchor, 0, sizeof(float) * A.m, st));
         if (A.g_phase) LAPLEX_TRY(cudaMemsetAsync(A.g_phase, 0, sizeof(float) * A.m, st));
     }
+    if (mode == kLmAccum && vec == 4 && lpr == 32)  // full-warp groups: the lean interval-sum pass
+        return phased ? launch_large_accum_w<true>(A, chunks, st) : launch_large_accum_w<false>(A, chunks, st);
     if (vec == 4) return phased ? large_mode<4, true>(A, mode, chunks, st) : large_mode<4, false>(A, mode, chunks, st);
     return phased ? large_mode<1, true>(A, mode, chunks, st) : large_mode<1, false>(A, mode, chunks, st);
 }
