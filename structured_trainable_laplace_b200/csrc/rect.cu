@@ -871,6 +871,167 @@ __global__ void __launch_bounds__(256, 3) k_large_accum_w(LargePass A) {
     flush(cur);
 }
 
+// The neighbour-state pass (expand and / or gradients) for full 32-lane groups,
+// 16-byte slices: the per-warp scalar slots of k_large_accum_w, then per row
+//   out = sum_p w_p (eLf P_(mp-1) + eR S_mp)          (EXPAND; eLf = 1 for a tie)
+//   ga  = sum_c h_c sum_p w_p (eR S_mp - eL P_(m-1))   (GRAD: strict right - left)
+//   gph = sum_c h_c (w_0 f_1 - w_1 f_0),  f_p = eLf P_(mp-1) + eR S_mp   (GRAD, phased)
+// from the small side's states P, S (reloaded only when the row's bins change) and
+// the gathered row h; the gradient shares of four rows are summed over the warp by
+// recursive halving.  The arithmetic is that of k_large's row body.
+struct ExpandSlot {
+    float4 w;  // (w_0, w_1, eL, eR)
+    uint4 ib;  // permutation entry, bin m (anchors < q), bin mp (anchors <= q), unused
+};
+
+template <bool PHASED, bool EXPAND, bool GRAD>
+__global__ void __launch_bounds__(256, 3) k_large_expand_w(LargePass A) {
+    constexpr int NP = PHASED ? 2 : 1, VEC = 4, U = 4;
+    __shared__ ExpandSlot slots[8][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    ExpandSlot* ws = slots[warp];
+    const int64_t gid = (int64_t)blockIdx.x * 8 + warp;
+    const int c0 = (blockIdx.y * 32 + lane) * VEC;
+    const bool cval = c0 < A.B;
+    const int64_t r0 = gid * A.rows_per_group;
+    const int64_t r1 = min(A.m, r0 + A.rows_per_group);
+    if (r0 >= r1) return;  // the whole warp leaves together; no block barrier follows
+    const int64_t ms = A.ms;
+    const int B = A.B, Cb = A.Cb;
+    const float* src = (A.rows2 != nullptr && c0 >= A.Bs) ? A.rows2 + (c0 - A.Bs) : A.rows + c0;
+    const int64_t stride = A.Bs;
+    int64_t m_run = lower_bound_f(A.sp, ms, __ldg(A.s + r0));
+    int64_t mp_run = upper_bound_f(A.sp, ms, __ldg(A.s + r0));
+    int64_t st_m = -1, st_mp = -1;
+    float Pm1[NP][VEC], Pmp[NP][VEC], Smp[NP][VEC];
+    auto put_grad = [&](float* dst, uint32_t pr, float v) {
+        if (dst == nullptr) return;
+        if (A.chunk_atomic)
+            atomicAdd(dst + pr, v);
+        else if (A.accumulate)
+            dst[pr] += v;  // every row is visited once per launch
+        else
+            dst[pr] = v;
+    };
+
+    for (int64_t rb = r0; rb < r1; rb += 32) {
+        const int nb = (int)min((int64_t)32, r1 - rb);
+        __syncwarp();  // the previous batch's slots have been read
+        if (lane < nb) {
+            const int64_t r = rb + lane;
+            const float q = __ldg(A.s + r);
+            const uint32_t pr = min(__ldg(A.perm + r), (uint32_t)(A.m - 1));
+            float w0 = 1.f, w1 = 0.f;
+            if (PHASED) sincosf(__ldg(A.theta + pr), &w1, &w0);
+            int64_t mm = m_run;
+            while (mm < ms && __ldg(A.sp + mm) < q) ++mm;
+            int64_t mmp = max(mp_run, mm);
+            while (mmp < ms && __ldg(A.sp + mmp) <= q) ++mmp;
+            const float eL = (mm > 0) ? expf(__ldg(A.sp + mm - 1) - q) : 0.f;
+            const float eR = (mmp < ms) ? expf(q - __ldg(A.sp + mmp)) : 0.f;
+            ExpandSlot sl;
+            sl.w = make_float4(w0, w1, eL, eR);
+            sl.ib = make_uint4(pr, (uint32_t)mm, (uint32_t)mmp, 0u);
+            ws[lane] = sl;
+        }
+        __syncwarp();
+        {
+            const uint4 last = ws[nb - 1].ib;
+            m_run = last.y;
+            mp_run = last.z;
+        }
+        for (int u0 = 0; u0 < nb; u0 += U) {
+            float4 h[U];
+#pragma unroll
+            for (int i = 0; i < U; ++i) {
+                h[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (GRAD && u0 + i < nb && cval)
+                    h[i] = __ldg(reinterpret_cast<const float4*>(src + (int64_t)ws[u0 + i].ib.x * stride));
+            }
+            float gpart[GRAD ? 2 * U : 1];
+#pragma unroll
+            for (int i = 0; i < U; ++i) {
+                float ga = 0.f, gph = 0.f;
+                if (u0 + i < nb) {
+                    const float4 w = ws[u0 + i].w;
+                    const uint4 ib = ws[u0 + i].ib;
+                    const int64_t mr = ib.y, mpr = ib.z;
+                    if (mr != st_m || mpr != st_mp) {
+#pragma unroll
+                        for (int q = 0; q < NP; ++q)
+#pragma unroll
+                            for (int v = 0; v < VEC; ++v) {
+                                const int ch = q * B + c0 + v;
+                                Pm1[q][v] = (GRAD && cval && mr > 0) ? __ldg(A.Pst + (mr - 1) * Cb + ch) : 0.f;
+                                Pmp[q][v] = (cval && mpr > 0) ? __ldg(A.Pst + (mpr - 1) * Cb + ch) : 0.f;
+                                Smp[q][v] = (cval && mpr < ms) ? __ldg(A.Sst + mpr * Cb + ch) : 0.f;
+                            }
+                        st_m = mr;
+                        st_mp = mpr;
+                    }
+                    const float wp[2] = {w.x, w.y};
+                    const float eL = w.z, eR = w.w, eLf = (mpr > mr) ? 1.f : eL;
+                    const float hv[4] = {h[i].x, h[i].y, h[i].z, h[i].w};
+                    float o[VEC];
+#pragma unroll
+                    for (int v = 0; v < VEC; ++v) {
+                        o[v] = 0.f;
+                        float t = 0.f;
+#pragma unroll
+                        for (int q = 0; q < NP; ++q) {
+                            const float fl = eLf * wp[q], fr = eR * wp[q], dl = eL * wp[q];
+                            o[v] = fmaf(fl, Pmp[q][v], fmaf(fr, Smp[q][v], o[v]));
+                            if (GRAD) t = fmaf(fr, Smp[q][v], fmaf(-dl, Pm1[q][v], t));
+                        }
+                        if (GRAD) {
+                            ga = fmaf(hv[v], t, ga);
+                            if (PHASED) {
+                                const float f0 = fmaf(eLf, Pmp[0][v], eR * Smp[0][v]);
+                                const float f1 = fmaf(eLf, Pmp[NP - 1][v], eR * Smp[NP - 1][v]);
+                                gph = fmaf(hv[v], fmaf(wp[0], f1, -wp[1] * f0), gph);
+                            }
+                        }
+                    }
+                    if (EXPAND && A.out != nullptr && cval)
+                        *reinterpret_cast<float4*>(A.out + (int64_t)ib.x * B + c0) = make_float4(o[0], o[1], o[2], o[3]);
+                }
+                if (GRAD) {
+                    gpart[i] = ga;
+                    gpart[U + i] = gph;
+                }
+            }
+            if (GRAD) {
+                // sum the 2U shares over the 32 lanes by recursive halving: after the
+                // halving rounds lane l holds the total of value index base, then the
+                // remaining rounds add whole totals
+                constexpr int NV = 2 * U;
+                int base = 0;
+#pragma unroll
+                for (int L = 0; (NV >> L) > 1; ++L) {
+                    const int o = 16 >> L;
+                    const bool upper = (lane & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < (NV >> (L + 1)); ++i) {
+                        const float keep = upper ? gpart[i + (NV >> (L + 1))] : gpart[i];
+                        const float send = upper ? gpart[i] : gpart[i + (NV >> (L + 1))];
+                        gpart[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                    }
+                    if (upper) base += NV >> (L + 1);
+                }
+                constexpr int HL = (NV == 8) ? 3 : 0;  // halving rounds taken (log2 NV)
+                static_assert(NV == 8, "four rows per reduction");
+                for (int o = (32 >> HL) >> 1; o >= 1; o >>= 1) gpart[0] += __shfl_xor_sync(0xffffffffu, gpart[0], o);
+                const bool writer = (lane & ((32 >> HL) - 1)) == 0;
+                const int u = base % U;
+                if (writer && u0 + u < nb) {
+                    const uint32_t pr = ws[u0 + u].ib.x;
+                    put_grad(base < U ? A.g_anchor : (PHASED ? A.g_phase : nullptr), pr, gpart[0]);
+                }
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ finish
 
 struct Finish {
@@ -1135,6 +1296,26 @@ cudaError_t launch_large_accum_w(LargePass A, int chunks, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <bool PHASED, bool EXPAND, bool GRAD>
+cudaError_t launch_large_expand_w(LargePass A, int chunks, const char* name, cudaStream_t st) {
+    static PerDevice occ_dev;
+    int& occ = occ_dev.here();
+    if (occ == 0) {
+        int o = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large_expand_w<PHASED, EXPAND, GRAD>, 256, 0) !=
+            cudaSuccess)
+            o = 1;
+        occ = std::max(o, 1);
+    }
+    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ / chunks);
+    const int64_t need = (A.m + 8 * kLargeMinRows - 1) / (8 * kLargeMinRows);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
+    A.rows_per_group = (A.m + blocks * 8 - 1) / (blocks * 8);
+    const dim3 grid((unsigned)blocks, (unsigned)chunks);
+    LAPLEX_TIMED(name, st, k_large_expand_w<PHASED, EXPAND, GRAD><<<grid, 256, 0, st>>>(A));
+    return cudaGetLastError();
+}
+
 cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
     const bool phased = A.theta != nullptr;
     if (A.Bs == 0) A.Bs = A.B;
@@ -1150,6 +1331,19 @@ cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
     }
     if (mode == kLmAccum && vec == 4 && lpr == 32)  // full-warp groups: the lean interval-sum pass
         return phased ? launch_large_accum_w<true>(A, chunks, st) : launch_large_accum_w<false>(A, chunks, st);
+    if (vec == 4 && lpr == 32 && (mode & kLmAccum) == 0) {  // full-warp groups: the lean neighbour-state pass
+        switch (mode | (phased ? 8 : 0)) {
+            case kLmExpand: return launch_large_expand_w<false, true, false>(A, chunks, "large_expand", st);
+            case kLmGrad: return launch_large_expand_w<false, false, true>(A, chunks, "large_grad", st);
+            case kLmExpand | kLmGrad:
+                return launch_large_expand_w<false, true, true>(A, chunks, "large_expand_grad", st);
+            case 8 | kLmExpand: return launch_large_expand_w<true, true, false>(A, chunks, "large_expand", st);
+            case 8 | kLmGrad: return launch_large_expand_w<true, false, true>(A, chunks, "large_grad", st);
+            case 8 | kLmExpand | kLmGrad:
+                return launch_large_expand_w<true, true, true>(A, chunks, "large_expand_grad", st);
+            default: return cudaErrorInvalidValue;
+        }
+    }
     if (vec == 4) return phased ? large_mode<4, true>(A, mode, chunks, st) : large_mode<4, false>(A, mode, chunks, st);
     return phased ? large_mode<1, true>(A, mode, chunks, st) : large_mode<1, false>(A, mode, chunks, st);
 }
