@@ -6,7 +6,8 @@
 // +0), values the original indices.  Least-significant digit first, 4 passes of
 // 8 bits.  Each pass is one kernel over tiles of 3840 keys claimed in order from
 // an atomic counter: the tile ranks its keys stably inside each warp (the lanes
-// sharing a digit found by ballots over its bits), publishes its per-digit counts, looks back over the tiles
+// sharing a digit found through per-digit lane words in shared memory), publishes
+// its per-digit counts, looks back over the tiles
 // before it for their per-digit prefixes (bounded waits), and scatters through
 // shared memory so that runs of equal digits leave as contiguous stores.
 // A histogram kernel computes the four global digit histograms in one read of
@@ -112,6 +113,10 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     __shared__ uint32_t s_start[kRadix];  // tile-local start of each digit
     __shared__ uint32_t s_scan[kNW];
     __shared__ int64_t s_tile;
+    // during the ranking, the lanes of the current item holding each digit (and a
+    // word for rows past n), per warp; the key buffer is free until the placement
+    static_assert(kNW * (kRadix + 1) <= kTile, "peer words fit in the key buffer");
+    uint32_t(*s_peer)[kRadix + 1] = reinterpret_cast<uint32_t(*)[kRadix + 1]>(s_keys);
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     if (n_dev != nullptr) {
@@ -122,6 +127,7 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     }
     if (tid == 0) s_tile = atomicAdd(counter, 1u);
     for (int i = tid; i < kNW * kRadix; i += kNT) (&s_whist[0][0])[i] = 0;
+    for (int i = tid; i < kNW * (kRadix + 1); i += kNT) (&s_peer[0][0])[i] = 0;
     __syncthreads();
     const int64_t tile = s_tile;
     const int64_t base = tile * kTile;
@@ -148,39 +154,29 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
             key[i] = 0xffffffffu;
         }
     }
-    // stable rank inside the warp, items in (i, lane) order = index order.  The
-    // masks of lanes holding the same digit do not depend on the running counts,
-    // so all are formed first; only the count updates form a chain.  Each mask is
-    // the AND over the digit's 8 bits of the ballot of lanes agreeing on that bit
-    // (plus the ballot of valid lanes, so that rows past n group apart).  rank[]
-    // holds the mask until the rank replaces it.
+    // stable rank inside the warp, items in (i, lane) order = index order.  For each
+    // item the lanes holding the same digit are found in shared memory: every lane
+    // ORs its lane bit into the warp's word for its digit (rows past n into a word
+    // of their own), reads the word back, and the lowest of those lanes advances
+    // the warp's running count of the digit and clears the word for the next item.
+    // rank = running count before the item + the lanes below in the word.
     // rows of this warp's slice below n (32-bit from here on: a slice holds 32 * kItems)
     const int wn = (int)max((int64_t)0, min((int64_t)(32 * kItems), n - wbase));
+    const uint32_t my_bit = 1u << lane, lt = lanemask_lt();
 #pragma unroll
     for (int i = 0; i < kItems; ++i) {
         const bool valid = i * 32 + lane < wn;
-        const uint32_t d = (key[i] >> shift) & 0xffu;
-        const uint32_t vb = __ballot_sync(0xffffffffu, valid);
-        uint32_t peers = valid ? vb : ~vb;
-#pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const bool bit = (d >> b) & 1u;
-            const uint32_t bal = __ballot_sync(0xffffffffu, bit);
-            peers &= bit ? bal : ~bal;
-        }
-        rank[i] = peers;
-    }
-#pragma unroll
-    for (int i = 0; i < kItems; ++i) {
-        const bool valid = i * 32 + lane < wn;
-        const uint32_t d = (key[i] >> shift) & 0xffu, peers = rank[i];
-        uint32_t before = 0;
-        if (valid) {
-            before = s_whist[w][d];
-            rank[i] = before + __popc(peers & lanemask_lt());
-        }
+        const uint32_t d = valid ? ((key[i] >> shift) & 0xffu) : (uint32_t)kRadix;
+        atomicOr(&s_peer[w][d], my_bit);
         __syncwarp();
-        if (valid && lane == __ffs(peers) - 1) s_whist[w][d] = before + __popc(peers);
+        const uint32_t peers = s_peer[w][d];
+        const uint32_t before = valid ? s_whist[w][d] : 0u;
+        rank[i] = before + __popc(peers & lt);
+        __syncwarp();
+        if (lane == __ffs(peers) - 1) {
+            if (valid) s_whist[w][d] = before + __popc(peers);
+            s_peer[w][d] = 0u;
+        }
         __syncwarp();
     }
     __syncthreads();
