@@ -383,14 +383,17 @@ def oracle_pass(w, ws):
 
 
 def oracle_sample_size(w, budget_s: float) -> int:
-    """Rows of the oracle sample that take about budget_s (grown from 2^14, at most
-    the workload's own n)."""
+    """Rows of the oracle sample that take about budget_s: grown from 2^14 until a
+    pass takes a tenth of the budget, then scaled in proportion to the time (the
+    oracle's cost is close to linear in n); at most the workload's own n."""
     n_s = 1 << 14
     while True:
         _, dt = oracle_pass(w, oracle_inputs(w, n_s))
-        if dt >= 0.5 * budget_s or n_s >= w.n:
-            return n_s
-        n_s = min(w.n, n_s * max(2, int(budget_s / max(dt, 1e-3))))
+        if n_s >= w.n:
+            return w.n
+        if dt >= 0.1 * budget_s:
+            return int(min(w.n, max(n_s, n_s * budget_s / dt)))
+        n_s = min(w.n, n_s * 4)
 
 
 def oracle_sample(w, budget_s: float):

@@ -723,20 +723,28 @@ struct AccumSlot {
     uint4 ib;  // permutation entry, bin m (anchors < q), bin mp (anchors <= q), unused
 };
 
-template <bool PHASED>
+// Rows per batch of a group of LPR lanes (at least 8, so that narrow groups too take
+// a batch of rows per pair of warp barriers) and the slots of a warp.
+template <int LPR>
+constexpr int kLeanBatch = LPR >= 8 ? LPR : 8;
+template <int LPR>
+constexpr int kLeanSlots = (32 / LPR) * kLeanBatch<LPR>;
+
+template <int LPR, bool PHASED>
 __global__ void __launch_bounds__(256, 3) k_large_accum_w(LargePass A) {
-    constexpr int NP = PHASED ? 2 : 1, VEC = 4, ND = 2 * NP * VEC, PF = 4;
+    constexpr int NP = PHASED ? 2 : 1, VEC = 4, ND = 2 * NP * VEC, S = kLeanBatch<LPR>, PF = S < 4 ? S : 4;
     extern __shared__ __align__(16) unsigned char accum_smem[];
     double(*s_dacc)[256] = reinterpret_cast<double(*)[256]>(accum_smem);
     AccumSlot* slots = reinterpret_cast<AccumSlot*>(accum_smem + sizeof(double) * ND * 256);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    AccumSlot* ws = slots + warp * 32;
-    const int64_t gid = (int64_t)blockIdx.x * 8 + warp;
-    const int c0 = (blockIdx.y * 32 + lane) * VEC;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gl = lane % LPR, gw = lane / LPR;
+    const unsigned gmask = (LPR == 32) ? 0xffffffffu : (((1u << LPR) - 1u) << (gw * LPR));
+    AccumSlot* ws = slots + warp * kLeanSlots<LPR> + gw * S;
+    const int64_t gid = ((int64_t)blockIdx.x * 8 + warp) * (32 / LPR) + gw;
+    const int c0 = (blockIdx.y * LPR + gl) * VEC;
     const bool cval = c0 < A.B;
     const int64_t r0 = gid * A.rows_per_group;
     const int64_t r1 = min(A.m, r0 + A.rows_per_group);
-    if (r0 >= r1) return;  // the whole warp leaves together; no block barrier follows
+    if (r0 >= r1) return;  // the whole group leaves together; no block barrier follows
     const int64_t ms = A.ms;
     const int B = A.B, Cb = A.Cb;
     // this lane's slice of a row: channels [0, Bs) from rows, [Bs, B) from rows2
@@ -797,11 +805,11 @@ __global__ void __launch_bounds__(256, 3) k_large_accum_w(LargePass A) {
             }
     };
 
-    for (int64_t rb = r0; rb < r1; rb += 32) {
-        const int nb = (int)min((int64_t)32, r1 - rb);
-        __syncwarp();  // the previous batch's slots have been read
-        if (lane < nb) {
-            const int64_t r = rb + lane;
+    for (int64_t rb = r0; rb < r1; rb += S) {
+        const int nb = (int)min((int64_t)S, r1 - rb);
+        __syncwarp(gmask);  // the previous batch's slots have been read
+        for (int j = gl; j < nb; j += LPR) {
+            const int64_t r = rb + j;
             const float q = __ldg(A.s + r);
             AccumSlot sl;
             const uint32_t pr = min(__ldg(A.perm + r), (uint32_t)(A.m - 1));
@@ -815,9 +823,9 @@ __global__ void __launch_bounds__(256, 3) k_large_accum_w(LargePass A) {
             const float eR = (mmp < ms) ? expf(q - __ldg(A.sp + mmp)) : 0.f;
             sl.w = (mmp > mm) ? make_float4(w0, w1, 0.f, 0.f) : make_float4(eR * w0, eR * w1, eL * w0, eL * w1);
             sl.ib = make_uint4(pr, (uint32_t)mm, (uint32_t)mmp, 0u);
-            ws[lane] = sl;
+            ws[j] = sl;
         }
-        __syncwarp();
+        __syncwarp(gmask);
         {
             const uint4 last = ws[nb - 1].ib;  // where the next batch's searches start
             m_run = last.y;
@@ -884,18 +892,20 @@ struct ExpandSlot {
     uint4 ib;  // permutation entry, bin m (anchors < q), bin mp (anchors <= q), unused
 };
 
-template <bool PHASED, bool EXPAND, bool GRAD>
+template <int LPR, bool PHASED, bool EXPAND, bool GRAD>
 __global__ void __launch_bounds__(256, 3) k_large_expand_w(LargePass A) {
-    constexpr int NP = PHASED ? 2 : 1, VEC = 4, U = 4;
-    __shared__ ExpandSlot slots[8][32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    ExpandSlot* ws = slots[warp];
-    const int64_t gid = (int64_t)blockIdx.x * 8 + warp;
-    const int c0 = (blockIdx.y * 32 + lane) * VEC;
+    static_assert(!GRAD || LPR == 32, "the gradient reduction is written for full warps");
+    constexpr int NP = PHASED ? 2 : 1, VEC = 4, U = 4, S = kLeanBatch<LPR>;
+    __shared__ ExpandSlot slots[8][kLeanSlots<LPR>];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gl = lane % LPR, gw = lane / LPR;
+    const unsigned gmask = (LPR == 32) ? 0xffffffffu : (((1u << LPR) - 1u) << (gw * LPR));
+    ExpandSlot* ws = slots[warp] + gw * S;
+    const int64_t gid = ((int64_t)blockIdx.x * 8 + warp) * (32 / LPR) + gw;
+    const int c0 = (blockIdx.y * LPR + gl) * VEC;
     const bool cval = c0 < A.B;
     const int64_t r0 = gid * A.rows_per_group;
     const int64_t r1 = min(A.m, r0 + A.rows_per_group);
-    if (r0 >= r1) return;  // the whole warp leaves together; no block barrier follows
+    if (r0 >= r1) return;  // the whole group leaves together; no block barrier follows
     const int64_t ms = A.ms;
     const int B = A.B, Cb = A.Cb;
     const float* src = (A.rows2 != nullptr && c0 >= A.Bs) ? A.rows2 + (c0 - A.Bs) : A.rows + c0;
@@ -914,11 +924,11 @@ __global__ void __launch_bounds__(256, 3) k_large_expand_w(LargePass A) {
             dst[pr] = v;
     };
 
-    for (int64_t rb = r0; rb < r1; rb += 32) {
-        const int nb = (int)min((int64_t)32, r1 - rb);
-        __syncwarp();  // the previous batch's slots have been read
-        if (lane < nb) {
-            const int64_t r = rb + lane;
+    for (int64_t rb = r0; rb < r1; rb += S) {
+        const int nb = (int)min((int64_t)S, r1 - rb);
+        __syncwarp(gmask);  // the previous batch's slots have been read
+        for (int j = gl; j < nb; j += LPR) {
+            const int64_t r = rb + j;
             const float q = __ldg(A.s + r);
             const uint32_t pr = min(__ldg(A.perm + r), (uint32_t)(A.m - 1));
             float w0 = 1.f, w1 = 0.f;
@@ -932,9 +942,9 @@ __global__ void __launch_bounds__(256, 3) k_large_expand_w(LargePass A) {
             ExpandSlot sl;
             sl.w = make_float4(w0, w1, eL, eR);
             sl.ib = make_uint4(pr, (uint32_t)mm, (uint32_t)mmp, 0u);
-            ws[lane] = sl;
+            ws[j] = sl;
         }
-        __syncwarp();
+        __syncwarp(gmask);
         {
             const uint4 last = ws[nb - 1].ib;
             m_run = last.y;
@@ -1274,46 +1284,62 @@ cudaError_t large_mode(LargePass A, int mode, int chunks, cudaStream_t st) {
     }
 }
 
-template <bool PHASED>
+// Grid of the lean large-side kernels: one wave at the kernel's occupancy, each
+// group of LPR lanes walking an equal contiguous run of at least kLargeMinRows rows.
+int64_t lean_grid(LargePass& A, int lpr, int chunks, int occ) {
+    const int64_t groups_per_block = 8 * (32 / lpr);
+    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ / chunks);
+    const int64_t need = (A.m + groups_per_block * kLargeMinRows - 1) / (groups_per_block * kLargeMinRows);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
+    A.rows_per_group = (A.m + blocks * groups_per_block - 1) / (blocks * groups_per_block);
+    return blocks;
+}
+
+template <int LPR, bool PHASED>
 cudaError_t launch_large_accum_w(LargePass A, int chunks, cudaStream_t st) {
     constexpr int NP = PHASED ? 2 : 1;
-    const size_t smem = sizeof(double) * 2 * NP * 4 * 256 + sizeof(AccumSlot) * 256;
+    const size_t smem = sizeof(double) * 2 * NP * 4 * 256 + sizeof(AccumSlot) * 8 * kLeanSlots<LPR>;
     static PerDevice occ_dev;
     int& occ = occ_dev.here();
     if (occ == 0) {
         int o = 1;
-        cudaFuncSetAttribute(k_large_accum_w<PHASED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large_accum_w<PHASED>, 256, smem) != cudaSuccess)
+        cudaFuncSetAttribute(k_large_accum_w<LPR, PHASED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large_accum_w<LPR, PHASED>, 256, smem) != cudaSuccess)
             o = 1;
         occ = std::max(o, 1);
     }
-    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ / chunks);
-    const int64_t need = (A.m + 8 * kLargeMinRows - 1) / (8 * kLargeMinRows);
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
-    A.rows_per_group = (A.m + blocks * 8 - 1) / (blocks * 8);
+    const int64_t blocks = lean_grid(A, LPR, chunks, occ);
     const dim3 grid((unsigned)blocks, (unsigned)chunks);
-    LAPLEX_TIMED("large_accum", st, k_large_accum_w<PHASED><<<grid, 256, smem, st>>>(A));
+    LAPLEX_TIMED("large_accum", st, k_large_accum_w<LPR, PHASED><<<grid, 256, smem, st>>>(A));
     return cudaGetLastError();
 }
 
-template <bool PHASED, bool EXPAND, bool GRAD>
+template <int LPR, bool PHASED, bool EXPAND, bool GRAD>
 cudaError_t launch_large_expand_w(LargePass A, int chunks, const char* name, cudaStream_t st) {
     static PerDevice occ_dev;
     int& occ = occ_dev.here();
     if (occ == 0) {
         int o = 1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large_expand_w<PHASED, EXPAND, GRAD>, 256, 0) !=
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large_expand_w<LPR, PHASED, EXPAND, GRAD>, 256, 0) !=
             cudaSuccess)
             o = 1;
         occ = std::max(o, 1);
     }
-    const int64_t wave = std::max<int64_t>(1, (int64_t)sm_count() * occ / chunks);
-    const int64_t need = (A.m + 8 * kLargeMinRows - 1) / (8 * kLargeMinRows);
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(wave, need));
-    A.rows_per_group = (A.m + blocks * 8 - 1) / (blocks * 8);
+    const int64_t blocks = lean_grid(A, LPR, chunks, occ);
     const dim3 grid((unsigned)blocks, (unsigned)chunks);
-    LAPLEX_TIMED(name, st, k_large_expand_w<PHASED, EXPAND, GRAD><<<grid, 256, 0, st>>>(A));
+    LAPLEX_TIMED(name, st, k_large_expand_w<LPR, PHASED, EXPAND, GRAD><<<grid, 256, 0, st>>>(A));
     return cudaGetLastError();
+}
+
+template <int LPR>
+cudaError_t lean_accum(LargePass A, bool phased, int chunks, cudaStream_t st) {
+    return phased ? launch_large_accum_w<LPR, true>(A, chunks, st) : launch_large_accum_w<LPR, false>(A, chunks, st);
+}
+
+template <int LPR>
+cudaError_t lean_expand(LargePass A, bool phased, int chunks, cudaStream_t st) {
+    return phased ? launch_large_expand_w<LPR, true, true, false>(A, chunks, "large_expand", st)
+                  : launch_large_expand_w<LPR, false, true, false>(A, chunks, "large_expand", st);
 }
 
 cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
@@ -1329,18 +1355,27 @@ cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
         if (A.g_anchor) LAPLEX_TRY(cudaMemsetAsync(A.g_anchor, 0, sizeof(float) * A.m, st));
         if (A.g_phase) LAPLEX_TRY(cudaMemsetAsync(A.g_phase, 0, sizeof(float) * A.m, st));
     }
-    if (mode == kLmAccum && vec == 4 && lpr == 32)  // full-warp groups: the lean interval-sum pass
-        return phased ? launch_large_accum_w<true>(A, chunks, st) : launch_large_accum_w<false>(A, chunks, st);
-    if (vec == 4 && lpr == 32 && (mode & kLmAccum) == 0) {  // full-warp groups: the lean neighbour-state pass
+    if (mode == kLmAccum && vec == 4) {  // the lean interval-sum pass, every group width
+        switch (lpr) {
+            case 1: break;  // one lane per row: k_large
+            case 2: return lean_accum<2>(A, phased, chunks, st);
+            case 4: return lean_accum<4>(A, phased, chunks, st);
+            case 8: return lean_accum<8>(A, phased, chunks, st);
+            case 16: return lean_accum<16>(A, phased, chunks, st);
+            default: return lean_accum<32>(A, phased, chunks, st);
+        }
+    }
+    // the lean output pass for full-warp groups (narrow groups measured faster in k_large:
+    // Gram image y = A (D w), two lanes per row, 0.090 against 0.081 ms)
+    if (mode == kLmExpand && vec == 4 && lpr == 32) return lean_expand<32>(A, phased, chunks, st);
+    if (vec == 4 && lpr == 32 && (mode & kLmAccum) == 0) {  // full-warp groups: the lean gradient pass
         switch (mode | (phased ? 8 : 0)) {
-            case kLmExpand: return launch_large_expand_w<false, true, false>(A, chunks, "large_expand", st);
-            case kLmGrad: return launch_large_expand_w<false, false, true>(A, chunks, "large_grad", st);
+            case kLmGrad: return launch_large_expand_w<32, false, false, true>(A, chunks, "large_grad", st);
             case kLmExpand | kLmGrad:
-                return launch_large_expand_w<false, true, true>(A, chunks, "large_expand_grad", st);
-            case 8 | kLmExpand: return launch_large_expand_w<true, true, false>(A, chunks, "large_expand", st);
-            case 8 | kLmGrad: return launch_large_expand_w<true, false, true>(A, chunks, "large_grad", st);
+                return launch_large_expand_w<32, false, true, true>(A, chunks, "large_expand_grad", st);
+            case 8 | kLmGrad: return launch_large_expand_w<32, true, false, true>(A, chunks, "large_grad", st);
             case 8 | kLmExpand | kLmGrad:
-                return launch_large_expand_w<true, true, true>(A, chunks, "large_expand_grad", st);
+                return launch_large_expand_w<32, true, true, true>(A, chunks, "large_expand_grad", st);
             default: return cudaErrorInvalidValue;
         }
     }
