@@ -1042,6 +1042,213 @@ __global__ void __launch_bounds__(256, 3) k_large_expand_w(LargePass A) {
     }
 }
 
+// Interval sums and anchor / phase gradients in one pass (kLmAccum | kLmGrad: the
+// backward over a larger output side) for groups of 2-16 lanes of 16-byte slices
+// (instantiated unphased; the phased form would spill):
+// the per-group row slots and interval sums of k_large_accum_w, plus per row the
+// gradient shares of k_large's row body from the cached small-side states, summed
+// over the group's lanes by xor-shuffles and written by its first lane.
+struct AccGradSlot {
+    float4 f;  // (e_R w_0, e_R w_1, e_L w_0, e_L w_1)
+    float4 x;  // (w_0, w_1, e_L, e_R)
+    uint4 ib;  // permutation entry, bin m (anchors < q), bin mp (anchors <= q), unused
+};
+
+template <int LPR, bool PHASED>
+__global__ void __launch_bounds__(256, 3) k_large_accgrad_n(LargePass A) {
+    static_assert(LPR >= 2 && LPR <= 16, "narrow groups");
+    constexpr int NP = PHASED ? 2 : 1, VEC = 4, ND = 2 * NP * VEC, S = kLeanBatch<LPR>, PF = 4;
+    extern __shared__ __align__(16) unsigned char accgrad_smem[];
+    double(*s_dacc)[256] = reinterpret_cast<double(*)[256]>(accgrad_smem);
+    AccGradSlot* slots = reinterpret_cast<AccGradSlot*>(accgrad_smem + sizeof(double) * ND * 256);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, gl = lane % LPR, gw = lane / LPR;
+    const unsigned gmask = ((1u << LPR) - 1u) << (gw * LPR);
+    AccGradSlot* ws = slots + warp * kLeanSlots<LPR> + gw * S;
+    const int64_t gid = ((int64_t)blockIdx.x * 8 + warp) * (32 / LPR) + gw;
+    const int c0 = (blockIdx.y * LPR + gl) * VEC;
+    const bool cval = c0 < A.B;
+    const int64_t r0 = gid * A.rows_per_group;
+    const int64_t r1 = min(A.m, r0 + A.rows_per_group);
+    if (r0 >= r1) return;  // the whole group leaves together; no block barrier follows
+    const int64_t ms = A.ms;
+    const int B = A.B, Cb = A.Cb;
+    const float* src = (A.rows2 != nullptr && c0 >= A.Bs) ? A.rows2 + (c0 - A.Bs) : A.rows + c0;
+    const int64_t stride = A.Bs;
+
+#pragma unroll
+    for (int i = 0; i < ND; ++i) s_dacc[i][threadIdx.x] = 0.0;
+    int64_t m_run = lower_bound_f(A.sp, ms, __ldg(A.s + r0));
+    int64_t mp_run = upper_bound_f(A.sp, ms, __ldg(A.s + r0));
+    const int64_t m_first = m_run;
+    const int64_t m_last = lower_bound_f(A.sp, ms, __ldg(A.s + r1 - 1));
+    int64_t cur = m_run, st_m = -1, st_mp = -1;
+    float fu[NP][VEC], fv[NP][VEC], Pm1[NP][VEC], Pmp[NP][VEC], Smp[NP][VEC];
+#pragma unroll
+    for (int q = 0; q < NP; ++q)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) fu[q][v] = fv[q][v] = 0.f;
+    int cnt = 0;
+    auto fold = [&]() {
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                s_dacc[q * VEC + v][threadIdx.x] += (double)fu[q][v];
+                s_dacc[NP * VEC + q * VEC + v][threadIdx.x] += (double)fv[q][v];
+                fu[q][v] = fv[q][v] = 0.f;
+            }
+        cnt = 0;
+    };
+    auto flush = [&](int64_t bin) {
+        fold();
+        if (!cval) return;
+        const bool owner = bin > m_first && bin < m_last;  // no other group touches this bin
+#pragma unroll
+        for (int q = 0; q < NP; ++q)
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) {
+                const int ch = q * B + c0 + v;
+                double& du = s_dacc[q * VEC + v][threadIdx.x];
+                double& dv = s_dacc[NP * VEC + q * VEC + v][threadIdx.x];
+                if (bin < ms) {
+                    double* dst = A.U + bin * Cb + ch;
+                    if (owner)
+                        *dst = du;
+                    else if (du != 0.0)
+                        atomicAdd(dst, du);
+                }
+                if (bin >= 1) {
+                    double* dst = A.V + (bin - 1) * Cb + ch;
+                    if (owner)
+                        *dst = dv;
+                    else if (dv != 0.0)
+                        atomicAdd(dst, dv);
+                }
+                du = 0.0;
+                dv = 0.0;
+            }
+    };
+    auto put_grad = [&](float* dst, uint32_t pr, float v) {
+        if (dst == nullptr) return;
+        if (A.chunk_atomic)
+            atomicAdd(dst + pr, v);
+        else if (A.accumulate)
+            dst[pr] += v;  // every row is visited once per launch
+        else
+            dst[pr] = v;
+    };
+
+    for (int64_t rb = r0; rb < r1; rb += S) {
+        const int nb = (int)min((int64_t)S, r1 - rb);
+        __syncwarp(gmask);  // the previous batch's slots have been read
+        for (int j = gl; j < nb; j += LPR) {
+            const int64_t r = rb + j;
+            const float q = __ldg(A.s + r);
+            const uint32_t pr = min(__ldg(A.perm + r), (uint32_t)(A.m - 1));
+            float w0 = 1.f, w1 = 0.f;
+            if (PHASED) sincosf(__ldg(A.theta + pr), &w1, &w0);
+            int64_t mm = m_run;
+            while (mm < ms && __ldg(A.sp + mm) < q) ++mm;
+            int64_t mmp = max(mp_run, mm);
+            while (mmp < ms && __ldg(A.sp + mmp) <= q) ++mmp;
+            const float eL = (mm > 0) ? expf(__ldg(A.sp + mm - 1) - q) : 0.f;
+            const float eR = (mmp < ms) ? expf(q - __ldg(A.sp + mmp)) : 0.f;
+            AccGradSlot sl;
+            sl.f = make_float4(eR * w0, eR * w1, eL * w0, eL * w1);
+            sl.x = make_float4(w0, w1, eL, eR);
+            sl.ib = make_uint4(pr, (uint32_t)mm, (uint32_t)mmp, 0u);
+            ws[j] = sl;
+        }
+        __syncwarp(gmask);
+        {
+            const uint4 last = ws[nb - 1].ib;  // where the next batch's searches start
+            m_run = last.y;
+            mp_run = last.z;
+        }
+        for (int u0 = 0; u0 < nb; u0 += PF) {
+            float4 h[PF];
+#pragma unroll
+            for (int i = 0; i < PF; ++i) {
+                h[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (u0 + i < nb && cval)
+                    h[i] = __ldg(reinterpret_cast<const float4*>(src + (int64_t)ws[u0 + i].ib.x * stride));
+            }
+#pragma unroll
+            for (int i = 0; i < PF; ++i) {
+                if (u0 + i >= nb) break;
+                const float4 f = ws[u0 + i].f, x = ws[u0 + i].x;
+                const uint4 ib = ws[u0 + i].ib;
+                const int64_t mr = ib.y, mpr = ib.z;
+                const bool tie = mpr > mr;
+                const float hv[4] = {h[i].x, h[i].y, h[i].z, h[i].w};
+                const float fr[2] = {f.x, f.y}, dl[2] = {f.z, f.w}, wp[2] = {x.x, x.y};
+                // interval sums
+                if (mr != cur) {
+                    flush(cur);
+                    cur = mr;
+                }
+                if (!tie) {
+#pragma unroll
+                    for (int q = 0; q < NP; ++q)
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) {
+                            fu[q][v] = fmaf(fr[q], hv[v], fu[q][v]);
+                            fv[q][v] = fmaf(dl[q], hv[v], fv[q][v]);
+                        }
+                } else if (cval) {
+#pragma unroll
+                    for (int q = 0; q < NP; ++q)
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) {
+                            const double val = (double)(wp[q] * hv[v]);
+                            atomicAdd(A.TL + mr * Cb + q * B + c0 + v, val);
+                            atomicAdd(A.TR + (mpr - 1) * Cb + q * B + c0 + v, val);
+                        }
+                }
+                if (++cnt == 16) fold();
+                // gradient shares from the small side's states
+                if (mr != st_m || mpr != st_mp) {
+#pragma unroll
+                    for (int q = 0; q < NP; ++q)
+#pragma unroll
+                        for (int v = 0; v < VEC; ++v) {
+                            const int ch = q * B + c0 + v;
+                            Pm1[q][v] = (cval && mr > 0) ? __ldg(A.Pst + (mr - 1) * Cb + ch) : 0.f;
+                            Pmp[q][v] = (cval && mpr > 0) ? __ldg(A.Pst + (mpr - 1) * Cb + ch) : 0.f;
+                            Smp[q][v] = (cval && mpr < ms) ? __ldg(A.Sst + mpr * Cb + ch) : 0.f;
+                        }
+                    st_m = mr;
+                    st_mp = mpr;
+                }
+                const float eL = x.z, eR = x.w, eLf = tie ? 1.f : eL;
+                float ga = 0.f, gph = 0.f;
+#pragma unroll
+                for (int v = 0; v < VEC; ++v) {
+                    float t = 0.f;
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) t = fmaf(fr[q], Smp[q][v], fmaf(-dl[q], Pm1[q][v], t));
+                    ga = fmaf(hv[v], t, ga);  // strict right - strict left
+                    if (PHASED) {
+                        const float f0 = fmaf(eLf, Pmp[0][v], eR * Smp[0][v]);
+                        const float f1 = fmaf(eLf, Pmp[NP - 1][v], eR * Smp[NP - 1][v]);
+                        gph = fmaf(hv[v], fmaf(wp[0], f1, -wp[1] * f0), gph);
+                    }
+                }
+#pragma unroll
+                for (int o = LPR / 2; o >= 1; o >>= 1) {
+                    ga += __shfl_xor_sync(gmask, ga, o);
+                    if (PHASED) gph += __shfl_xor_sync(gmask, gph, o);
+                }
+                if (gl == 0) {
+                    put_grad(A.g_anchor, ib.x, ga);
+                    if (PHASED) put_grad(A.g_phase, ib.x, gph);
+                }
+            }
+        }
+    }
+    flush(cur);
+}
+
 // ------------------------------------------------------------------ finish
 
 struct Finish {
@@ -1342,6 +1549,31 @@ cudaError_t lean_expand(LargePass A, bool phased, int chunks, cudaStream_t st) {
                   : launch_large_expand_w<LPR, false, true, false>(A, chunks, "large_expand", st);
 }
 
+template <int LPR, bool PHASED>
+cudaError_t launch_large_accgrad_n(LargePass A, int chunks, cudaStream_t st) {
+    constexpr int NP = PHASED ? 2 : 1;
+    const size_t smem = sizeof(double) * 2 * NP * 4 * 256 + sizeof(AccGradSlot) * 8 * kLeanSlots<LPR>;
+    static PerDevice occ_dev;
+    int& occ = occ_dev.here();
+    if (occ == 0) {
+        int o = 1;
+        cudaFuncSetAttribute(k_large_accgrad_n<LPR, PHASED>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, k_large_accgrad_n<LPR, PHASED>, 256, smem) !=
+            cudaSuccess)
+            o = 1;
+        occ = std::max(o, 1);
+    }
+    const int64_t blocks = lean_grid(A, LPR, chunks, occ);
+    const dim3 grid((unsigned)blocks, (unsigned)chunks);
+    LAPLEX_TIMED("large_accum_grad", st, k_large_accgrad_n<LPR, PHASED><<<grid, 256, smem, st>>>(A));
+    return cudaGetLastError();
+}
+
+template <int LPR>
+cudaError_t lean_accgrad(LargePass A, int chunks, cudaStream_t st) {
+    return launch_large_accgrad_n<LPR, false>(A, chunks, st);
+}
+
 cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
     const bool phased = A.theta != nullptr;
     if (A.Bs == 0) A.Bs = A.B;
@@ -1363,6 +1595,17 @@ cudaError_t large_pass(LargePass A, int mode, cudaStream_t st) {
             case 8: return lean_accum<8>(A, phased, chunks, st);
             case 16: return lean_accum<16>(A, phased, chunks, st);
             default: return lean_accum<32>(A, phased, chunks, st);
+        }
+    }
+    // the lean sums + gradients pass, narrow unphased groups (the phased one holds three
+    // more state arrays and would spill: k_large)
+    if (mode == (kLmAccum | kLmGrad) && vec == 4 && !phased) {
+        switch (lpr) {
+            case 2: return lean_accgrad<2>(A, chunks, st);
+            case 4: return lean_accgrad<4>(A, chunks, st);
+            case 8: return lean_accgrad<8>(A, chunks, st);
+            case 16: return lean_accgrad<16>(A, chunks, st);
+            default: break;  // one lane per row, or full warps: k_large
         }
     }
     // the lean output pass for full-warp groups (narrow groups measured faster in k_large:
