@@ -1989,13 +1989,28 @@ cudaError_t launch_gram_backward(Side A, Side Bs, const float* D, const float* v
                                                                         (paired && need_ab) ? xp : nullptr, gD, Bs.m,
                                                                         (int)B));
     LAPLEX_TRY(cudaGetLastError());
-    if (gv != nullptr) LAPLEX_TRY(launch_rect_forward(A, Bs, x2, B, gv, nullptr, ws, status, st));  // gv = A (D u)
     if (need_ab && paired) {
+        // the scan states of D w | D u over b, once: the paired backward reads them, and
+        // their second half (D u) gives gv = A (D u) without a scan of its own
+        const RectPlan pb = plan_rect(A.m, Bs.m, 2 * B, false, ws);
+        const int64_t szb = pb.ms * (int64_t)pb.Cb;
+        float* P = pb.bufA;
+        LAPLEX_TRY(side_scan(pb, values_scan(Bs, xp, 2 * B, P, P + szb), false, status, st));
+        if (gv != nullptr) {
+            LargePass E = large_args(A, Bs, pb, B);  // B channels, states with the 2B-channel stride
+            E.Pst = P + B;
+            E.Sst = P + szb + B;
+            E.out = gv;
+            LAPLEX_TRY(large_pass(E, kLmExpand, st));
+        }
         // both general products in one backward over 2B channels: inputs D w | D u at
         // b, rows g | v at a (ga sums over all 2B channels, and so does gb)
-        LAPLEX_TRY(launch_rect_backward(A, Bs, xp, g, 2 * B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status,
-                                        st, false, v));
-    } else if (need_ab) {
+        LAPLEX_TRY(launch_rect_backward(A, Bs, xp, g, 2 * B, P, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
+                                        false, v));
+        return cudaSuccess;
+    }
+    if (gv != nullptr) LAPLEX_TRY(launch_rect_forward(A, Bs, x2, B, gv, nullptr, ws, status, st));  // gv = A (D u)
+    if (need_ab) {
         LAPLEX_TRY(launch_rect_backward(A, Bs, x1, g, B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
                                         false));
         LAPLEX_TRY(launch_rect_backward(A, Bs, x2, v, B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
