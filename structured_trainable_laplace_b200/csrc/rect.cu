@@ -110,6 +110,7 @@ __global__ void __launch_bounds__(kSideNT) k_side_right(SideScan a, ChainSet cs,
     // phases need two scan channels per input channel, so C == 1 never carries them
     __shared__ float cw[(BINS || C == 1) ? 1 : R], sw[(BINS || C == 1) ? 1 : R];
     __shared__ ScanSmem<C, NT / 32> sm;
+    __shared__ LookbackSmem<C, NT> lb;
     __shared__ int64_t s_tile;
     const int grp = blockIdx.y;
     if (threadIdx.x == 0) s_tile = a.T - 1 - (int64_t)atomicAdd(&counters[grp], 1u);
@@ -136,11 +137,9 @@ __global__ void __launch_bounds__(kSideNT) k_side_right(SideScan a, ChainSet cs,
     LP excl;
     bool has;
     block_scan_dir<C, NT, true>(st, -s_sm[k * E + 1], -s_sm[(k + 1) * E + 1], sm, excl, has);
-    if (threadIdx.x < 32) {
-        bool hc;
-        const LP tot = threadIdx.x < C ? sm.tot[threadIdx.x] : LP{0.f, 0.f};
-        lookback<C, true>(cs.chain(grp), t, a.T, a.s, a.m, R, tot, -s_sm[1], -s_sm[R + 1], status, hc);
-    }
+    bool hc;
+    const LP tot = threadIdx.x < C ? sm.tot[threadIdx.x] : LP{0.f, 0.f};
+    (void)block_lookback<C, true, NT>(cs.chain(grp), t, a.T, a.s, a.m, R, tot, -s_sm[1], -s_sm[R + 1], status, lb, hc);
 }
 
 template <int C, bool BINS>
@@ -151,9 +150,8 @@ __global__ void __launch_bounds__(kSideNT) k_side_left(SideScan a, ChainSet left
     __shared__ uint32_t p_sm[BINS ? 1 : R];
     __shared__ float cw[(BINS || C == 1) ? 1 : R], sw[(BINS || C == 1) ? 1 : R];
     __shared__ ScanSmem<C, NT / 32> smL, smR;
-    __shared__ double2 s_carry[C];
+    __shared__ LookbackSmem<C, NT> lb;
     __shared__ int64_t s_tile;
-    __shared__ bool s_has;
     const int grp = blockIdx.y;
     if (threadIdx.x == 0) s_tile = (int64_t)atomicAdd(&counters[grp], 1u);
     __syncthreads();
@@ -188,16 +186,12 @@ __global__ void __launch_bounds__(kSideNT) k_side_left(SideScan a, ChainSet left
     bool hr, hl;
     block_scan_dir<C, NT, true>(str, -s_sm[k * E + 1], ub_r, smR, exr, hr);
     block_scan_dir<C, NT, false>(stl, s_sm[k * E + E], ub_l, smL, exl, hl);
-    if (threadIdx.x < 32) {
-        bool hc;
-        const LP tot = threadIdx.x < C ? smL.tot[threadIdx.x] : LP{0.f, 0.f};
-        const double2 cin = lookback<C, false>(left.chain(grp), t, a.T, a.s, a.m, R, tot, s_sm[R], s_sm[0], status, hc);
-        if (threadIdx.x < C) s_carry[threadIdx.x] = cin;
-        if (threadIdx.x == 0) s_has = hc;
-    }
-    __syncthreads();
-    const LP cl = {(float)s_carry[c].x, (float)s_carry[c].y};
-    const LP left_in = seg_incoming(s_has, cl, s_sm[0], hl, exl, ub_l);
+    bool hcl;
+    const LP tot = threadIdx.x < C ? smL.tot[threadIdx.x] : LP{0.f, 0.f};
+    const double2 cin =
+        block_lookback<C, false, NT>(left.chain(grp), t, a.T, a.s, a.m, R, tot, s_sm[R], s_sm[0], status, lb, hcl);
+    const LP cl = {(float)cin.x, (float)cin.y};
+    const LP left_in = seg_incoming(hcl, cl, s_sm[0], hl, exl, ub_l);
     LP cr = {0.f, 0.f};
     const bool hasr = (t + 1 < a.T);
     if (hasr) {
@@ -1436,9 +1430,10 @@ constexpr int64_t kLargeMinRows = 64;
 
 // One warp as tile 1 of a two-tile chain whose tile 0 never publishes: the
 // lookback must give up after its bound and record the timeout.
-__global__ void k_check_wait_bound(Chain ch, const float* s, int32_t* status) {
+__global__ void __launch_bounds__(32) k_check_wait_bound(Chain ch, const float* s, int32_t* status) {
+    __shared__ LookbackSmem<1, 32> lb;
     bool has = false;
-    (void)lookback<1, false>(ch, 1, 2, s, 2, 1, LP{1.f, 1.f}, s[1], s[0], status, has);
+    (void)block_lookback<1, false, 32>(ch, 1, 2, s, 2, 1, LP{1.f, 1.f}, s[1], s[0], status, lb, has);
 }
 
 // Dynamic shared memory of k_large<VEC, PHASED, MODE>: the fp64 partials, plus the

@@ -156,103 +156,145 @@ struct ChainSet {
     }
 };
 
+// Shared scratch of a block-wide lookback (NT threads, C channels).  A window
+// holds W predecessors: thread (c, g) = (tid % C, tid / C) takes channel c of
+// slots g, g + NT / C, ... (Q of them), so a window's states are read with one
+// round of independent loads whatever its width.
+template <int C, int NT>
+struct LookbackSmem {
+    static constexpr int Q = (128 * C / NT) > 1 ? 128 * C / NT : 1;
+    static constexpr int W = NT / C * Q;
+    double2 part[NT / 32][C];
+    double2 run[C];
+    double e[W];
+    int flag[W];
+    int stop[2];
+    bool brk[W];
+};
+
 // Publish tile t's total and look back over its predecessors (t-1, t-2, ... or
-// t+1, t+2, ... when REV).  Called by one full warp; lane c < C handles channel c.
-// tot: this lane's tile total (anchored at u_tile_end).  u_before_tile: oriented
-// anchor of the last row of the predecessor tile.  Returns the incoming carry
-// (anchored at u_before_tile) and whether one exists.
+// t+1, t+2, ... when REV).  Called by every thread of the block; thread c < C
+// passes channel c's tile total in tot (anchored at u_tile_end).  u_before_tile:
+// oriented anchor of the last row of the predecessor tile.  Returns, to every
+// thread, the incoming carry of channel tid % C (anchored at u_before_tile), and
+// whether one exists.
 //
-// The predecessors are read 32 at a time: lane i polls the flag of the i-th
-// predecessor of the window, a ballot finds the nearest one that holds an
-// inclusive state, and once every tile up to it has published, the channel lanes
-// prepend the window's states in order (their loads are independent).  A window
-// without an inclusive state is prepended whole and the next one is read.  Waits
-// are bounded: past kSpinLimit polls the tile records kStatusTimeout and
+// A window is W predecessors: thread i < W polls the flag of the i-th and reads
+// the anchor at its end, the nearest one that holds an inclusive state bounds
+// the window, and once every tile up to it has published, the block sums the
+// window's states and the next window is read only if none was inclusive.
+// Waits are bounded: past kSpinLimit polls the tile records kStatusTimeout and
 // proceeds with what it has.
-template <int C, bool REV>
-__device__ __forceinline__ double2 lookback(Chain ch, int64_t t, int64_t T, const float* s, int64_t n, int64_t R, LP tot,
-                                            float u_tile_end, float u_before_tile, int32_t* status, bool& has_carry) {
-    const int lane = threadIdx.x & 31;
+template <int C, bool REV, int NT>
+__device__ __forceinline__ double2 block_lookback(Chain ch, int64_t t, int64_t T, const float* s, int64_t n, int64_t R,
+                                                  LP tot, float u_tile_end, float u_before_tile, int32_t* status,
+                                                  LookbackSmem<C, NT>& sm, bool& has_carry) {
+    using S = LookbackSmem<C, NT>;
+    constexpr int Q = S::Q, W = S::W, SG = NT / C;
+    const int tid = threadIdx.x, c = tid % C, g = tid / C;
     const bool first = REV ? (t == T - 1) : (t == 0);
     const double2 totd = make_double2((double)tot.L, (double)tot.P);
-    double2 run = make_double2(0.0, 0.0);
     if (first) {
-        if (lane < C) ch.inc[t * C + lane] = totd;
+        if (tid < C) ch.inc[t * C + tid] = totd;
         __threadfence();
-        __syncwarp();
-        if (lane == 0) st_release(&ch.flags[t], 2);
+        __syncthreads();
+        if (tid == 0) st_release(&ch.flags[t], 2);
         has_carry = false;
-        return run;
+        return make_double2(0.0, 0.0);
     }
-    if (lane < C) ch.agg[t * C + lane] = totd;
+    if (tid == 0) sm.stop[0] = sm.stop[1] = W;
+    if (tid < C) {
+        ch.agg[t * C + tid] = totd;
+        sm.run[tid] = make_double2(0.0, 0.0);
+    }
     __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release(&ch.flags[t], 1);
+    __syncthreads();
+    if (tid == 0) st_release(&ch.flags[t], 1);
     bool have = false;
     int64_t jb = REV ? t + 1 : t - 1;  // nearest predecessor of the window
     uint32_t spins = 0;
     bool timed_out = false;
-    while (true) {
-        const int64_t jl = REV ? jb + lane : jb - lane;  // this lane's predecessor
-        const bool exists = REV ? (jl < T) : (jl >= 0);
-        // 3 marks a slot past the end tile (which always publishes an inclusive
-        // state, so the window never takes one)
-        int f = exists ? ld_acquire(&ch.flags[jl]) : 3;
-        unsigned incl = __ballot_sync(0xffffffffu, f >= 2);
-        unsigned zero = __ballot_sync(0xffffffffu, f == 0);
-        const int stop = incl ? __ffs(incl) - 1 : 31;           // last window slot to take
-        const unsigned need = (stop == 31) ? 0xffffffffu : ((2u << stop) - 1u);
-        if ((zero & need) != 0u && !timed_out) {
+    for (int it = 0;; ++it) {
+        // Every state taken is weighted to the same anchor (the end of the nearest
+        // predecessor), so the carry is a plain sum of independent terms: slot i
+        // adds e_i P_i to P and, to L, e_i P_i when its end lies strictly before
+        // that anchor, else its own strict part L_i.  A slot still unpublished
+        // after the bound counts as zero.
+        for (int i = tid; i < W; i += NT) {
+            const int64_t jl = REV ? jb + i : jb - i;
+            const bool exists = REV ? (jl < T) : (jl >= 0);
+            // 3 marks a slot past the end tile (which always publishes an
+            // inclusive state, so the window never reaches one)
+            const int f = exists ? ld_acquire(&ch.flags[jl]) : 3;
+            const float uj = exists ? (REV ? -s[jl * R] : s[min(n, (jl + 1) * R) - 1]) : 0.f;
+            const bool brk = u_before_tile > uj;
+            sm.flag[i] = f;
+            sm.brk[i] = brk;
+            sm.e[i] = brk ? exp((double)uj - (double)u_before_tile) : 1.0;
+            if (f >= 2) atomicMin(&sm.stop[it & 1], i);
+        }
+        __syncthreads();
+        const int stop = sm.stop[it & 1];  // last window slot to take
+        if (tid == 0) sm.stop[(it + 1) & 1] = W;
+        bool zero = false;
+        for (int i = tid; i <= stop && i < W; i += NT) zero = zero || (sm.flag[i] == 0);
+        if (__syncthreads_or(zero) && !timed_out) {
             if (++spins > kSpinLimit) {
-                if (lane == 0) raise_status(status, kStatusTimeout);
+                if (tid == 0) raise_status(status, kStatusTimeout);
                 timed_out = true;
             } else {
                 __nanosleep(64);
             }
             continue;
         }
-        // Every state taken is weighted to the same anchor (the end of the nearest
-        // predecessor), so the carry is a plain sum of independent terms: slot i
-        // adds e_i P_i to P and, to L, e_i P_i when its end lies strictly before
-        // that anchor, else its own strict part L_i.  Lane i computes slot i's
-        // fp64 decay; a slot still unpublished after the bound counts as zero.
-        const float uj = exists ? (REV ? -s[jl * R] : s[min(n, (jl + 1) * R) - 1]) : 0.f;
-        const bool brk_me = u_before_tile > uj;
-        const double e_me = brk_me ? exp((double)uj - (double)u_before_tile) : 1.0;
-        // slots are taken 4 at a time: their loads are issued together
-        for (int i0 = 0; i0 <= stop; i0 += 4) {
-            int fk[4];
-            double2 vk[4];
+        double2 vk[Q];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = (i0 + k) & 31;
-                fk[k] = __shfl_sync(0xffffffffu, f, i);
-                if (i0 + k > stop) fk[k] = 0;
-                const int64_t ji = REV ? jb + i : jb - i;
-                vk[k] = make_double2(0.0, 0.0);
-                if (lane < C && (fk[k] == 1 || fk[k] == 2))
-                    vk[k] = (fk[k] == 1) ? __ldcg(&ch.agg[ji * C + lane]) : __ldcg(&ch.inc[ji * C + lane]);
-            }
+        for (int q = 0; q < Q; ++q) {
+            const int i = g + q * SG;
+            const int f = (i <= stop) ? sm.flag[i] : 0;
+            const int64_t ji = REV ? jb + i : jb - i;
+            vk[q] = make_double2(0.0, 0.0);
+            if (f == 1) vk[q] = __ldcg(&ch.agg[ji * C + c]);
+            if (f == 2) vk[q] = __ldcg(&ch.inc[ji * C + c]);
+        }
+        double2 part = make_double2(0.0, 0.0);
+        bool took = false;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = (i0 + k) & 31;
-                const double ei = __shfl_sync(0xffffffffu, e_me, i);
-                const bool bi = __shfl_sync(0xffffffffu, brk_me, i);
-                const bool take = (fk[k] == 1 || fk[k] == 2);
-                if (lane < C && take) {
-                    run.y = fma(ei, vk[k].y, run.y);
-                    run.x = bi ? fma(ei, vk[k].y, run.x) : run.x + vk[k].x;
-                }
-                have = have || take;
+        for (int q = 0; q < Q; ++q) {
+            const int i = g + q * SG;
+            const int f = (i <= stop) ? sm.flag[i] : 0;
+            if (f == 1 || f == 2) {
+                const double e = sm.e[i];
+                part.y = fma(e, vk[q].y, part.y);
+                part.x = sm.brk[i] ? fma(e, vk[q].y, part.x) : part.x + vk[q].x;
+                took = true;
             }
         }
-        if (incl != 0u || timed_out) break;
-        jb = REV ? jb + 32 : jb - 32;
+#pragma unroll
+        for (int off = C; off < 32; off <<= 1) {
+            part.x += __shfl_xor_sync(0xffffffffu, part.x, off);
+            part.y += __shfl_xor_sync(0xffffffffu, part.y, off);
+        }
+        if ((tid & 31) < C) sm.part[tid >> 5][tid & 31] = part;
+        have = __syncthreads_or(took) || have;
+        if (tid < C) {
+            double2 r = sm.run[tid];
+#pragma unroll
+            for (int w = 0; w < NT / 32; ++w) {
+                r.x += sm.part[w][tid].x;
+                r.y += sm.part[w][tid].y;
+            }
+            sm.run[tid] = r;
+        }
+        if (stop < W || timed_out) break;
+        jb = REV ? jb + W : jb - W;
     }
-    if (lane < C) ch.inc[t * C + lane] = have ? lpd_combine(run, u_before_tile, totd, u_tile_end) : totd;
+    __syncthreads();
+    const double2 run = sm.run[c];
+    if (tid < C) ch.inc[t * C + tid] = have ? lpd_combine(run, u_before_tile, totd, u_tile_end) : totd;
     __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release(&ch.flags[t], 2);
+    __syncthreads();
+    if (tid == 0) st_release(&ch.flags[t], 2);
     has_carry = have;
     return run;
 }
