@@ -142,9 +142,11 @@ __global__ void __launch_bounds__(kSideNT) k_side_right(SideScan a, ChainSet cs,
     (void)block_lookback<C, true, NT>(cs.chain(grp), t, a.T, a.s, a.m, R, tot, -s_sm[1], -s_sm[R + 1], status, lb, hc);
 }
 
+// The inputs are read twice (the summaries, then the final sweeps; the second
+// read hits L2) so that none is held through the lookback: two CTAs fit per SM.
 template <int C, bool BINS>
-__global__ void __launch_bounds__(kSideNT) k_side_left(SideScan a, ChainSet left, ChainSet right, unsigned* counters,
-                                                       int32_t* status) {
+__global__ void __launch_bounds__(kSideNT, 2) k_side_left(SideScan a, ChainSet left, ChainSet right,
+                                                          unsigned* counters, int32_t* status) {
     constexpr int NT = kSideNT, E = kSideE, R = kTileValues / C;
     __shared__ float s_sm[R + 2];
     __shared__ uint32_t p_sm[BINS ? 1 : R];
@@ -156,17 +158,21 @@ __global__ void __launch_bounds__(kSideNT) k_side_left(SideScan a, ChainSet left
     if (threadIdx.x == 0) s_tile = (int64_t)atomicAdd(&counters[grp], 1u);
     __syncthreads();
     const int64_t t = s_tile, lo = t * R;
-    side_meta<R>(a, lo, s_sm, p_sm, cw, sw, BINS, !(BINS || C == 1));
-    __syncthreads();
     const int c = threadIdx.x % C, k = threadIdx.x / C;
     const int cb = grp * C + c;
-    float lin[E], tin[E], rin[E], tpin[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) side_inputs<BINS>(a, lo, k * E + e, cb, p_sm, cw, sw, lin[e], tin[e], rin[e], tpin[e]);
+    // the right scan's inclusive state of the next tile (written by the previous launch)
+    const bool hasr = (t + 1 < a.T);
+    const double2 crd = hasr ? __ldcg(&right.chain(grp).inc[(t + 1) * C + c]) : make_double2(0.0, 0.0);
+    side_meta<R>(a, lo, s_sm, p_sm, cw, sw, BINS, !(BINS || C == 1));
+    __syncthreads();
     const float ub_r = -s_sm[(k + 1) * E + 1];
     const float ub_l = s_sm[k * E];
     LP str = {0.f, 0.f}, stl = {0.f, 0.f};
     {
+        float lin[E], tin[E], rin[E], tpin[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            side_inputs<BINS>(a, lo, k * E + e, cb, p_sm, cw, sw, lin[e], tin[e], rin[e], tpin[e]);
         float up = ub_r;
 #pragma unroll
         for (int e = E - 1; e >= 0; --e) {
@@ -192,20 +198,17 @@ __global__ void __launch_bounds__(kSideNT) k_side_left(SideScan a, ChainSet left
         block_lookback<C, false, NT>(left.chain(grp), t, a.T, a.s, a.m, R, tot, s_sm[R], s_sm[0], status, lb, hcl);
     const LP cl = {(float)cin.x, (float)cin.y};
     const LP left_in = seg_incoming(hcl, cl, s_sm[0], hl, exl, ub_l);
-    LP cr = {0.f, 0.f};
-    const bool hasr = (t + 1 < a.T);
-    if (hasr) {
-        const double2 v = __ldcg(&right.chain(grp).inc[(t + 1) * C + c]);
-        cr = LP{(float)v.x, (float)v.y};
-    }
+    const LP cr = {(float)crd.x, (float)crd.y};
     const LP right_in = seg_incoming(hasr, cr, -s_sm[R + 1], hr, exr, ub_r);
     float rres[E];  // values: S; bins: strict R
     LP st = right_in;
     float up = ub_r;
 #pragma unroll
     for (int e = E - 1; e >= 0; --e) {
+        float l, tt, r, tp;
+        side_inputs<BINS>(a, lo, k * E + e, cb, p_sm, cw, sw, l, tt, r, tp);
         const float u = -s_sm[k * E + e + 1];
-        st = lp_step(st, up, u, rin[e], tpin[e]);
+        st = lp_step(st, up, u, r, tp);
         rres[e] = BINS ? st.L : st.P;
         up = u;
     }
@@ -215,8 +218,224 @@ __global__ void __launch_bounds__(kSideNT) k_side_left(SideScan a, ChainSet left
 #pragma unroll
     for (int e = 0; e < E; ++e) {
         const int r = k * E + e;
+        float l, tt, rr, tp;
+        side_inputs<BINS>(a, lo, r, cb, p_sm, cw, sw, l, tt, rr, tp);
         const float u = s_sm[r + 1];
-        st = lp_step(st, up, u, lin[e], tin[e]);
+        st = lp_step(st, up, u, l, tt);
+        up = u;
+        if (cval && lo + r < a.m) {
+            const int64_t idx = (lo + r) * (int64_t)a.Cb + cb;
+            if (BINS) {
+                a.o0[idx] = st.L;
+                a.o1[idx] = rres[e];
+                a.o2[idx] = st.P + rres[e];
+            } else {
+                a.o0[idx] = st.P;
+                a.o1[idx] = rres[e];
+            }
+        }
+    }
+}
+
+// ---------------------------------------------- side scan without waits (T small)
+//
+// When the small side has few tiles the scan runs as two launches with no wait
+// between CTAs: k_side_totals writes each tile's totals in both directions
+// (chain agg arrays), and k_side_apply gives each tile its incoming states
+// directly as sums over all its predecessors' / successors' totals, every term
+// weighted straight to the tile's boundary anchor (the sum form of the
+// recurrence, as in the lookback), then evaluates the tile.  Each apply CTA reads
+// (T - 1) * C totals, so the form is used while T * C stays small.
+constexpr int64_t kSideDirectMaxTiles = 1024;
+constexpr int64_t kSideDirectMaxValues = 8192;  // T * C
+
+template <int C, bool BINS>
+__global__ void __launch_bounds__(kSideNT, 2) k_side_totals(SideScan a, ChainSet left, ChainSet right) {
+    constexpr int NT = kSideNT, E = kSideE, R = kTileValues / C;
+    __shared__ float s_sm[R + 2];
+    __shared__ uint32_t p_sm[BINS ? 1 : R];
+    __shared__ float cw[(BINS || C == 1) ? 1 : R], sw[(BINS || C == 1) ? 1 : R];
+    __shared__ ScanSmem<C, NT / 32> smL, smR;
+    const int grp = blockIdx.y;
+    const int64_t t = blockIdx.x, lo = t * R;
+    side_meta<R>(a, lo, s_sm, p_sm, cw, sw, BINS, !(BINS || C == 1));
+    __syncthreads();
+    const int c = threadIdx.x % C, k = threadIdx.x / C;
+    const int cb = grp * C + c;
+    const float ub_r = -s_sm[(k + 1) * E + 1];
+    const float ub_l = s_sm[k * E];
+    LP str = {0.f, 0.f}, stl = {0.f, 0.f};
+    {
+        float lin[E], tin[E], rin[E], tpin[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            side_inputs<BINS>(a, lo, k * E + e, cb, p_sm, cw, sw, lin[e], tin[e], rin[e], tpin[e]);
+        float up = ub_r;
+#pragma unroll
+        for (int e = E - 1; e >= 0; --e) {
+            const float u = -s_sm[k * E + e + 1];
+            str = lp_step(str, up, u, rin[e], tpin[e]);
+            up = u;
+        }
+        up = ub_l;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float u = s_sm[k * E + e + 1];
+            stl = lp_step(stl, up, u, lin[e], tin[e]);
+            up = u;
+        }
+    }
+    LP exr, exl;
+    bool hr, hl;
+    block_scan_dir<C, NT, true>(str, -s_sm[k * E + 1], ub_r, smR, exr, hr);
+    block_scan_dir<C, NT, false>(stl, s_sm[k * E + E], ub_l, smL, exl, hl);
+    if (threadIdx.x < C) {
+        const LP tl = smL.tot[threadIdx.x], tr = smR.tot[threadIdx.x];
+        left.chain(grp).agg[t * C + threadIdx.x] = make_double2((double)tl.L, (double)tl.P);
+        right.chain(grp).agg[t * C + threadIdx.x] = make_double2((double)tr.L, (double)tr.P);
+    }
+}
+
+// Shared scratch of the direct carries: per other tile its fp64 weight and
+// whether its end lies strictly before the anchor, then the per-warp sums.
+template <int C, int NT>
+struct DirectSmem {
+    double e[kSideDirectMaxTiles];
+    bool brk[kSideDirectMaxTiles];
+    double2 part[2][NT / 32][C];
+    double2 carry[2][C];
+};
+
+// Incoming states of tile t (every thread of the block): left = sum over tiles
+// j < t of their left totals weighted to the row before the tile, right = sum over
+// j > t of their right totals weighted to -(the row after the tile).  A term with
+// decay 1 (its end tied with the anchor) adds its strict part L to L, every other
+// term adds e P to both.  Returns channel tid % C's carries.
+template <int C, int NT>
+__device__ __forceinline__ void direct_carries(const SideScan& a, Chain left, Chain right, int64_t t, int64_t R,
+                                               float u_left, float u_right, DirectSmem<C, NT>& sm, double2& cl,
+                                               double2& cr) {
+    const int64_t T = a.T;
+    const int tid = threadIdx.x, c = tid % C, g = tid / C;
+    constexpr int SG = NT / C;
+    // slot i in [0, T - 1) is tile j = i (< t: left) or i + 1 (> t: right)
+    for (int64_t i = tid; i < T - 1; i += NT) {
+        const int64_t j = i < t ? i : i + 1;
+        const bool isl = j < t;
+        const float uj = isl ? __ldg(a.s + min(a.m, (j + 1) * R) - 1) : -__ldg(a.s + j * R);
+        const float ub = isl ? u_left : u_right;
+        const bool brk = ub > uj;
+        sm.e[i] = brk ? exp((double)uj - (double)ub) : 1.0;
+        sm.brk[i] = brk;
+    }
+    __syncthreads();
+    double2 pl = make_double2(0.0, 0.0), pr = make_double2(0.0, 0.0);
+#pragma unroll 4
+    for (int64_t i = g; i < T - 1; i += SG) {
+        const double e = sm.e[i];
+        if (e == 0.0) continue;  // underflowed: the tile adds nothing
+        const int64_t j = i < t ? i : i + 1;
+        const bool isl = j < t;
+        const double2 v = __ldcg(&(isl ? left : right).agg[j * C + c]);
+        double2& acc = isl ? pl : pr;
+        acc.y = fma(e, v.y, acc.y);
+        acc.x = sm.brk[i] ? fma(e, v.y, acc.x) : acc.x + v.x;
+    }
+#pragma unroll
+    for (int off = C; off < 32; off <<= 1) {
+        pl.x += __shfl_xor_sync(0xffffffffu, pl.x, off);
+        pl.y += __shfl_xor_sync(0xffffffffu, pl.y, off);
+        pr.x += __shfl_xor_sync(0xffffffffu, pr.x, off);
+        pr.y += __shfl_xor_sync(0xffffffffu, pr.y, off);
+    }
+    if ((tid & 31) < C) {
+        sm.part[0][tid >> 5][tid & 31] = pl;
+        sm.part[1][tid >> 5][tid & 31] = pr;
+    }
+    __syncthreads();
+    if (tid < 2 * C) {
+        const int d = tid / C, cc = tid % C;
+        double2 r = make_double2(0.0, 0.0);
+#pragma unroll
+        for (int w = 0; w < NT / 32; ++w) {
+            r.x += sm.part[d][w][cc].x;
+            r.y += sm.part[d][w][cc].y;
+        }
+        sm.carry[d][cc] = r;
+    }
+    __syncthreads();
+    cl = sm.carry[0][c];
+    cr = sm.carry[1][c];
+}
+
+template <int C, bool BINS>
+__global__ void __launch_bounds__(kSideNT, 2) k_side_apply(SideScan a, ChainSet left, ChainSet right) {
+    constexpr int NT = kSideNT, E = kSideE, R = kTileValues / C;
+    __shared__ float s_sm[R + 2];
+    __shared__ uint32_t p_sm[BINS ? 1 : R];
+    __shared__ float cw[(BINS || C == 1) ? 1 : R], sw[(BINS || C == 1) ? 1 : R];
+    __shared__ ScanSmem<C, NT / 32> smL, smR;
+    __shared__ DirectSmem<C, NT> dsm;
+    const int grp = blockIdx.y;
+    const int64_t t = blockIdx.x, lo = t * R;
+    const int c = threadIdx.x % C, k = threadIdx.x / C;
+    const int cb = grp * C + c;
+    const bool hasl = t > 0, hasr = t + 1 < a.T;
+    side_meta<R>(a, lo, s_sm, p_sm, cw, sw, BINS, !(BINS || C == 1));
+    __syncthreads();
+    double2 cld, crd;
+    direct_carries<C, NT>(a, left.chain(grp), right.chain(grp), t, R, s_sm[0], -s_sm[R + 1], dsm, cld, crd);
+    const float ub_r = -s_sm[(k + 1) * E + 1];
+    const float ub_l = s_sm[k * E];
+    LP str = {0.f, 0.f}, stl = {0.f, 0.f};
+    {
+        float lin[E], tin[E], rin[E], tpin[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            side_inputs<BINS>(a, lo, k * E + e, cb, p_sm, cw, sw, lin[e], tin[e], rin[e], tpin[e]);
+        float up = ub_r;
+#pragma unroll
+        for (int e = E - 1; e >= 0; --e) {
+            const float u = -s_sm[k * E + e + 1];
+            str = lp_step(str, up, u, rin[e], tpin[e]);
+            up = u;
+        }
+        up = ub_l;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float u = s_sm[k * E + e + 1];
+            stl = lp_step(stl, up, u, lin[e], tin[e]);
+            up = u;
+        }
+    }
+    LP exr, exl;
+    bool hr, hl;
+    block_scan_dir<C, NT, true>(str, -s_sm[k * E + 1], ub_r, smR, exr, hr);
+    block_scan_dir<C, NT, false>(stl, s_sm[k * E + E], ub_l, smL, exl, hl);
+    const LP left_in = seg_incoming(hasl, LP{(float)cld.x, (float)cld.y}, s_sm[0], hl, exl, ub_l);
+    const LP right_in = seg_incoming(hasr, LP{(float)crd.x, (float)crd.y}, -s_sm[R + 1], hr, exr, ub_r);
+    float rres[E];  // values: S; bins: strict R
+    LP st = right_in;
+    float up = ub_r;
+#pragma unroll
+    for (int e = E - 1; e >= 0; --e) {
+        float l, tt, r, tp;
+        side_inputs<BINS>(a, lo, k * E + e, cb, p_sm, cw, sw, l, tt, r, tp);
+        const float u = -s_sm[k * E + e + 1];
+        st = lp_step(st, up, u, r, tp);
+        rres[e] = BINS ? st.L : st.P;
+        up = u;
+    }
+    st = left_in;
+    up = ub_l;
+    const bool cval = cb < a.Cb;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int r = k * E + e;
+        float l, tt, rr, tp;
+        side_inputs<BINS>(a, lo, r, cb, p_sm, cw, sw, l, tt, rr, tp);
+        const float u = s_sm[r + 1];
+        st = lp_step(st, up, u, l, tt);
         up = u;
         if (cval && lo + r < a.m) {
             const int64_t idx = (lo + r) * (int64_t)a.Cb + cb;
@@ -1330,6 +1549,35 @@ __global__ void __launch_bounds__(256) k_gram_mid(const float* __restrict__ D, c
     }
 }
 
+// The middle of the Gram apply straight from the paired reduce pass's full parts
+// (sorted order, rows of ld floats: w in [0, B), u = A^T g in [B, 2B)).  LPR lanes
+// per sorted row j, original row p = perm[j]: x2[j] = D_p w (sorted order, so that
+// the expand pass reads it without the permutation), w_saved[p] = w (optional) and
+// gD[p] = <u, w>.  Replaces the un-permuting finish and k_gram_mid.
+template <int LPR>
+__global__ void __launch_bounds__(256) k_gram_mid_sorted(const uint32_t* __restrict__ perm, const float* __restrict__ D,
+                                                         const float* __restrict__ ZF, int ld, float* __restrict__ x2,
+                                                         float* __restrict__ w_saved, float* __restrict__ gD,
+                                                         int64_t k, int B) {
+    const int64_t j = (int64_t)blockIdx.x * (256 / LPR) + threadIdx.x / LPR;
+    const int q = threadIdx.x % LPR;
+    const bool in = j < k;
+    const int64_t jj = in ? j : 0;
+    const uint32_t pr = min(__ldg(perm + jj), (uint32_t)(k - 1));
+    const float d = __ldg(D + pr);
+    float acc = 0.f;
+    if (in)
+        for (int c = q; c < B; c += LPR) {
+            const float wv = __ldg(ZF + jj * ld + c);
+            x2[jj * B + c] = d * wv;
+            if (w_saved != nullptr) w_saved[(int64_t)pr * B + c] = wv;
+            acc = fmaf(__ldg(ZF + jj * ld + B + c), wv, acc);
+        }
+#pragma unroll
+    for (int off = LPR / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (in && q == 0) gD[pr] = acc;
+}
+
 // ------------------------------------------------------------------ host side
 
 struct RectPlan {
@@ -1392,6 +1640,14 @@ cudaError_t side_scan_t(const RectPlan& p, SideScan a, int32_t* status, cudaStre
     ChainSet cl{p.flags + (int64_t)p.G * p.T, p.agg + (int64_t)p.G * p.T * p.C, p.inc + (int64_t)p.G * p.T * p.C,
                 p.T, p.C};
     const dim3 grid((unsigned)p.T, (unsigned)p.G);
+    if (p.T <= kSideDirectMaxTiles && p.T * C <= kSideDirectMaxValues) {
+        LAPLEX_TIMED("side_totals", st, k_side_totals<C, BINS><<<grid, kSideNT, 0, st>>>(a, cl, cr));
+        LAPLEX_TIMED("side_apply", st, k_side_apply<C, BINS><<<grid, kSideNT, 0, st>>>(a, cl, cr));
+        return cudaGetLastError();
+    }
+    // the lookback kernels claim tiles from counters and wait on flags: both start at zero
+    const cudaError_t e = cudaMemsetAsync(p.counters, 0, p.memset_bytes, st);
+    if (e != cudaSuccess) return e;
     LAPLEX_TIMED("side_right", st, k_side_right<C, BINS><<<grid, kSideNT, 0, st>>>(a, cr, p.counters, status));
     LAPLEX_TIMED("side_left", st, k_side_left<C, BINS><<<grid, kSideNT, 0, st>>>(a, cl, cr, p.counters + p.G, status));
     return cudaGetLastError();
@@ -1400,8 +1656,6 @@ cudaError_t side_scan_t(const RectPlan& p, SideScan a, int32_t* status, cudaStre
 cudaError_t side_scan(const RectPlan& p, SideScan a, bool bins, int32_t* status, cudaStream_t st) {
     a.T = p.T;
     a.Cb = p.Cb;
-    cudaError_t e = cudaMemsetAsync(p.counters, 0, p.memset_bytes, st);
-    if (e != cudaSuccess) return e;
 #define SIDE_CASE(CC)                                                                                  \
     case CC:                                                                                           \
         return bins ? side_scan_t<CC, true>(p, a, status, st) : side_scan_t<CC, false>(p, a, status, st);
@@ -1902,28 +2156,32 @@ cudaError_t launch_gram(Side A, Side Bs, const float* D, const float* v, int64_t
                         const float* g, float* gD, void* ws, int32_t* status, cudaStream_t st) {
     const RectPlan p2 = plan_rect(A.m, Bs.m, 2 * B, false, ws, Bs.m);  // layout: rows3 after the paired scratch
     const int64_t kb = Bs.m * B;
-    float* wpair = p2.rows3;      // [k][2B]: A^T v | A^T g (paired pass)
-    float* w2 = p2.rows3 + 2 * kb;  // [k][B]: D (A^T v)
+    float* wpair = p2.rows3;      // [k][2B]: A^T v | A^T g (separate passes)
+    float* w2 = p2.rows3 + 2 * kb;  // [k][B]: D (A^T v); in b's sorted order after the paired pass
     if (g != nullptr && gD != nullptr && A.m > Bs.m) {
         // A^T v and A^T g in one reduce pass over the pixel side (2B channels)
         const RectPlan pp = plan_rect(Bs.m, A.m, 2 * B, false, ws);
         const int64_t sz = pp.ms * (int64_t)pp.Cb;
         LAPLEX_TRY(reduce_parts(pp, Bs, A, v, 2 * B, pp.bufA, pp.bufA + sz, pp.bufA + 2 * sz, status, st, g));
-        Finish F{};
-        F.perm = Bs.perm;
-        F.m = Bs.m;
-        F.ZL = pp.bufA;
-        F.ZR = pp.bufA + sz;
-        F.ZF = pp.bufA + 2 * sz;
-        F.B = (int)(2 * B);
-        F.Cb = pp.Cb;
-        F.out = wpair;
-        LAPLEX_TRY(finish(F, st));
-        LAPLEX_TIMED("gram_mid", st,
-                     k_gram_mid<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, wpair, 2 * B, wpair + B, w2, w_saved,
-                                                                           gD, Bs.m, (int)B));
+        // w2 = D w in b's sorted order, so the expand reads b's side without the permutation
+        const float* ZF = pp.bufA + 2 * sz;
+        const int ld = pp.Cb;
+#define GRAM_MID_CASE(LP)                                                                                    \
+    LAPLEX_TIMED("gram_mid", st,                                                                           \
+                 k_gram_mid_sorted<LP><<<(unsigned)((Bs.m + (256 / LP) - 1) / (256 / LP)), 256, 0, st>>>(  \
+                     Bs.perm, D, ZF, ld, w2, w_saved, gD, Bs.m, (int)B))
+        if (B <= 4)
+            GRAM_MID_CASE(4);
+        else if (B <= 8)
+            GRAM_MID_CASE(8);
+        else if (B <= 16)
+            GRAM_MID_CASE(16);
+        else
+            GRAM_MID_CASE(32);
+#undef GRAM_MID_CASE
         LAPLEX_TRY(cudaGetLastError());
-        return launch_rect_forward(A, Bs, w2, B, y, nullptr, ws, status, st);  // y = A (D w)
+        const Side Bsorted{Bs.s, nullptr, nullptr, Bs.m};
+        return launch_rect_forward(A, Bsorted, w2, B, y, nullptr, ws, status, st);  // y = A (D w)
     }
     float* w = w_saved ? w_saved : wpair;
     float* wg = wpair + kb;

@@ -194,9 +194,13 @@ __device__ __forceinline__ double2 block_lookback(Chain ch, int64_t t, int64_t T
     const int tid = threadIdx.x, c = tid % C, g = tid / C;
     const bool first = REV ? (t == T - 1) : (t == 0);
     const double2 totd = make_double2((double)tot.L, (double)tot.P);
+    // only the threads that wrote a value fence before the block barrier that
+    // precedes the flag's release
     if (first) {
-        if (tid < C) ch.inc[t * C + tid] = totd;
-        __threadfence();
+        if (tid < C) {
+            ch.inc[t * C + tid] = totd;
+            __threadfence();
+        }
         __syncthreads();
         if (tid == 0) st_release(&ch.flags[t], 2);
         has_carry = false;
@@ -206,8 +210,8 @@ __device__ __forceinline__ double2 block_lookback(Chain ch, int64_t t, int64_t T
     if (tid < C) {
         ch.agg[t * C + tid] = totd;
         sm.run[tid] = make_double2(0.0, 0.0);
+        __threadfence();
     }
-    __threadfence();
     __syncthreads();
     if (tid == 0) st_release(&ch.flags[t], 1);
     bool have = false;
@@ -291,8 +295,10 @@ __device__ __forceinline__ double2 block_lookback(Chain ch, int64_t t, int64_t T
     }
     __syncthreads();
     const double2 run = sm.run[c];
-    if (tid < C) ch.inc[t * C + tid] = have ? lpd_combine(run, u_before_tile, totd, u_tile_end) : totd;
-    __threadfence();
+    if (tid < C) {
+        ch.inc[t * C + tid] = have ? lpd_combine(run, u_before_tile, totd, u_tile_end) : totd;
+        __threadfence();
+    }
     __syncthreads();
     if (tid == 0) st_release(&ch.flags[t], 2);
     has_carry = have;

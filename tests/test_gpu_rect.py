@@ -76,6 +76,22 @@ def test_rect_ops(L, op, n, k, B, quant, saved):
     compare_rect(L, op, a, b, x, g, phi, psi, saved, tag=f"n{n} k{k} B{B} q{quant} saved{saved}")
 
 
+@pytest.mark.parametrize("op", ["general", "phased_transpose"])
+def test_rect_small_side_past_direct_tiles(L, op):
+    """A small side of more than 1024 scan tiles (600 000 rows, 16 scan channels:
+    B = 16, or B = 8 phased: 2344 tiles), so that its scans take the
+    decoupled-lookback kernels instead of the totals-then-apply pair."""
+    phased, transpose = OPS[op]
+    B = 8 if phased else 16
+    n, k = 600_000, 600_011
+    a, b, rng = draw(n, k, B, seed=77, quant=0.002, span=2000.0)
+    x = rng.standard_normal(((n if transpose else k), B)).astype(np.float32)
+    g = rng.standard_normal(((k if transpose else n), B)).astype(np.float32)
+    phi = rng.uniform(0, 2 * np.pi, n).astype(np.float32)
+    psi = rng.uniform(0, 2 * np.pi, k).astype(np.float32)
+    compare_rect(L, op, a, b, x, g, phi, psi, saved=True, tag=f"n{n} k{k} B{B}")
+
+
 def test_phased_head_full_size(L):
     """n = 2^22 -> k = 1024 phased head, B = 128, forward and all five gradients."""
     w = inputs.phased_head_2p22(0)
