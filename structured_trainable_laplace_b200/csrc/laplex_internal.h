@@ -108,6 +108,10 @@ struct Side {
     const uint32_t* perm;  // s[r] = anchors[perm[r]]
     const float* theta;    // phases in original order, or nullptr
     int64_t m;             // number of anchors
+    // the vector rows read at this side (the input of a scan over it, the h of its
+    // finish) are stored in sorted order, row r at sorted position r; outputs are
+    // still placed through perm.  Only without phases.
+    bool rows_sorted = false;
 };
 
 size_t rect_workspace_bytes(int64_t n_out, int64_t n_in, int64_t B, bool phased);

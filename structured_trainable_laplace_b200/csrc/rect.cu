@@ -1473,7 +1473,8 @@ struct Finish {
     const float* ZF;
     int B;
     int Cb;
-    const float* h;  // [m][B] original order (for gradients)
+    const float* h;  // [m][B] original order (for gradients), or sorted order when h_sorted
+    bool h_sorted;
     float* out;      // [m][B] original order: sum_p w_p ZF
     float* g_anchor;  // sum_c h sum_p w_p (ZR - ZL)
     float* g_phase;   // sum_c h sum_p w'_p ZF
@@ -1501,7 +1502,7 @@ __global__ void __launch_bounds__(256) k_finish(Finish F) {
     }
     float ga = 0.f, gp = 0.f;
     for (int c = lane; c < F.B; c += 32) {
-        const float hv = F.h ? __ldg(F.h + (int64_t)pr * F.B + c) : 0.f;
+        const float hv = F.h ? __ldg(F.h + (int64_t)(F.h_sorted ? r : pr) * F.B + c) : 0.f;
         float o = 0.f;
 #pragma unroll
         for (int p = 0; p < NP; ++p) {
@@ -1549,15 +1550,16 @@ __global__ void __launch_bounds__(256) k_gram_mid(const float* __restrict__ D, c
     }
 }
 
-// The middle of the Gram apply straight from the paired reduce pass's full parts
-// (sorted order, rows of ld floats: w in [0, B), u = A^T g in [B, 2B)).  LPR lanes
-// per sorted row j, original row p = perm[j]: x2[j] = D_p w (sorted order, so that
-// the expand pass reads it without the permutation), w_saved[p] = w (optional) and
-// gD[p] = <u, w>.  Replaces the un-permuting finish and k_gram_mid.
-template <int LPR>
+// The middle of the Gram operator straight from the paired reduce pass's full parts
+// (sorted order, rows of ld floats: w = A^T v in [0, B), u = A^T g in [B, 2B)).
+// LPR lanes per sorted row j, original row p = perm[j]: x[j] = D_p w, followed by
+// D_p u when WITH_U (rows of x_ld floats, sorted order, so that the next scan reads
+// them without the permutation), w_saved[p] = w (optional) and gD[p] = <u, w>
+// (optional).
+template <int LPR, bool WITH_U>
 __global__ void __launch_bounds__(256) k_gram_mid_sorted(const uint32_t* __restrict__ perm, const float* __restrict__ D,
-                                                         const float* __restrict__ ZF, int ld, float* __restrict__ x2,
-                                                         float* __restrict__ w_saved, float* __restrict__ gD,
+                                                         const float* __restrict__ ZF, int ld, float* __restrict__ x,
+                                                         int x_ld, float* __restrict__ w_saved, float* __restrict__ gD,
                                                          int64_t k, int B) {
     const int64_t j = (int64_t)blockIdx.x * (256 / LPR) + threadIdx.x / LPR;
     const int q = threadIdx.x % LPR;
@@ -1568,14 +1570,34 @@ __global__ void __launch_bounds__(256) k_gram_mid_sorted(const uint32_t* __restr
     float acc = 0.f;
     if (in)
         for (int c = q; c < B; c += LPR) {
-            const float wv = __ldg(ZF + jj * ld + c);
-            x2[jj * B + c] = d * wv;
+            const float wv = __ldg(ZF + jj * ld + c), uv = __ldg(ZF + jj * ld + B + c);
+            x[jj * x_ld + c] = d * wv;
+            if (WITH_U) x[jj * x_ld + B + c] = d * uv;
             if (w_saved != nullptr) w_saved[(int64_t)pr * B + c] = wv;
-            acc = fmaf(__ldg(ZF + jj * ld + B + c), wv, acc);
+            acc = fmaf(uv, wv, acc);
         }
 #pragma unroll
     for (int off = LPR / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (in && q == 0) gD[pr] = acc;
+    if (in && q == 0 && gD != nullptr) gD[pr] = acc;
+}
+
+template <bool WITH_U>
+cudaError_t launch_gram_mid_sorted(const uint32_t* perm, const float* D, const float* ZF, int ld, float* x, int x_ld,
+                                   float* w_saved, float* gD, int64_t k, int64_t B, cudaStream_t st) {
+#define GRAM_MID_CASE(LP)                                                                                       \
+    LAPLEX_TIMED("gram_mid", st,                                                                              \
+                 (k_gram_mid_sorted<LP, WITH_U><<<(unsigned)((k + (256 / LP) - 1) / (256 / LP)), 256, 0, st>>>( \
+                     perm, D, ZF, ld, x, x_ld, w_saved, gD, k, (int)B)))
+    if (B <= 4)
+        GRAM_MID_CASE(4);
+    else if (B <= 8)
+        GRAM_MID_CASE(8);
+    else if (B <= 16)
+        GRAM_MID_CASE(16);
+    else
+        GRAM_MID_CASE(32);
+#undef GRAM_MID_CASE
+    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ host side
@@ -1887,7 +1909,7 @@ cudaError_t finish(Finish F, cudaStream_t st) {
 SideScan values_scan(Side S, const float* X, int64_t B, float* P, float* Sout) {
     SideScan a{};
     a.s = S.s;
-    a.perm = S.perm;
+    a.perm = S.rows_sorted ? nullptr : S.perm;  // no permutation: row r is sorted row r
     a.theta = S.theta;
     a.m = S.m;
     a.X = X;
@@ -2034,6 +2056,7 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
                 F.B = (int)B;
                 F.Cb = p.Cb;
                 F.h = g;
+                F.h_sorted = O.rows_sorted;
                 F.g_anchor = gO;
                 F.g_phase = gtO;
                 F.accumulate = accumulate;
@@ -2096,6 +2119,7 @@ cudaError_t launch_rect_backward(Side O, Side I, const float* x, const float* g,
         F.B = (int)B;
         F.Cb = p.Cb;
         F.h = x;
+        F.h_sorted = I.rows_sorted;
         F.out = gx;
         F.g_anchor = gI;
         F.g_phase = gtI;
@@ -2115,15 +2139,12 @@ cudaError_t launch_check_wait_bound(void* ws, int32_t* status, cudaStream_t st) 
     return cudaGetLastError();
 }
 
-// The middle of the Gram backward, one warp per small-side row j: x1 = D_j w_j,
-// x2 = D_j u_j (the inputs of the general products A (D w) and A (D u)) and
-// gD_j = <u_j, w_j>.  w and u are rows of ld floats.
-// xp (nullable): [k][2B], D_j w_j followed by D_j u_j (the input of the paired
-// backward, which takes both general products at once).
+// The middle of the Gram backward after separate passes, one warp per small-side
+// row j (original order): x1 = D_j w_j, x2 = D_j u_j (the inputs of the general
+// products A (D w) and A (D u)) and gD_j = <u_j, w_j>.  w and u are rows of ld floats.
 __global__ void __launch_bounds__(256) k_gram_mid2(const float* __restrict__ D, const float* __restrict__ w,
                                                    const float* __restrict__ u, int ld, float* __restrict__ x1,
-                                                   float* __restrict__ x2, float* __restrict__ xp,
-                                                   float* __restrict__ gD, int64_t k, int B) {
+                                                   float* __restrict__ x2, float* __restrict__ gD, int64_t k, int B) {
     const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (r >= k) return;
     const int lane = threadIdx.x & 31;
@@ -2133,10 +2154,6 @@ __global__ void __launch_bounds__(256) k_gram_mid2(const float* __restrict__ D, 
         const float wv = __ldg(w + r * ld + c), uv = __ldg(u + r * ld + c);
         x1[r * B + c] = d * wv;
         x2[r * B + c] = d * uv;
-        if (xp != nullptr) {
-            xp[r * 2 * B + c] = d * wv;
-            xp[r * 2 * B + B + c] = d * uv;
-        }
         acc = fmaf(uv, wv, acc);
     }
     if (gD != nullptr) {
@@ -2164,24 +2181,10 @@ cudaError_t launch_gram(Side A, Side Bs, const float* D, const float* v, int64_t
         const int64_t sz = pp.ms * (int64_t)pp.Cb;
         LAPLEX_TRY(reduce_parts(pp, Bs, A, v, 2 * B, pp.bufA, pp.bufA + sz, pp.bufA + 2 * sz, status, st, g));
         // w2 = D w in b's sorted order, so the expand reads b's side without the permutation
-        const float* ZF = pp.bufA + 2 * sz;
-        const int ld = pp.Cb;
-#define GRAM_MID_CASE(LP)                                                                                    \
-    LAPLEX_TIMED("gram_mid", st,                                                                           \
-                 k_gram_mid_sorted<LP><<<(unsigned)((Bs.m + (256 / LP) - 1) / (256 / LP)), 256, 0, st>>>(  \
-                     Bs.perm, D, ZF, ld, w2, w_saved, gD, Bs.m, (int)B))
-        if (B <= 4)
-            GRAM_MID_CASE(4);
-        else if (B <= 8)
-            GRAM_MID_CASE(8);
-        else if (B <= 16)
-            GRAM_MID_CASE(16);
-        else
-            GRAM_MID_CASE(32);
-#undef GRAM_MID_CASE
-        LAPLEX_TRY(cudaGetLastError());
-        const Side Bsorted{Bs.s, nullptr, nullptr, Bs.m};
-        return launch_rect_forward(A, Bsorted, w2, B, y, nullptr, ws, status, st);  // y = A (D w)
+        LAPLEX_TRY(launch_gram_mid_sorted<false>(Bs.perm, D, pp.bufA + 2 * sz, pp.Cb, w2, (int)B, w_saved, gD, Bs.m,
+                                                 B, st));
+        const Side Bss{Bs.s, Bs.perm, nullptr, Bs.m, true};
+        return launch_rect_forward(A, Bss, w2, B, y, nullptr, ws, status, st);  // y = A (D w)
     }
     float* w = w_saved ? w_saved : wpair;
     float* wg = wpair + kb;
@@ -2204,53 +2207,28 @@ cudaError_t launch_gram_backward(Side A, Side Bs, const float* D, const float* v
                                  cudaStream_t st) {
     const RectPlan p2 = plan_rect(A.m, Bs.m, 2 * B, false, ws, Bs.m);
     const int64_t kb = Bs.m * B;
-    float* wpair = p2.rows3;           // [k][2B] (paired) or w | u ([k][B] each)
+    float* wpair = p2.rows3;           // w | u ([k][B] each, separate passes)
     float* x1 = p2.rows3 + 2 * kb;     // [k][B]  D w
     float* x2 = p2.rows3 + 3 * kb;     // [k][B]  D u
-    float* xp = p2.rows3 + 4 * kb;     // [k][2B] D w | D u (paired backward)
-    const bool paired = A.m > Bs.m;
-    const float* w;
-    const float* u;
-    int ld;
-    if (paired) {  // A^T v and A^T g in one paired reduce pass
+    float* xp = p2.rows3 + 4 * kb;     // [k][2B] D w | D u in b's sorted order (paired pass)
+    const bool need_ab = ga != nullptr || gb != nullptr;
+    if (A.m > Bs.m) {
+        // A^T v and A^T g in one paired reduce pass; then D w | D u (and gD) in b's
+        // sorted order, and the scan states of D w | D u over b, once: the paired
+        // backward reads them, and their second half (D u) gives gv = A (D u)
         const RectPlan pp = plan_rect(Bs.m, A.m, 2 * B, false, ws);
         const int64_t sz = pp.ms * (int64_t)pp.Cb;
         LAPLEX_TRY(reduce_parts(pp, Bs, A, v, 2 * B, pp.bufA, pp.bufA + sz, pp.bufA + 2 * sz, status, st, g));
-        Finish F{};
-        F.perm = Bs.perm;
-        F.m = Bs.m;
-        F.ZL = pp.bufA;
-        F.ZR = pp.bufA + sz;
-        F.ZF = pp.bufA + 2 * sz;
-        F.B = (int)(2 * B);
-        F.Cb = pp.Cb;
-        F.out = wpair;
-        LAPLEX_TRY(finish(F, st));
-        w = wpair;
-        u = wpair + B;
-        ld = (int)(2 * B);
-    } else {
-        LAPLEX_TRY(launch_rect_forward(Bs, A, v, B, wpair, nullptr, ws, status, st));       // w = A^T v
-        LAPLEX_TRY(launch_rect_forward(Bs, A, g, B, wpair + kb, nullptr, ws, status, st));  // u = A^T g
-        w = wpair;
-        u = wpair + kb;
-        ld = (int)B;
-    }
-    const bool need_ab = ga != nullptr || gb != nullptr;
-    LAPLEX_TIMED("gram_mid", st,
-                 k_gram_mid2<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, w, u, ld, x1, x2,
-                                                                        (paired && need_ab) ? xp : nullptr, gD, Bs.m,
-                                                                        (int)B));
-    LAPLEX_TRY(cudaGetLastError());
-    if (need_ab && paired) {
-        // the scan states of D w | D u over b, once: the paired backward reads them, and
-        // their second half (D u) gives gv = A (D u) without a scan of its own
+        LAPLEX_TRY(launch_gram_mid_sorted<true>(Bs.perm, D, pp.bufA + 2 * sz, pp.Cb, xp, (int)(2 * B), nullptr, gD,
+                                                Bs.m, B, st));
+        if (gv == nullptr && !need_ab) return cudaSuccess;
+        const Side Bss{Bs.s, Bs.perm, nullptr, Bs.m, true};
         const RectPlan pb = plan_rect(A.m, Bs.m, 2 * B, false, ws);
         const int64_t szb = pb.ms * (int64_t)pb.Cb;
         float* P = pb.bufA;
-        LAPLEX_TRY(side_scan(pb, values_scan(Bs, xp, 2 * B, P, P + szb), false, status, st));
+        LAPLEX_TRY(side_scan(pb, values_scan(Bss, xp, 2 * B, P, P + szb), false, status, st));
         if (gv != nullptr) {
-            LargePass E = large_args(A, Bs, pb, B);  // B channels, states with the 2B-channel stride
+            LargePass E = large_args(A, Bss, pb, B);  // B channels, states with the 2B-channel stride
             E.Pst = P + B;
             E.Sst = P + szb + B;
             E.out = gv;
@@ -2258,10 +2236,17 @@ cudaError_t launch_gram_backward(Side A, Side Bs, const float* D, const float* v
         }
         // both general products in one backward over 2B channels: inputs D w | D u at
         // b, rows g | v at a (ga sums over all 2B channels, and so does gb)
-        LAPLEX_TRY(launch_rect_backward(A, Bs, xp, g, 2 * B, P, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
-                                        false, v));
+        if (need_ab)
+            LAPLEX_TRY(launch_rect_backward(A, Bss, xp, g, 2 * B, P, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
+                                            false, v));
         return cudaSuccess;
     }
+    LAPLEX_TRY(launch_rect_forward(Bs, A, v, B, wpair, nullptr, ws, status, st));       // w = A^T v
+    LAPLEX_TRY(launch_rect_forward(Bs, A, g, B, wpair + kb, nullptr, ws, status, st));  // u = A^T g
+    LAPLEX_TIMED("gram_mid", st,
+                 k_gram_mid2<<<(unsigned)((Bs.m + 7) / 8), 256, 0, st>>>(D, wpair, wpair + kb, (int)B, x1, x2, gD,
+                                                                        Bs.m, (int)B));
+    LAPLEX_TRY(cudaGetLastError());
     if (gv != nullptr) LAPLEX_TRY(launch_rect_forward(A, Bs, x2, B, gv, nullptr, ws, status, st));  // gv = A (D u)
     if (need_ab) {
         LAPLEX_TRY(launch_rect_backward(A, Bs, x1, g, B, nullptr, nullptr, ga, gb, nullptr, nullptr, ws, status, st,
