@@ -11,8 +11,9 @@
 //   k_sym_agg    walks its ranges right to left and writes, per tile, the fp64
 //                suffix state of the base range from that tile's first row on
 //                (RS), and each base range's aggregates in both directions;
-//   k_sym_carry  scans the P range aggregates (one CTA per channel group) into
-//                the fp64 carries entering each base range from the left/right;
+//   k_sym_carry_direct  gives each base range its fp64 carries from the
+//                left/right as sums of the other ranges' aggregates, each
+//                weighted straight to the range's boundary;
 //   k_sym_sweep  walks its ranges left to right, folding the left state tile by
 //                tile and taking the right state from RS and the range carry,
 //                evaluates both directions inside each tile and writes
@@ -428,112 +429,96 @@ __global__ void __launch_bounds__(SymGeo<C>::NT, (SymGeo<C>::NT == 256 ? 3 : 1))
 
 // ------------------------------------------------------------------ pass B
 
-// One CTA of kCarryThreads per channel group.  First every thread computes the
-// fp64 decays between consecutive range ends (shared by all channels) into
-// shared memory, so that the scans below are chains of fused multiply-adds only.
-// Thread (c, q) owns block q of PS consecutive ranges: it folds their aggregates
-// in both directions, the NB block aggregates are scanned in shared memory by
-// doubling (log2 NB steps), and each thread then re-walks its block, writing the
-// carry entering every range.
-constexpr int kCarryThreads = 1024;
-constexpr int kCarryBatch = 4;
-
-// Decay between the end anchors of two consecutive ranges, encoded with its break
-// flag: exp(uA - uB) when uB > uA, -1 for a tie (decay 1, no break).
-__device__ __forceinline__ double enc_decay_d(float uA, float uB) {
-    return (uB > uA) ? exp((double)uA - (double)uB) : -1.0;
-}
-
-__device__ __forceinline__ double2 fold_d(double2 A, double2 B, double ev) {
-    return combine_ed(A, B, fabs(ev), ev >= 0.0);
-}
+// The carries entering each base range, from the range aggregates, in direct form:
+// one CTA per base range J (grid P x G).  The carry from the left is the sum over
+// the ranges J' < J of their left aggregates,
+// each weighted by the fp64 decay from its end straight to the row before J (a
+// range whose end ties with that row adds its strict part L to L), and mirrored
+// from the right.  The anchors are sorted, so the weights fall with the distance:
+// ranges are taken in windows of kDirW nearest ones per side, and the walk stops
+// at the first weight that underflows to zero (every farther one does too).  No
+// chain of dependent folds: a window is one round of loads and a block reduction.
+constexpr int kDirNT = 128;
+constexpr int kDirW = 64;
 
 template <int C>
-__global__ void __launch_bounds__(kCarryThreads) k_sym_carry(SymScan a, RangeState st) {
-    constexpr int QS = kCarryThreads / C;
-    __shared__ double2 sL[QS][C], sR[QS][C];
-    extern __shared__ double s_dec[];  // [2][P]: left decay into range j (from j-1), right decay into j (from j+1)
-    const int grp = blockIdx.x;
-    const int c = threadIdx.x % C, q = threadIdx.x / C;
-    const int P = a.P;
-    const int PS = (P + QS - 1) / QS, NB = (P + PS - 1) / PS;
-    const int j0 = min(P, q * PS), j1 = min(P, j0 + PS);
+__global__ void __launch_bounds__(kDirNT) k_sym_carry_direct(SymScan a, RangeState st) {
+    constexpr int SG = kDirNT / C;  // slot groups
+    __shared__ double s_e[2][kDirW];
+    __shared__ bool s_brk[2][kDirW];
+    __shared__ double2 s_part[2][kDirNT / 32][C];
+    __shared__ int s_more;
+    const int J = blockIdx.x, grp = blockIdx.y, P = a.P;
+    const int tid = threadIdx.x, c = tid % C, g = tid / C;
     const int64_t RR = a.tpr * (int64_t)tile_rows<C>();  // rows per range
-    auto uL = [&](int jj) { return __ldg(a.s + min(a.n, (jj + 1) * RR) - 1); };  // left anchor of range jj
-    auto uR = [&](int jj) { return -__ldg(a.s + jj * RR); };                    // right anchor of range jj
-    double* dL = s_dec;
-    double* dR = s_dec + P;
-    for (int jj = threadIdx.x; jj < P; jj += kCarryThreads) {
-        dL[jj] = jj > 0 ? enc_decay_d(uL(jj - 1), uL(jj)) : 0.0;
-        dR[jj] = jj + 1 < P ? enc_decay_d(uR(jj + 1), uR(jj)) : 0.0;
-    }
-    const double2* Lagg = st.Lagg + (int64_t)grp * P * C + c;
-    const double2* Ragg = st.Ragg + (int64_t)grp * P * C + c;
-    const bool mine = q < NB;  // blocks q >= NB are empty
-    __syncthreads();
-
-    // block aggregates (left: ranges j0 .. j1-1 in order; right: j1-1 .. j0); the
-    // aggregates are loaded kCarryBatch at a time, ahead of the dependent folds
-    if (mine) {
-        double2 fl = make_double2(0.0, 0.0), fr = make_double2(0.0, 0.0);
-        for (int ub = 0; ub < j1 - j0; ub += kCarryBatch) {
-            double2 vl[kCarryBatch], vr[kCarryBatch];
-#pragma unroll
-            for (int u = 0; u < kCarryBatch; ++u) {
-                const int uu = min(ub + u, j1 - j0 - 1);
-                vl[u] = Lagg[(int64_t)(j0 + uu) * C];
-                vr[u] = Ragg[(int64_t)(j1 - 1 - uu) * C];
+    auto uL = [&](int jj) { return __ldg(a.s + min(a.n, (jj + 1) * RR) - 1); };  // left aggregate's anchor
+    auto uR = [&](int jj) { return -__ldg(a.s + jj * RR); };                    // right aggregate's anchor
+    const float ubL = J > 0 ? uL(J - 1) : 0.f;       // the row before range J
+    const float ubR = J + 1 < P ? uR(J + 1) : 0.f;   // -(the row after range J)
+    const double2* Lagg = st.Lagg + (int64_t)grp * P * C;
+    const double2* Ragg = st.Ragg + (int64_t)grp * P * C;
+    double2 accL = make_double2(0.0, 0.0), accR = make_double2(0.0, 0.0);
+    for (int base = 0;; base += kDirW) {
+        // weights of this window: slot i is range J-1-base-i (left) / J+1+base+i (right)
+        if (tid < 2 * kDirW) {
+            const int side = tid / kDirW, i = tid % kDirW;
+            const int jj = side ? J + 1 + base + i : J - 1 - base - i;
+            double e = 0.0;
+            bool brk = true;
+            if (jj >= 0 && jj < P) {
+                const float uj = side ? uR(jj) : uL(jj), ub = side ? ubR : ubL;
+                brk = ub > uj;
+                e = brk ? exp((double)uj - (double)ub) : 1.0;
             }
+            s_e[side][i] = e;
+            s_brk[side][i] = brk;
+        }
+        if (tid == 0) s_more = 0;
+        __syncthreads();
 #pragma unroll
-            for (int u = 0; u < kCarryBatch; ++u) {
-                const int uu = ub + u;
-                if (uu >= j1 - j0) break;
-                fl = uu ? fold_d(fl, vl[u], dL[j0 + uu]) : vl[u];
-                fr = uu ? fold_d(fr, vr[u], dR[j1 - 1 - uu]) : vr[u];
+        for (int side = 0; side < 2; ++side) {
+            const double2* agg = side ? Ragg : Lagg;
+            double2& acc = side ? accR : accL;
+            for (int i = g; i < kDirW; i += SG) {
+                const double e = s_e[side][i];
+                if (e == 0.0) continue;  // underflowed (or past the ends): adds nothing
+                const int jj = side ? J + 1 + base + i : J - 1 - base - i;
+                const double2 v = __ldcg(agg + (int64_t)jj * C + c);
+                acc.y = fma(e, v.y, acc.y);
+                acc.x = s_brk[side][i] ? fma(e, v.y, acc.x) : acc.x + v.x;
             }
         }
-        sL[q][c] = fl;
-        sR[q][c] = fr;
+        // another window only while the farthest range of this one still contributes
+        if (tid == 0 && ((s_e[0][kDirW - 1] != 0.0 && J - 1 - base - kDirW >= 0) ||
+                         (s_e[1][kDirW - 1] != 0.0 && J + 1 + base + kDirW < P)))
+            s_more = 1;
+        __syncthreads();
+        const bool more = s_more != 0;
+        __syncthreads();  // the window's weights are read before the next one writes them
+        if (!more) break;
+    }
+#pragma unroll
+    for (int off = C; off < 32; off <<= 1) {
+        accL.x += __shfl_xor_sync(0xffffffffu, accL.x, off);
+        accL.y += __shfl_xor_sync(0xffffffffu, accL.y, off);
+        accR.x += __shfl_xor_sync(0xffffffffu, accR.x, off);
+        accR.y += __shfl_xor_sync(0xffffffffu, accR.y, off);
+    }
+    if ((tid & 31) < C) {
+        s_part[0][tid >> 5][tid & 31] = accL;
+        s_part[1][tid >> 5][tid & 31] = accR;
     }
     __syncthreads();
-    // inclusive scans over the blocks: left over 0..q, right over q..NB-1; the decay
-    // between block q-off's end and block q's end is the product of the range
-    // decays between them, taken here as exp of the anchor difference
-    for (int off = 1; off < NB; off <<= 1) {
-        const bool dl = mine && q >= off, dr = mine && q + off < NB;
-        double2 nl, nr;
-        if (dl) nl = fold_d(sL[q - off][c], sL[q][c], enc_decay_d(uL(min(P, (q - off + 1) * PS) - 1), uL(j1 - 1)));
-        if (dr) nr = fold_d(sR[q + off][c], sR[q][c], enc_decay_d(uR((q + off) * PS), uR(j0)));
-        __syncthreads();
-        if (dl) sL[q][c] = nl;
-        if (dr) sR[q][c] = nr;
-        __syncthreads();
-    }
-    if (!mine) return;
-    // carries entering the block, then entering each of its ranges
-    double2* Lin = st.Lin + (int64_t)grp * P * C + c;
-    double2* Rin = st.Rin + (int64_t)grp * P * C + c;
-    const bool hl = q >= 1, hr = q + 1 < NB;
-    double2 cl = hl ? sL[q - 1][c] : make_double2(0.0, 0.0);
-    double2 cr = hr ? sR[q + 1][c] : make_double2(0.0, 0.0);
-    for (int ub = 0; ub < j1 - j0; ub += kCarryBatch) {
-        double2 vl[kCarryBatch], vr[kCarryBatch];
+    if (tid < 2 * C) {
+        const int side = tid / C, cc = tid % C;
+        double2 r = make_double2(0.0, 0.0);
 #pragma unroll
-        for (int u = 0; u < kCarryBatch; ++u) {
-            const int uu = min(ub + u, j1 - j0 - 1);
-            vl[u] = Lagg[(int64_t)(j0 + uu) * C];
-            vr[u] = Ragg[(int64_t)(j1 - 1 - uu) * C];
+        for (int w = 0; w < kDirNT / 32; ++w) {
+            r.x += s_part[side][w][cc].x;
+            r.y += s_part[side][w][cc].y;
         }
-#pragma unroll
-        for (int u = 0; u < kCarryBatch; ++u) {
-            const int uu = ub + u;
-            if (uu >= j1 - j0) break;
-            const int jl = j0 + uu, jr = j1 - 1 - uu;
-            Lin[(int64_t)jl * C] = cl;  // zero (unused) for the first range
-            Rin[(int64_t)jr * C] = cr;  // zero (unused) for the last range
-            cl = (hl || uu > 0) ? fold_d(cl, vl[u], dL[jl]) : vl[u];
-            cr = (hr || uu > 0) ? fold_d(cr, vr[u], dR[jr]) : vr[u];
-        }
+        // zero (unused) for the first range's left and the last range's right carry
+        (side ? st.Rin : st.Lin)[((int64_t)grp * P + J) * C + cc] = r;
     }
 }
 
@@ -1322,14 +1307,8 @@ cudaError_t sym_ranges_t(const SymPlan& p, const float* s, const uint32_t* perm,
                      k_sym_agg<C, kAheadAgg><<<grid, SymGeo<C>::NT, sizeof(SM), stream>>>(a, v, st, vs));
     }
     const SymScan a = scan_args(p, s, perm, n, B, sms, 1);
-    const size_t dsm = sizeof(double) * 2 * (size_t)p.P;
-    static PerDevice carry_ready;
-    if (!carry_ready.here()) {
-        cudaFuncSetAttribute(k_sym_carry<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(sizeof(double) * 2 * kMaxRanges));
-        carry_ready.here() = 1;
-    }
-    LAPLEX_TIMED("sym_carry", stream, k_sym_carry<C><<<p.G, kCarryThreads, dsm, stream>>>(a, st));
+    LAPLEX_TIMED("sym_carry", stream,
+                 k_sym_carry_direct<C><<<dim3((unsigned)p.P, (unsigned)p.G), kDirNT, 0, stream>>>(a, st));
     return cudaGetLastError();
 }
 
