@@ -21,6 +21,12 @@ namespace {
 constexpr int kNT = 256;
 constexpr int kItems = 15;  // 3840-key tiles: with the values loaded late, four CTAs per SM
 constexpr int kTile = kNT * kItems;
+// Up to kShortMax keys a sort can take tiles of kItemsShort keys per thread
+// instead, when its grid is a few waves and the smaller tiles end the last wave
+// sooner (see sort_items); its workspace is sized for the smaller tiles.
+constexpr int kItemsShort = 11;
+constexpr int kTileShort = kNT * kItemsShort;
+constexpr int64_t kShortMax = 1ll << 23;
 constexpr int kNW = kNT / 32;
 constexpr int kRadix = 256;
 constexpr unsigned long long kValMask = (1ull << 62) - 1;
@@ -56,11 +62,12 @@ __device__ __forceinline__ uint32_t block_excl_scan_256(uint32_t v, uint32_t* s_
 }
 
 __global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a, int64_t n, const int64_t* n_dev,
-                                                    uint32_t* hist, unsigned long long* look0, int32_t* status) {
+                                                    int tile_keys, uint32_t* hist, unsigned long long* look0,
+                                                    int32_t* status) {
     __shared__ uint32_t s_hist[kNW][4][kRadix];  // one histogram set per warp: fewer colliding atomics
     if (n_dev != nullptr) n = min(n, *n_dev);  // count known only on the device (<= the launch bound)
     if (n <= 0) return;
-    const int64_t look_words = (n + kTile - 1) / kTile * kRadix;
+    const int64_t look_words = (n + tile_keys - 1) / tile_keys * kRadix;
     for (int i = threadIdx.x; i < kNW * 4 * kRadix; i += kNT) (&s_hist[0][0][0])[i] = 0;
     __syncthreads();
     const int64_t stride = (int64_t)gridDim.x * kNT;
@@ -99,38 +106,39 @@ __global__ void __launch_bounds__(kNT) k_radix_hist(const float* __restrict__ a,
 // One LSD pass.  MODE 0: keys from the fp32 anchors, values = indices.
 // MODE 1: keys/values from the previous pass.  MODE 2: like 1, and the keys
 // leave as fp32 anchors (last pass).
-template <int MODE>
+template <int MODE, int ITEMS>
 __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__ a, const uint32_t* __restrict__ keys_in,
                                                     const uint32_t* __restrict__ vals_in, uint32_t* __restrict__ keys_out,
                                                     uint32_t* __restrict__ vals_out, int64_t n, const int64_t* n_dev,
                                                     int shift, const uint32_t* __restrict__ hist, uint32_t* counter,
                                                     unsigned long long* look, unsigned long long* look_next,
                                                     int32_t* status) {
+    constexpr int TILE = kNT * ITEMS;
     __shared__ uint32_t s_whist[kNW][kRadix];
-    __shared__ uint32_t s_keys[kTile];
-    __shared__ uint32_t s_vals[kTile];
+    __shared__ uint32_t s_keys[TILE];
+    __shared__ uint32_t s_vals[TILE];
     __shared__ uint32_t s_base[kRadix];   // global destination of the tile's first key per digit
     __shared__ uint32_t s_start[kRadix];  // tile-local start of each digit
     __shared__ uint32_t s_scan[kNW];
     __shared__ int64_t s_tile;
     // during the ranking, the lanes of the current item holding each digit (and a
     // word for rows past n), per warp; the key buffer is free until the placement
-    static_assert(kNW * (kRadix + 1) <= kTile, "peer words fit in the key buffer");
+    static_assert(kNW * (kRadix + 1) <= TILE, "peer words fit in the key buffer");
     uint32_t(*s_peer)[kRadix + 1] = reinterpret_cast<uint32_t(*)[kRadix + 1]>(s_keys);
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     if (n_dev != nullptr) {
         // count known only on the device (<= the launch bound): the first
-        // ceil(n / kTile) CTAs claim one tile each, the others leave at once
+        // ceil(n / TILE) CTAs claim one tile each, the others leave at once
         n = min(n, *n_dev);
-        if ((int64_t)blockIdx.x * kTile >= n) return;
+        if ((int64_t)blockIdx.x * TILE >= n) return;
     }
     if (tid == 0) s_tile = atomicAdd(counter, 1u);
     for (int i = tid; i < kNW * kRadix; i += kNT) (&s_whist[0][0])[i] = 0;
     for (int i = tid; i < kNW * (kRadix + 1); i += kNT) (&s_peer[0][0])[i] = 0;
     __syncthreads();
     const int64_t tile = s_tile;
-    const int64_t base = tile * kTile;
+    const int64_t base = tile * TILE;
     if (base >= n) return;  // the tiles of a smaller device-side count (uniform per CTA)
     look_next[tile * kRadix + tid] = 0ull;  // the pass after next reuses this region
 
@@ -140,10 +148,10 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
 
     // keys now; the values are loaded only when they are placed (fewer live
     // registers: four CTAs per SM)
-    uint32_t key[kItems], rank[kItems];
-    const int64_t wbase = base + (int64_t)w * 32 * kItems;
+    uint32_t key[ITEMS], rank[ITEMS];
+    const int64_t wbase = base + (int64_t)w * 32 * ITEMS;
 #pragma unroll
-    for (int i = 0; i < kItems; ++i) {
+    for (int i = 0; i < ITEMS; ++i) {
         const int64_t idx = wbase + i * 32 + lane;
         if (idx < n) {
             if (MODE == 0)
@@ -160,11 +168,11 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     // of their own), reads the word back, and the lowest of those lanes advances
     // the warp's running count of the digit and clears the word for the next item.
     // rank = running count before the item + the lanes below in the word.
-    // rows of this warp's slice below n (32-bit from here on: a slice holds 32 * kItems)
-    const int wn = (int)max((int64_t)0, min((int64_t)(32 * kItems), n - wbase));
+    // rows of this warp's slice below n (32-bit from here on: a slice holds 32 * ITEMS)
+    const int wn = (int)max((int64_t)0, min((int64_t)(32 * ITEMS), n - wbase));
     const uint32_t my_bit = 1u << lane, lt = lanemask_lt();
 #pragma unroll
-    for (int i = 0; i < kItems; ++i) {
+    for (int i = 0; i < ITEMS; ++i) {
         const bool valid = i * 32 + lane < wn;
         const uint32_t d = valid ? ((key[i] >> shift) & 0xffu) : (uint32_t)kRadix;
         atomicOr(&s_peer[w][d], my_bit);
@@ -198,7 +206,7 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
     __syncthreads();
     // place keys in shared memory in (digit, rank) order
 #pragma unroll
-    for (int i = 0; i < kItems; ++i) {
+    for (int i = 0; i < ITEMS; ++i) {
         if (i * 32 + lane < wn) {
             const int64_t idx = wbase + i * 32 + lane;
             const uint32_t d = (key[i] >> shift) & 0xffu;
@@ -244,7 +252,7 @@ __global__ void __launch_bounds__(kNT, 4) k_radix_pass(const float* __restrict__
         s_base[tid] = gexcl + (uint32_t)excl;
     }
     __syncthreads();
-    const int valid_count = (n - base) < kTile ? (int)(n - base) : kTile;
+    const int valid_count = (n - base) < TILE ? (int)(n - base) : TILE;
     for (int p = tid; p < valid_count; p += kNT) {
         const uint32_t k = s_keys[p];
         const uint32_t d = (k >> shift) & 0xffu;
@@ -574,14 +582,60 @@ cudaError_t launch_place(const uint32_t* perm, const float* v, int64_t n, float*
     return cudaGetLastError();
 }
 
+// Tiles of a sort of n keys at the smallest tile sort_items may choose for it (the
+// lookback regions are sized by this count).
+int64_t sort_max_tiles(int64_t n) {
+    const int tile = n <= kShortMax ? kTileShort : kTile;
+    return (n + tile - 1) / tile;
+}
+
+// Keys per thread of the radix passes.  The tiles run as about ceil(T / slots)
+// rounds of the resident CTAs (four per SM), each round lasting about one tile's
+// keys per thread: when that estimate is at least 10 % lower for the short tiles,
+// a sort of up to kShortMax keys takes them (n = 3 145 728: 819 tiles of 3840 keys
+// are two rounds of 15, 1117 tiles of 2816 two rounds of 11).
+int sort_items(int64_t n, int sms) {
+    if (n > kShortMax) return kItems;
+    const int64_t slots = 4ll * sms;
+    auto rounds = [&](int tile) { return ((n + tile - 1) / tile + slots - 1) / slots; };
+    return 10 * rounds(kTileShort) * kItemsShort <= 9 * rounds(kTile) * kItems ? kItemsShort : kItems;
+}
+
 size_t sort_workspace_bytes(int64_t n) {
-    const int64_t T = (n + kTile - 1) / kTile;
+    const int64_t T = sort_max_tiles(n);
     size_t b = 0;
     b += align_up((size_t)n * 4, 256);            // keys_alt
     b += align_up((size_t)n * 4, 256);            // vals_alt
     b += align_up(4 * kRadix * 4 + 64, 256);      // hist + counters
     b += 2 * align_up((size_t)T * kRadix * 8, 256);  // two lookback regions
     return b;
+}
+
+// The four LSD passes over T tiles of ITEMS keys per thread.
+// pass 0: a -> alt; pass 1: alt -> out; pass 2: out -> alt; pass 3: alt -> out
+template <int ITEMS>
+cudaError_t launch_passes(const float* a, int64_t n, const int64_t* n_dev, int64_t T, uint32_t* keys_alt,
+                          uint32_t* vals_alt, float* a_sorted, uint32_t* perm, const uint32_t* hist,
+                          uint32_t* counters, unsigned long long* const* look, int32_t* status, cudaStream_t stream) {
+    uint32_t* ka = (uint32_t*)a_sorted;
+    const dim3 grid((unsigned)T);
+    LAPLEX_TIMED("radix_pass", stream,
+                 (k_radix_pass<0, ITEMS><<<grid, kNT, 0, stream>>>(a, nullptr, nullptr, keys_alt, vals_alt, n, n_dev, 0,
+                                                                   hist + 0 * kRadix, counters + 0, look[0], look[1],
+                                                                   status)));
+    LAPLEX_TIMED("radix_pass", stream,
+                 (k_radix_pass<1, ITEMS><<<grid, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, n_dev, 8,
+                                                                   hist + 1 * kRadix, counters + 1, look[1], look[0],
+                                                                   status)));
+    LAPLEX_TIMED("radix_pass", stream,
+                 (k_radix_pass<1, ITEMS><<<grid, kNT, 0, stream>>>(nullptr, ka, perm, keys_alt, vals_alt, n, n_dev, 16,
+                                                                   hist + 2 * kRadix, counters + 2, look[0], look[1],
+                                                                   status)));
+    LAPLEX_TIMED("radix_pass", stream,
+                 (k_radix_pass<2, ITEMS><<<grid, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, n_dev, 24,
+                                                                   hist + 3 * kRadix, counters + 3, look[1], look[0],
+                                                                   status)));
+    return cudaGetLastError();
 }
 
 cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* perm, void* ws, int32_t* status,
@@ -599,7 +653,6 @@ cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* pe
                                     sizeof(unsigned long long) * n, stream>>>(a, (int)n, a_sorted, perm, status));
         return cudaGetLastError();
     }
-    const int64_t T = (n + kTile - 1) / kTile;
     char* p = (char*)ws;
     uint32_t* keys_alt = (uint32_t*)p;
     p += align_up((size_t)n * 4, 256);
@@ -610,7 +663,7 @@ cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* pe
     p += align_up(4 * kRadix * 4 + 64, 256);
     unsigned long long* look[2];
     look[0] = (unsigned long long*)p;
-    p += align_up((size_t)T * kRadix * 8, 256);
+    p += align_up((size_t)sort_max_tiles(n) * kRadix * 8, 256);
     look[1] = (unsigned long long*)p;
 
     cudaError_t e = cudaMemsetAsync(hist, 0, 4 * kRadix * 4 + 64, stream);
@@ -618,20 +671,17 @@ cudaError_t launch_sort(const float* a, int64_t n, float* a_sorted, uint32_t* pe
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int items = sort_items(n, sms);
+    const int tile_keys = kNT * items;
     const int64_t want = (n + kNT * 8 - 1) / (kNT * 8);
     const int hblocks = (int)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)sms * 8));
-    LAPLEX_TIMED("radix_hist", stream, k_radix_hist<<<hblocks, kNT, 0, stream>>>(a, n, n_dev, hist, look[0], status));
-    uint32_t* ka = (uint32_t*)a_sorted;
-    // pass 0: a -> alt; pass 1: alt -> out; pass 2: out -> alt; pass 3: alt -> out
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<0><<<(unsigned)T, kNT, 0, stream>>>(a, nullptr, nullptr, keys_alt, vals_alt, n, n_dev, 0,
-                                                     hist + 0 * kRadix, counters + 0, look[0], look[1], status));
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, n_dev, 8,
-                                                     hist + 1 * kRadix, counters + 1, look[1], look[0], status));
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<1><<<(unsigned)T, kNT, 0, stream>>>(nullptr, ka, perm, keys_alt, vals_alt, n, n_dev, 16,
-                                                     hist + 2 * kRadix, counters + 2, look[0], look[1], status));
-    LAPLEX_TIMED("radix_pass", stream, k_radix_pass<2><<<(unsigned)T, kNT, 0, stream>>>(nullptr, keys_alt, vals_alt, ka, perm, n, n_dev, 24,
-                                                     hist + 3 * kRadix, counters + 3, look[1], look[0], status));
-    return cudaGetLastError();
+    LAPLEX_TIMED("radix_hist", stream,
+                 k_radix_hist<<<hblocks, kNT, 0, stream>>>(a, n, n_dev, tile_keys, hist, look[0], status));
+    const int64_t T = (n + tile_keys - 1) / tile_keys;
+    return items == kItemsShort ? launch_passes<kItemsShort>(a, n, n_dev, T, keys_alt, vals_alt, a_sorted, perm, hist,
+                                                            counters, look, status, stream)
+                                : launch_passes<kItems>(a, n, n_dev, T, keys_alt, vals_alt, a_sorted, perm, hist,
+                                                       counters, look, status, stream);
 }
 
 }  // namespace laplex
