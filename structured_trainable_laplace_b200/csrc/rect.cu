@@ -7,7 +7,7 @@
 // is one scan over the merged sorted sequence of O and I: the state just left
 // of an output o is the prefix over the inputs q <= o, the state right of it the
 // suffix over q > o, and out(o) = prefix + suffix.  It is evaluated in whichever
-// of two ways keeps the lookback scan on the SMALLER side:
+// of two ways keeps the scan on the SMALLER side:
 //   expand (|I| <= |O|): scan the inputs over sorted I (prefix P and suffix S per
 //       input row), then every output reads the states of its two neighbours in
 //       I:  out(o) = exp(q_(m'-1) - o) P_(m'-1) + exp(o - q_(m')) S_(m'),
@@ -20,14 +20,20 @@
 // 2B scan channels (cos part, then sin part) per B input channels.
 //
 // Kernels:
-//   k_side_right / k_side_left  bounded decoupled-lookback scan over the small
-//       side (inputs: gathered rows x phase weights, or fp64 interval sums),
-//       writing per-row states (P, S) or parts (strict L, strict R, full).
+//   k_side_totals / k_side_apply  scan over the small side of up to 1024 tiles
+//       with no wait between CTAs (tile totals, then per tile direct weighted
+//       sums of the other tiles' totals and the tile's evaluation); inputs:
+//       gathered rows x phase weights, or fp64 interval sums; outputs: per-row
+//       states (P, S) or parts (strict L, strict R, full).
+//   k_side_right / k_side_left  the same scan for larger small sides, by bounded
+//       decoupled lookback.
 //   k_large  one streaming pass over the large side: interval sums into fp64
 //       bins (reduce), neighbour lookups (expand), and the fused anchor / phase
 //       gradients of that side.
 //   k_finish  per small-side row: combine the cos/sin parts into outputs and
 //       gradients.
+//   k_gram_mid_sorted / k_gram_mid2  the middle of the Gram apply and backward
+//       (D w, D u, gD) between its two rectangular products.
 #include "laplex_internal.h"
 #include "pipeline.cuh"
 
